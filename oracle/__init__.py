@@ -1,0 +1,261 @@
+"""CPU oracle for the Fathom per-query read-depth top-k key scan.
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package.  The CUDA
+library never imports or links it, and it imports nothing from the CUDA
+library.  The arithmetic lives in ``fathom_oracle.c`` (plain C, fp64 scores);
+this module compiles it with gcc and marshals numpy arrays.
+
+Parity unpinned: ``recall`` (a quality number; the pages print none).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fathom_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_fathom_oracle.so")
+_lib = None
+
+OK, ERR_ARG, ERR_NONFINITE = 0, 1, 3
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fused multiply-add, IEEE float)."""
+    if (force or not os.path.exists(_LIB_PATH)
+            or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off",
+                               "-fno-fast-math", "-fPIC", "-shared", "-o", tmp,
+                               _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int64
+        sig = {
+            "fo_quantize": ([P, I, I, I, P, P, P], ctypes.c_int),
+            "fo_pack_planes": ([P, I, I, I, I, P], ctypes.c_int),
+            "fo_unpack_planes": ([P, I, I, I, I, P], ctypes.c_int),
+            "fo_channel_stats": ([P, I, I, I, P, P, P, P], ctypes.c_int),
+            "fo_importance": ([P, P, I, P], ctypes.c_int),
+            "fo_plan_greedy": ([P, I, I, P], ctypes.c_int),
+            "fo_fixed_plan": ([P, I, I, P], ctypes.c_int),
+            "fo_union": ([P, I, I, P], None),
+            "fo_plan_bytes": ([P, I, I], ctypes.c_uint64),
+            "fo_score_planes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
+            "fo_score_codes": ([P, P, P, P, P, I, I, P], ctypes.c_int),
+            "fo_score_abs_planes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
+            "fo_exact_scores": ([P, P, I, I, P], None),
+            "fo_topk": ([P, I, I, P, P], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise ValueError(f"oracle {what} failed with code {rc}")
+
+
+def n_words_for(n: int) -> int:
+    """Words per plane: keys rounded up to 128 (16-byte plane rows)."""
+    return ((n + 127) // 128) * 4
+
+
+# ---------------------------------------------------------------- storage side
+def quantize(keys: np.ndarray):
+    """keys float32 [H][n][d] -> (mn [H][d], scale [H][d], codes uint8 [H][d][n])."""
+    keys = np.ascontiguousarray(keys, dtype=np.float32)
+    H, n, d = keys.shape
+    mn = np.empty((H, d), np.float32)
+    scale = np.empty((H, d), np.float32)
+    codes = np.empty((H, d, n), np.uint8)
+    _check(_load().fo_quantize(_p(keys), H, n, d, _p(mn), _p(scale), _p(codes)), "quantize")
+    return mn, scale, codes
+
+
+def pack_planes(codes: np.ndarray, n_words: Optional[int] = None) -> np.ndarray:
+    """codes uint8 [H][d][n] -> planes uint32 [H][d][4][n_words]."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    H, d, n = codes.shape
+    n_words = n_words_for(n) if n_words is None else n_words
+    planes = np.empty((H, d, 4, n_words), np.uint32)
+    _check(_load().fo_pack_planes(_p(codes), H, n, d, n_words, _p(planes)), "pack_planes")
+    return planes
+
+
+def unpack_planes(planes: np.ndarray, n: int) -> np.ndarray:
+    planes = np.ascontiguousarray(planes, dtype=np.uint32)
+    H, d, _, n_words = planes.shape
+    codes = np.empty((H, d, n), np.uint8)
+    _check(_load().fo_unpack_planes(_p(planes), H, n, d, n_words, _p(codes)), "unpack_planes")
+    return codes
+
+
+def channel_stats(codes: np.ndarray, scale: np.ndarray):
+    """-> (S1 int64 [H][d], S2 int64 [H][d], sigma2 float32 [H][d])."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    H, d, n = codes.shape
+    s1 = np.empty((H, d), np.int64)
+    s2 = np.empty((H, d), np.int64)
+    sigma2 = np.empty((H, d), np.float32)
+    _check(_load().fo_channel_stats(_p(codes), H, n, d, _p(scale), _p(s1), _p(s2),
+                                    _p(sigma2)), "channel_stats")
+    return s1, s2, sigma2
+
+
+# ------------------------------------------------------------------- read side
+def importance(q_bf16: np.ndarray, sigma2: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    s2 = np.ascontiguousarray(sigma2, dtype=np.float32)
+    d = q.shape[-1]
+    w = np.empty(d, np.float32)
+    _check(_load().fo_importance(_p(q), _p(s2), d, _p(w)), "importance")
+    return w
+
+
+def plan_greedy(w: np.ndarray, B: int) -> np.ndarray:
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    t = np.empty(w.shape[0], np.uint8)
+    _check(_load().fo_plan_greedy(_p(w), w.shape[0], int(B), _p(t)), "plan_greedy")
+    return t
+
+
+def fixed_plan(q_bf16: np.ndarray, r: int) -> np.ndarray:
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    t = np.empty(q.shape[0], np.uint8)
+    _check(_load().fo_fixed_plan(_p(q), q.shape[0], int(r), _p(t)), "fixed_plan")
+    return t
+
+
+def union(t_group: np.ndarray) -> np.ndarray:
+    t = np.ascontiguousarray(t_group, dtype=np.uint8)
+    G, d = t.shape
+    T = np.empty(d, np.uint8)
+    _load().fo_union(_p(t), G, d, _p(T))
+    return T
+
+
+def plan_bytes(t: np.ndarray, n_words: int) -> int:
+    t = np.ascontiguousarray(t, dtype=np.uint8)
+    return int(_load().fo_plan_bytes(_p(t), t.shape[0], int(n_words)))
+
+
+def score_planes(planes_h, mn_h, scale_h, q_bf16, t, n: int) -> np.ndarray:
+    planes_h = np.ascontiguousarray(planes_h, dtype=np.uint32)
+    d, _, n_words = planes_h.shape
+    mn_h = np.ascontiguousarray(mn_h, np.float32)
+    scale_h = np.ascontiguousarray(scale_h, np.float32)
+    q = np.ascontiguousarray(q_bf16, np.uint16)
+    t = np.ascontiguousarray(t, np.uint8)
+    s = np.empty(n, np.float64)
+    _check(_load().fo_score_planes(_p(planes_h), _p(mn_h), _p(scale_h), _p(q), _p(t),
+                                   d, n, n_words, _p(s)), "score_planes")
+    return s
+
+
+def score_abs_planes(planes_h, mn_h, scale_h, q_bf16, t, n: int) -> np.ndarray:
+    planes_h = np.ascontiguousarray(planes_h, dtype=np.uint32)
+    d, _, n_words = planes_h.shape
+    a = np.empty(n, np.float64)
+    _check(_load().fo_score_abs_planes(
+        _p(planes_h), _p(np.ascontiguousarray(mn_h, np.float32)),
+        _p(np.ascontiguousarray(scale_h, np.float32)),
+        _p(np.ascontiguousarray(q_bf16, np.uint16)), _p(np.ascontiguousarray(t, np.uint8)),
+        d, n, n_words, _p(a)), "score_abs_planes")
+    return a
+
+
+def score_codes(codes_h, mn_h, scale_h, q_bf16, t) -> np.ndarray:
+    codes_h = np.ascontiguousarray(codes_h, dtype=np.uint8)
+    d, n = codes_h.shape
+    s = np.empty(n, np.float64)
+    _check(_load().fo_score_codes(
+        _p(codes_h), _p(np.ascontiguousarray(mn_h, np.float32)),
+        _p(np.ascontiguousarray(scale_h, np.float32)),
+        _p(np.ascontiguousarray(q_bf16, np.uint16)), _p(np.ascontiguousarray(t, np.uint8)),
+        d, n, _p(s)), "score_codes")
+    return s
+
+
+def exact_scores(keys_h: np.ndarray, q_bf16: np.ndarray) -> np.ndarray:
+    keys_h = np.ascontiguousarray(keys_h, dtype=np.float32)
+    n, d = keys_h.shape
+    s = np.empty(n, np.float64)
+    _load().fo_exact_scores(_p(keys_h), _p(np.ascontiguousarray(q_bf16, np.uint16)), n, d, _p(s))
+    return s
+
+
+def topk(s: np.ndarray, k: int):
+    """-> (idx int32 [k], score float64 [k]) by (score desc, index asc)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    idx = np.empty(k, np.int32)
+    top = np.empty(k, np.float64)
+    _check(_load().fo_topk(_p(s), s.shape[0], int(k), _p(idx), _p(top)), "topk")
+    return idx, top
+
+
+def recall(selected, reference) -> float:
+    """|S intersect S*| / |S*|.  Parity unpinned: a quality number only."""
+    ref = set(int(x) for x in np.asarray(reference).ravel())
+    got = set(int(x) for x in np.asarray(selected).ravel())
+    return len(ref & got) / max(1, len(ref))
+
+
+# --------------------------------------------------------------- whole pipeline
+def build_index(keys: np.ndarray) -> Dict[str, np.ndarray]:
+    """Storage side for one session: quantise, pack, channel statistics."""
+    mn, scale, codes = quantize(keys)
+    n = keys.shape[1]
+    planes = pack_planes(codes)
+    s1, s2, sigma2 = channel_stats(codes, scale)
+    return dict(mn=mn, scale=scale, codes=codes, planes=planes, s1=s1, s2=s2,
+                sigma2=sigma2, n=n, n_words=planes.shape[-1])
+
+
+def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
+                 fixed_r: Optional[int] = None):
+    """-> (t uint8 [Q][d], T uint8 [H][d], bytes uint64 [Q+H])."""
+    H, d = index["mn"].shape
+    Q = H * group
+    t = np.empty((Q, d), np.uint8)
+    for q in range(Q):
+        h = q // group
+        if fixed_r is None:
+            t[q] = plan_greedy(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
+        else:
+            t[q] = fixed_plan(q_bf16[q], fixed_r)
+    T = np.stack([union(t[h * group:(h + 1) * group]) for h in range(H)])
+    nb = np.array([plan_bytes(t[q], index["n_words"]) for q in range(Q)]
+                  + [plan_bytes(T[h], index["n_words"]) for h in range(H)], np.uint64)
+    return t, T, nb
+
+
+def scan_query(index, q_bf16_row, t_row, h: int, k: int):
+    """Score one query against KV head h and select its top-k.
+    -> (idx [k], top scores [k], all scores [n], abs sums [n])."""
+    n = index["n"]
+    s = score_planes(index["planes"][h], index["mn"][h], index["scale"][h], q_bf16_row, t_row, n)
+    idx, top = topk(s, k)
+    return idx, top, s

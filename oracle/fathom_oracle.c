@@ -1,0 +1,386 @@
+/*
+ * fathom_oracle.c -- plain, slow CPU oracle for the Fathom per-query
+ * read-depth top-k key scan.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this file.  It shares no code, header, table or
+ * helper with the CUDA library, and the CUDA library never calls it.
+ *
+ * Source: "Fathom：面向卸载 KV 缓存稀疏解码的每查询读取深度" (the
+ * papers.ananclaw.com explainer of arXiv 2609.17652), section 核心方法
+ * (method): 存储侧 (storage side) and 读侧 (read side), and its simplified
+ * reverse water-filling walk; plus the method summary on the proomt.com page
+ * ("Fathom: Per-Query Read Depth for Sparse Decoding over Offloaded KV
+ * Caches", Summary).  Every choice the pages leave open is a stated reading:
+ *
+ *   quantiser   per (head, channel) asymmetric min/max over all n keys,
+ *               scale = (max-min)/15, code = clamp(floor((k-min)/scale+0.5),
+ *               0, 15) in float32 round-to-nearest with no fused ops; a
+ *               constant channel gets scale 0 and code 0.
+ *   planes      bit p of a code (p = 0 least significant, as on the page)
+ *               is stored in slot 3-p, so reading slots 0..t-1 reads the
+ *               t most significant bits ("the first t planes are the t-bit
+ *               quantiser" only holds MSB-first).
+ *   variance    sigma^2 = population variance of the dequantised 4-bit keys,
+ *               from exact integer sums of codes.
+ *   importance  w_c = (q_c*q_c)*sigma^2_c in float32, q widened from bf16.
+ *   plan        channels in order of (w descending, channel ascending); each
+ *               takes min(4, remaining budget) bits until the budget is
+ *               spent, so channels of zero importance still take leftovers.
+ *   score       reading t bits gives u = code >> (4-t); the key is rebuilt
+ *               at the middle of that coarse bin and dotted with q in fp64.
+ *   top-k       score descending, ties to the lower key index.
+ *
+ * Parity unpinned: recall against the exact top-k is a quality number only;
+ * the pages print no recall to check it against.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared -lm.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define FO_OK 0
+#define FO_ERR_ARG 1
+#define FO_ERR_NONFINITE 3
+
+#define FO_BITS 4   /* 4-bit K cache (storage side) */
+#define FO_LEVELS 15
+
+/* ------------------------------------------------------------------ */
+/* Storage side: 4-bit quantisation of each channel.                    */
+/* ------------------------------------------------------------------ */
+
+/* keys: float32 [H][n][d] (token-major, as a K cache holds them).
+ * Outputs: mn, scale float32 [H][d]; codes uint8 [H][d][n] (channel-major). */
+int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d,
+                float *mn, float *scale, uint8_t *codes)
+{
+    if (H <= 0 || n <= 0 || d <= 0) return FO_ERR_ARG;
+    for (int64_t h = 0; h < H; ++h) {
+        const float *kh = keys + h * n * d;
+        for (int64_t c = 0; c < d; ++c) {
+            float lo = kh[c], hi = kh[c];
+            for (int64_t j = 0; j < n; ++j) {
+                float x = kh[j * d + c];
+                if (!isfinite(x)) return FO_ERR_NONFINITE;
+                if (x < lo) lo = x;
+                if (x > hi) hi = x;
+            }
+            uint8_t *out = codes + (h * d + c) * n;
+            mn[h * d + c] = lo;
+            if (hi == lo) {
+                scale[h * d + c] = 0.0f;
+                memset(out, 0, (size_t)n);
+                continue;
+            }
+            float sc = (hi - lo) / (float)FO_LEVELS;
+            scale[h * d + c] = sc;
+            for (int64_t j = 0; j < n; ++j) {
+                float diff = kh[j * d + c] - lo;
+                float ratio = diff / sc;
+                float shifted = ratio + 0.5f;
+                float level = floorf(shifted);
+                int v = (int)level;
+                if (v < 0) v = 0;
+                if (v > FO_LEVELS) v = FO_LEVELS;
+                out[j] = (uint8_t)v;
+            }
+        }
+    }
+    return FO_OK;
+}
+
+/* Channel-major bit planes: planes uint32 [H][d][4][n_words]; slot s holds
+ * bit (3-s) of the code; bit i of word w belongs to key 32*w+i; words past
+ * the last key are zero.  n_words >= ceil(n/32). */
+int fo_pack_planes(const uint8_t *codes, int64_t H, int64_t n, int64_t d,
+                   int64_t n_words, uint32_t *planes)
+{
+    if (n_words * 32 < n) return FO_ERR_ARG;
+    memset(planes, 0, (size_t)(H * d * FO_BITS * n_words) * sizeof(uint32_t));
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t c = 0; c < d; ++c) {
+            const uint8_t *cc = codes + (h * d + c) * n;
+            uint32_t *pc = planes + (h * d + c) * FO_BITS * n_words;
+            for (int64_t j = 0; j < n; ++j)
+                for (int p = 0; p < FO_BITS; ++p)
+                    if ((cc[j] >> p) & 1u)
+                        pc[(FO_BITS - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
+        }
+    return FO_OK;
+}
+
+/* Inverse of fo_pack_planes (reads all four slots). */
+int fo_unpack_planes(const uint32_t *planes, int64_t H, int64_t n, int64_t d,
+                     int64_t n_words, uint8_t *codes)
+{
+    if (n_words * 32 < n) return FO_ERR_ARG;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t c = 0; c < d; ++c) {
+            const uint32_t *pc = planes + (h * d + c) * FO_BITS * n_words;
+            uint8_t *cc = codes + (h * d + c) * n;
+            for (int64_t j = 0; j < n; ++j) {
+                int v = 0;
+                for (int p = 0; p < FO_BITS; ++p)
+                    v |= (int)((pc[(FO_BITS - 1 - p) * n_words + j / 32] >> (j % 32)) & 1u) << p;
+                cc[j] = (uint8_t)v;
+            }
+        }
+    return FO_OK;
+}
+
+/* Per-channel statistics of the stored 4-bit keys: S1 = sum code,
+ * S2 = sum code^2 (exact int64) and the population variance of the
+ * dequantised keys mn + scale*code:
+ *   sigma^2 = scale^2 * (n*S2 - S1^2) / n^2,
+ * evaluated as (double)(scale*scale) * ((double)num / ((double)n*n)),
+ * then rounded to float32. */
+int fo_channel_stats(const uint8_t *codes, int64_t H, int64_t n, int64_t d,
+                     const float *scale, int64_t *s1, int64_t *s2, float *sigma2)
+{
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t c = 0; c < d; ++c) {
+            const uint8_t *cc = codes + (h * d + c) * n;
+            int64_t a = 0, b = 0;
+            for (int64_t j = 0; j < n; ++j) {
+                a += cc[j];
+                b += (int64_t)cc[j] * cc[j];
+            }
+            s1[h * d + c] = a;
+            s2[h * d + c] = b;
+            int64_t num = n * b - a * a;
+            double sc = (double)scale[h * d + c];
+            double sc2 = sc * sc;
+            double nn = (double)n * (double)n;
+            double frac = (double)num / nn;
+            sigma2[h * d + c] = (float)(sc2 * frac);
+        }
+    return FO_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Read side: importance, reverse water-filling, union, bytes.          */
+/* ------------------------------------------------------------------ */
+
+static float bf16_value(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* w_c = (q_c * q_c) * sigma^2_c, float32. */
+int fo_importance(const uint16_t *q_bf16, const float *sigma2, int64_t d, float *w)
+{
+    for (int64_t c = 0; c < d; ++c) {
+        float qc = bf16_value(q_bf16[c]);
+        float qq = qc * qc;
+        float wc = qq * sigma2[c];
+        if (!isfinite(wc)) return FO_ERR_NONFINITE;
+        w[c] = wc;
+    }
+    return FO_OK;
+}
+
+typedef struct { float key; int64_t c; } fo_rank_item;
+
+/* (key descending, channel ascending) */
+static int fo_rank_cmp(const void *pa, const void *pb)
+{
+    const fo_rank_item *a = (const fo_rank_item *)pa, *b = (const fo_rank_item *)pb;
+    if (a->key > b->key) return -1;
+    if (a->key < b->key) return 1;
+    return (a->c < b->c) ? -1 : (a->c > b->c);
+}
+
+/* Reverse water-filling: visit channels from the most important down and
+ * give each min(4, remaining) bits; once the budget is gone the rest get 0.
+ * B must lie in [0, 4d]. */
+int fo_plan_greedy(const float *w, int64_t d, int64_t B, uint8_t *t)
+{
+    if (B < 0 || B > FO_BITS * d) return FO_ERR_ARG;
+    fo_rank_item *order = (fo_rank_item *)malloc((size_t)d * sizeof *order);
+    if (!order) return FO_ERR_ARG;
+    for (int64_t c = 0; c < d; ++c) {
+        if (!isfinite(w[c])) { free(order); return FO_ERR_NONFINITE; }
+        order[c].key = w[c];
+        order[c].c = c;
+    }
+    qsort(order, (size_t)d, sizeof *order, fo_rank_cmp);
+    int64_t left = B;
+    for (int64_t i = 0; i < d; ++i) {
+        int64_t take = 0;
+        if (left > 0) {
+            take = left < FO_BITS ? left : FO_BITS;
+            left -= take;
+        }
+        t[order[i].c] = (uint8_t)take;
+    }
+    free(order);
+    return FO_OK;
+}
+
+/* Fixed-width baseline plan: the r channels of largest |q_c| (ties to the
+ * lower channel) are read at all 4 bits, the rest not at all. */
+int fo_fixed_plan(const uint16_t *q_bf16, int64_t d, int64_t r, uint8_t *t)
+{
+    if (r < 0 || r > d) return FO_ERR_ARG;
+    fo_rank_item *order = (fo_rank_item *)malloc((size_t)d * sizeof *order);
+    if (!order) return FO_ERR_ARG;
+    for (int64_t c = 0; c < d; ++c) {
+        order[c].key = fabsf(bf16_value(q_bf16[c]));
+        order[c].c = c;
+    }
+    qsort(order, (size_t)d, sizeof *order, fo_rank_cmp);
+    for (int64_t i = 0; i < d; ++i) t[order[i].c] = (uint8_t)(i < r ? FO_BITS : 0);
+    free(order);
+    return FO_OK;
+}
+
+/* GQA union: planes are nested MSB-first, so a KV head that serves G query
+ * heads reads T_c = max_g t_c^(g) planes of channel c. */
+void fo_union(const uint8_t *t, int64_t G, int64_t d, uint8_t *T)
+{
+    for (int64_t c = 0; c < d; ++c) {
+        uint8_t m = 0;
+        for (int64_t g = 0; g < G; ++g)
+            if (t[g * d + c] > m) m = t[g * d + c];
+        T[c] = m;
+    }
+}
+
+/* Bytes read = sum_c t_c * bytes_per_plane, one plane being n_words*4 bytes. */
+uint64_t fo_plan_bytes(const uint8_t *t, int64_t d, int64_t n_words)
+{
+    uint64_t total = 0;
+    for (int64_t c = 0; c < d; ++c) total += (uint64_t)t[c] * (uint64_t)n_words * 4u;
+    return total;
+}
+
+/* ------------------------------------------------------------------ */
+/* Scoring from the selected planes.                                    */
+/* ------------------------------------------------------------------ */
+
+/* A key read at t bits with value u = code >> (4-t) lies in the coarse bin
+ * of fine levels [u*2^(4-t), u*2^(4-t) + 2^(4-t) - 1]; it is rebuilt at the
+ * bin's middle.  t = 4 gives mn + scale*code; t = 0 gives mn + 7.5*scale. */
+static double fo_coarse_midpoint(float mn, float scale, int t, int u)
+{
+    int width = 1 << (FO_BITS - t);
+    double level = (double)(width * u) + (double)(width - 1) / 2.0;
+    return (double)mn + (double)scale * level;
+}
+
+/* Score every key of one KV head for one query from its plan t:
+ * planes_h uint32 [d][4][n_words]; mn, scale [d]; q bf16 [d]; t [d];
+ * s float64 [n].  Reads slots 0..t_c-1 of each channel (MSB first). */
+int fo_score_planes(const uint32_t *planes_h, const float *mn, const float *scale,
+                    const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
+                    int64_t n_words, double *s)
+{
+    for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) {
+            int tc = t[c];
+            if (tc < 0 || tc > FO_BITS) return FO_ERR_ARG;
+            int u = 0;
+            for (int slot = 0; slot < tc; ++slot) {
+                uint32_t word = planes_h[(c * FO_BITS + slot) * n_words + j / 32];
+                u = (u << 1) | (int)((word >> (j % 32)) & 1u);
+            }
+            acc += (double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u);
+        }
+        s[j] = acc;
+    }
+    return FO_OK;
+}
+
+/* The same score from the 4-bit codes by re-quantising to t bits:
+ * codes_h uint8 [d][n]. */
+int fo_score_codes(const uint8_t *codes_h, const float *mn, const float *scale,
+                   const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
+                   double *s)
+{
+    for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) {
+            int tc = t[c];
+            if (tc < 0 || tc > FO_BITS) return FO_ERR_ARG;
+            int u = codes_h[c * n + j] >> (FO_BITS - tc);
+            acc += (double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u);
+        }
+        s[j] = acc;
+    }
+    return FO_OK;
+}
+
+/* sum_c |q_c * khat_c,j| for the same reading: the scale a score's
+ * rounding error is measured against. */
+int fo_score_abs_planes(const uint32_t *planes_h, const float *mn, const float *scale,
+                        const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
+                        int64_t n_words, double *a)
+{
+    for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) {
+            int tc = t[c];
+            int u = 0;
+            for (int slot = 0; slot < tc; ++slot) {
+                uint32_t word = planes_h[(c * FO_BITS + slot) * n_words + j / 32];
+                u = (u << 1) | (int)((word >> (j % 32)) & 1u);
+            }
+            acc += fabs((double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u));
+        }
+        a[j] = acc;
+    }
+    return FO_OK;
+}
+
+/* Exact score against the full-precision keys: keys_h float32 [n][d]. */
+void fo_exact_scores(const float *keys_h, const uint16_t *q_bf16, int64_t n, int64_t d,
+                     double *s)
+{
+    for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            acc += (double)bf16_value(q_bf16[c]) * (double)keys_h[j * d + c];
+        s[j] = acc;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Top-k: a full sort.                                                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct { double s; int64_t j; } fo_score_item;
+
+static int fo_score_cmp(const void *pa, const void *pb)
+{
+    const fo_score_item *a = (const fo_score_item *)pa, *b = (const fo_score_item *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+/* The k keys of largest score, in order (score descending, index ascending). */
+int fo_topk(const double *s, int64_t n, int64_t k, int32_t *idx, double *top_s)
+{
+    if (k < 1 || k > n) return FO_ERR_ARG;
+    fo_score_item *items = (fo_score_item *)malloc((size_t)n * sizeof *items);
+    if (!items) return FO_ERR_ARG;
+    for (int64_t j = 0; j < n; ++j) {
+        if (!isfinite(s[j])) { free(items); return FO_ERR_NONFINITE; }
+        items[j].s = s[j];
+        items[j].j = j;
+    }
+    qsort(items, (size_t)n, sizeof *items, fo_score_cmp);
+    for (int64_t i = 0; i < k; ++i) {
+        idx[i] = (int32_t)items[i].j;
+        if (top_s) top_s[i] = items[i].s;
+    }
+    free(items);
+    return FO_OK;
+}

@@ -1,0 +1,69 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check
+that the pins catch every one of them."""
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+from tests.conftest import read_golden
+
+MUTATIONS = {
+    "dropped_half_in_rounding": ("float shifted = ratio + 0.5f;", "float shifted = ratio;"),
+    "scale_over_16": ("(hi - lo) / (float)FO_LEVELS", "(hi - lo) / 16.0f"),
+    "lsb_first_planes": ("pc[(FO_BITS - 1 - p) * n_words + j / 32] |=", "pc[p * n_words + j / 32] |="),
+    "variance_missing_square": ("double sc2 = sc * sc;", "double sc2 = sc;"),
+    "importance_uses_abs_q": ("float qq = qc * qc;", "float qq = fabsf(qc);"),
+    "plan_ascending_importance": ("if (a->key > b->key) return -1;\n    if (a->key < b->key) return 1;",
+                                  "if (a->key < b->key) return -1;\n    if (a->key > b->key) return 1;"),
+    "plan_cap_3_bits": ("take = left < FO_BITS ? left : FO_BITS;", "take = left < 3 ? left : 3;"),
+    "bin_low_edge_not_middle": ("(double)(width - 1) / 2.0", "0.0"),
+    "planes_read_lsb_first": ("u = (u << 1) | (int)((word >> (j % 32)) & 1u);",
+                              "u = u | (int)(((word >> (j % 32)) & 1u) << slot);"),
+    "topk_ties_to_higher_index": ("return (a->j < b->j) ? -1 : (a->j > b->j);",
+                                  "return (a->j > b->j) ? -1 : (a->j < b->j);"),
+    "union_takes_min": ("if (t[g * d + c] > m) m = t[g * d + c];", "if (g == 0) m = t[g * d + c];"),
+}
+
+PIN_TESTS = [
+    lambda: pins.test_quantize_hand_worked(read_golden),
+    pins.test_quantize_error_bound_and_extremes,
+    pins.test_sigma2_matches_variance_of_dequantised_keys,
+    lambda: pins.test_plane_layout_hand_worked(read_golden),
+    pins.test_importance_values,
+    lambda: pins.test_plan_hand_worked(read_golden),
+    lambda: pins.test_fixed_plan_hand_worked(read_golden),
+    pins.test_union_and_bytes,
+    lambda: pins.test_coarse_bin_midpoint_hand_worked(read_golden),
+    pins.test_reading_t_planes_equals_requantising_to_t_bits,
+    lambda: pins.test_topk_hand_worked(read_golden),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    old, new = MUTATIONS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found"
+    tmp = tempfile.mkdtemp()
+    try:
+        csrc = os.path.join(tmp, "mut.c")
+        so = os.path.join(tmp, "mut.so")
+        open(csrc, "w").write(src.replace(old, new, 1))   # first occurrence
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC",
+                               "-shared", "-o", so, csrc, "-lm"])
+        monkeypatch.setattr(oracle, "_LIB_PATH", so)
+        monkeypatch.setattr(oracle, "build", lambda force=False: so)
+        monkeypatch.setattr(oracle, "_lib", None)
+        caught = 0
+        for fn in PIN_TESTS:
+            try:
+                fn()
+            except (AssertionError, ValueError):
+                caught += 1
+        assert caught >= 1, f"no pin caught mutation {name}"
+    finally:
+        shutil.rmtree(tmp)

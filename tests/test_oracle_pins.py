@@ -1,0 +1,339 @@
+"""Pins for the CPU oracle: hand-worked examples, brute force, closed forms and
+invariants that the explainer's method section fixes.  CPU only."""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def _floats(v):
+    return np.array([float(x) for x in v], dtype=np.float64)
+
+
+def _ints(v):
+    return np.array([int(x, 0) for x in v], dtype=np.int64)
+
+
+# ----------------------------------------------------------------- quantiser
+def test_quantize_hand_worked(golden):
+    g = golden("quantize_worked.txt")
+    keys = np.stack([_floats(g["keys_channel_A"]), _floats(g["keys_channel_B"]),
+                     _floats(g["keys_channel_C"])], axis=1).astype(np.float32)[None]
+    mn, scale, codes = oracle.quantize(keys)
+    assert np.array_equal(mn[0], _floats(g["mn"]).astype(np.float32))
+    assert np.array_equal(scale[0], _floats(g["scale"]).astype(np.float32))
+    for c, name in enumerate("ABC"):
+        assert np.array_equal(codes[0, c], _ints(g["codes_" + name])), name
+    s1, s2, sigma2 = oracle.channel_stats(codes, scale)
+    assert np.array_equal(s1[0], _ints(g["S1"]))
+    assert np.array_equal(s2[0], _ints(g["S2"]))
+    assert np.array_equal(sigma2[0], _floats(g["sigma2"]).astype(np.float32))
+
+
+def test_quantize_error_bound_and_extremes():
+    """Round-to-nearest over 16 evenly spaced levels: each key is within half a
+    step of its level; the channel min maps to 0 and the max to 15."""
+    ses = synth.make_session(3, 2, 1, 1000, 16)
+    mn, scale, codes = oracle.quantize(ses.keys)
+    k = ses.keys.transpose(0, 2, 1).astype(np.float64)          # [H][d][n]
+    deq = mn[..., None].astype(np.float64) + scale[..., None].astype(np.float64) * codes
+    err = np.abs(deq - k)
+    assert np.all(err <= scale[..., None] * (0.5 + 1e-5) + 1e-6)
+    assert np.all(codes <= 15)
+    jmin = np.argmin(k, axis=2)
+    jmax = np.argmax(k, axis=2)
+    assert np.all(np.take_along_axis(codes, jmin[..., None], 2) == 0)
+    assert np.all(np.take_along_axis(codes, jmax[..., None], 2) == 15)
+    # every level is used by a Gaussian channel of 1000 keys except possibly a few
+    assert len(np.unique(codes[0, 0])) >= 10
+
+
+def test_sigma2_matches_variance_of_dequantised_keys():
+    """sigma^2 is the population variance of mn + scale*code: compare with
+    numpy's two-pass variance (a different algorithm) in fp64."""
+    ses = synth.make_session(5, 2, 1, 3000, 16)
+    mn, scale, codes = oracle.quantize(ses.keys)
+    _, _, sigma2 = oracle.channel_stats(codes, scale)
+    deq = mn[..., None].astype(np.float64) + scale[..., None].astype(np.float64) * codes
+    ref = deq.var(axis=2)
+    assert np.allclose(sigma2, ref, rtol=1e-6, atol=0)
+    # and it estimates the generating variance (4-bit noise adds scale^2/12)
+    ratio = sigma2 / (ses.sigma ** 2)
+    assert np.all((ratio > 0.8) & (ratio < 1.25))
+
+
+# -------------------------------------------------------------------- planes
+def test_plane_layout_hand_worked(golden):
+    g = golden("plane_layout.txt")
+    n = int(g["n"][0])
+    codes = np.zeros((1, 1, n), np.uint8)
+    codes[0, 0, 0] = int(g["code_key_0"][0])
+    codes[0, 0, 37] = int(g["code_key_37"][0])
+    codes[0, 0, 63] = int(g["code_key_63"][0])
+    planes = oracle.pack_planes(codes)
+    assert planes.shape == (1, 1, 4, 4)
+    for s, name in enumerate(["slot0_bit3", "slot1_bit2", "slot2_bit1", "slot3_bit0"]):
+        assert np.array_equal(planes[0, 0, s], _ints(g[name]).astype(np.uint32)), name
+
+
+@pytest.mark.parametrize("n", [1, 31, 32, 33, 127, 128, 129, 1000])
+def test_planes_round_trip_and_padding(n):
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 16, size=(2, 3, n), dtype=np.uint8)
+    planes = oracle.pack_planes(codes)
+    n_w = oracle.n_words_for(n)
+    assert planes.shape == (2, 3, 4, n_w) and n_w % 4 == 0
+    assert np.array_equal(oracle.unpack_planes(planes, n), codes)
+    # keys past n carry no bits
+    full = oracle.unpack_planes(planes, n_w * 32)
+    assert not full[..., n:].any()
+
+
+def test_index_is_the_4bit_cache_size():
+    """No extra copy: the planes of a head hold exactly n*d/2 bytes (4 bits per
+    key per channel) when n is a multiple of 128."""
+    ses = synth.make_session(1, 2, 1, 4096, 16)
+    ix = oracle.build_index(ses.keys)
+    assert ix["planes"].nbytes == 2 * 4096 * 128 // 2
+
+
+# ---------------------------------------------------------------- importance
+def test_importance_values():
+    sigma2 = np.array([3.0, 3.0, 5.0, 0.0], np.float32)
+    q = synth.f32_to_bf16_bits(np.array([2.0, -2.0, 0.0, 7.0], np.float32))
+    w = oracle.importance(q, sigma2)
+    assert np.array_equal(w, np.array([12.0, 12.0, 0.0, 0.0], np.float32))
+
+
+def test_importance_rejects_nonfinite():
+    q = synth.f32_to_bf16_bits(np.array([1e30, 1.0], np.float32))
+    with pytest.raises(ValueError):
+        oracle.importance(q, np.array([1e30, 1.0], np.float32))
+
+
+# ---------------------------------------------------------------------- plan
+def test_plan_hand_worked(golden):
+    g = golden("plan_worked.txt")
+    for case in ("case1", "case2", "case3", "case4"):
+        w = _floats(g[case + "_w"]).astype(np.float32)
+        t = oracle.plan_greedy(w, int(g[case + "_B"][0]))
+        assert np.array_equal(t, _ints(g[case + "_t"])), case
+    t1 = oracle.plan_greedy(_floats(g["case1_w"]).astype(np.float32), 18)
+    n = int(g["case1_n"][0])
+    assert oracle.plan_bytes(t1, oracle.n_words_for(n)) == int(g["case1_bytes"][0])
+
+
+def _brute_force_best(w, B):
+    d = len(w)
+    best = -1.0
+    w64 = w.astype(np.float64)
+    for alloc in itertools.product(range(5), repeat=d):
+        if sum(alloc) <= B:
+            v = float(np.dot(w64, alloc))
+            best = max(best, v)
+    return best
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 5])
+def test_plan_is_optimal_by_brute_force_small(d):
+    rng = np.random.default_rng(100 + d)
+    for trial in range(6):
+        w = rng.lognormal(0, 1, size=d).astype(np.float32)
+        if trial == 0:
+            w[:] = 1.0                      # all tied
+        if trial == 1 and d > 1:
+            w[0] = 0.0                      # zero importance
+        for B in range(0, 4 * d + 1):
+            t = oracle.plan_greedy(w, B)
+            assert int(t.sum()) == min(B, 4 * d)
+            assert np.all(t <= 4)
+            got = float(np.dot(w.astype(np.float64), t))
+            assert got == pytest.approx(_brute_force_best(w, B), rel=1e-12, abs=0)
+
+
+def test_plan_is_optimal_by_brute_force_d8():
+    """All 5^8 = 390625 allocations of head_dim 8, vectorised."""
+    d = 8
+    allocs = np.array(list(itertools.product(range(5), repeat=d)), dtype=np.int64)
+    sums = allocs.sum(axis=1)
+    rng = np.random.default_rng(8)
+    for trial in range(4):
+        w = rng.lognormal(0, 1.5, size=d).astype(np.float32)
+        vals = allocs @ w.astype(np.float64)
+        for B in (0, 1, 3, 4, 7, 8, 13, 18, 20, 31, 32):
+            t = oracle.plan_greedy(w, B)
+            best = vals[sums <= B].max()
+            assert float(np.dot(w.astype(np.float64), t)) == pytest.approx(best, rel=1e-12)
+            assert int(t.sum()) == min(B, 32)
+
+
+def test_plan_tiny_budget_reads_two_channels():
+    """Intuition example 3: at 8 bits/key or less at most 2 channels are read."""
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        w = rng.lognormal(0, 1, size=128).astype(np.float32)
+        for B in range(0, 9):
+            t = oracle.plan_greedy(w, B)
+            assert (t > 0).sum() == (B + 3) // 4 <= 2
+
+
+def test_plan_rejects_bad_budget():
+    w = np.ones(4, np.float32)
+    for B in (-1, 17):
+        with pytest.raises(ValueError):
+            oracle.plan_greedy(w, B)
+
+
+# ------------------------------------------------------------- fixed plans
+def test_fixed_plan_hand_worked(golden):
+    g = golden("fixed_plan_worked.txt")
+    q = synth.f32_to_bf16_bits(_floats(g["q"]).astype(np.float32))
+    assert np.array_equal(oracle.fixed_plan(q, int(g["r"][0])), _ints(g["t"]))
+    assert np.array_equal(oracle.fixed_plan(q, int(g["r1"][0])), _ints(g["r1_t"]))
+
+
+def test_fixed_plan_widths():
+    """Fixed 136-bit and 68-bit scans: 34 / 17 channels at 4 bits."""
+    q = synth.make_session(0, 1, 1, 128, 16).q_bf16[0]
+    for r, bits in ((34, 136), (17, 68)):
+        t = oracle.fixed_plan(q, r)
+        assert int(t.sum()) == bits and set(np.unique(t)) <= {0, 4}
+        absq = np.abs(synth.bf16_bits_to_f32(q))
+        assert absq[t == 4].min() >= absq[t == 0].max()
+
+
+# --------------------------------------------------------- union and bytes
+def test_union_and_bytes():
+    ses = synth.make_session(11, 2, 4, 4096, 92)
+    ix = oracle.build_index(ses.keys)
+    t, T, nb = oracle.plan_session(ix, ses.q_bf16, ses.budgets, 4)
+    n = 4096
+    Q = 8
+    for q in range(Q):
+        assert int(nb[q]) == 92 * n // 8          # bytes = B * n / 8
+    for h in range(2):
+        grp = t[4 * h:4 * h + 4]
+        assert np.array_equal(T[h], grp.max(axis=0))
+        assert int(nb[Q + h]) == int(T[h].sum()) * n // 8
+        assert max(nb[4 * h:4 * h + 4]) <= nb[Q + h] <= sum(nb[4 * h:4 * h + 4])
+
+
+# -------------------------------------------------------------------- score
+def test_coarse_bin_midpoint_hand_worked(golden):
+    g = golden("midpoint_worked.txt")
+    code = int(g["code"][0])
+    one = synth.f32_to_bf16_bits(np.array([1.0], np.float32))
+    for t, kh in zip(_ints(g["t"]), _floats(g["khat"])):
+        codes = np.array([[[code]]], np.uint8)
+        planes = oracle.pack_planes(codes)
+        s = oracle.score_planes(planes[0], np.zeros(1, np.float32), np.ones(1, np.float32),
+                                one, np.array([t], np.uint8), 1)
+        assert s[0] == kh
+
+
+def test_coarse_bin_is_mean_of_its_fine_levels():
+    """Reading t bits rebuilds a key at the mean of the 2^(4-t) fine levels of
+    its coarse bin (all bins are equally wide)."""
+    mn, sc = np.float32(-1.25), np.float32(0.375)
+    one = synth.f32_to_bf16_bits(np.array([1.0], np.float32))
+    codes = np.arange(16, dtype=np.uint8)[None, None, :]
+    planes = oracle.pack_planes(codes)
+    for t in range(5):
+        s = oracle.score_planes(planes[0], np.array([mn]), np.array([sc]), one,
+                                np.array([t], np.uint8), 16)
+        width = 1 << (4 - t)
+        for code in range(16):
+            lo = (code // width) * width
+            levels = float(mn) + float(sc) * np.arange(lo, lo + width, dtype=np.float64)
+            assert s[code] == pytest.approx(levels.mean(), rel=1e-15, abs=1e-15)
+
+
+def test_full_depth_score_is_the_4bit_dot_product():
+    """t_c = 4 for every channel: the score is the exact dot product with the
+    dequantised 4-bit keys (computed here by a numpy fp64 matmul)."""
+    ses = synth.make_session(2, 2, 2, 700, 512)
+    ix = oracle.build_index(ses.keys)
+    t4 = np.full(128, 4, np.uint8)
+    for h in range(2):
+        deq = ix["mn"][h][:, None].astype(np.float64) + \
+            ix["scale"][h][:, None].astype(np.float64) * ix["codes"][h]   # [d][n]
+        for g in range(2):
+            q = ses.q_bf16[2 * h + g]
+            s = oracle.score_planes(ix["planes"][h], ix["mn"][h], ix["scale"][h], q, t4, 700)
+            ref = synth.bf16_bits_to_f32(q).astype(np.float64) @ deq
+            mag = np.abs(synth.bf16_bits_to_f32(q).astype(np.float64)) @ np.abs(deq)
+            assert np.all(np.abs(s - ref) <= 1e-13 * mag)
+
+
+def test_reading_t_planes_equals_requantising_to_t_bits():
+    """Storage-side invariant: the score from the first t_c planes equals the
+    score from the codes re-quantised to t_c bits (code >> (4 - t_c)); the two
+    oracle routes agree bit for bit, for greedy and arbitrary plans."""
+    ses = synth.make_session(9, 1, 3, 1500, 50)
+    ix = oracle.build_index(ses.keys)
+    rng = np.random.default_rng(0)
+    plans = [oracle.plan_greedy(oracle.importance(ses.q_bf16[g], ix["sigma2"][0]), B)
+             for g, B in ((0, 18), (1, 92), (2, 136))]
+    plans.append(rng.integers(0, 5, size=128).astype(np.uint8))
+    for t in plans:
+        for g in range(3):
+            a = oracle.score_planes(ix["planes"][0], ix["mn"][0], ix["scale"][0],
+                                    ses.q_bf16[g], t, 1500)
+            b = oracle.score_codes(ix["codes"][0], ix["mn"][0], ix["scale"][0],
+                                   ses.q_bf16[g], t)
+            assert np.array_equal(a, b)
+
+
+def test_zero_depth_score_is_constant():
+    ses = synth.make_session(4, 1, 1, 300, 0)
+    ix = oracle.build_index(ses.keys)
+    s = oracle.score_planes(ix["planes"][0], ix["mn"][0], ix["scale"][0], ses.q_bf16[0],
+                            np.zeros(128, np.uint8), 300)
+    qf = synth.bf16_bits_to_f32(ses.q_bf16[0]).astype(np.float64)
+    const = qf @ (ix["mn"][0].astype(np.float64) + 7.5 * ix["scale"][0].astype(np.float64))
+    assert np.allclose(s, const, rtol=1e-13, atol=0)
+    assert np.all(s == s[0])
+
+
+def test_exact_scores_match_matmul():
+    ses = synth.make_session(6, 1, 1, 500, 0)
+    s = oracle.exact_scores(ses.keys[0], ses.q_bf16[0])
+    ref = ses.keys[0].astype(np.float64) @ synth.bf16_bits_to_f32(ses.q_bf16[0]).astype(np.float64)
+    assert np.allclose(s, ref, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------- top-k
+def test_topk_hand_worked(golden):
+    g = golden("topk_worked.txt")
+    s = _floats(g["scores"])
+    assert np.array_equal(oracle.topk(s, 3)[0], _ints(g["k3_idx"]))
+    assert np.array_equal(oracle.topk(s, 4)[0], _ints(g["k4_idx"]))
+
+
+def test_topk_matches_full_sort_with_ties():
+    rng = np.random.default_rng(1)
+    s = rng.integers(0, 50, size=5000).astype(np.float64)      # many ties
+    for k in (1, 7, 64, 2048, 5000):
+        idx, top = oracle.topk(s, k)
+        ref = np.lexsort((np.arange(5000), -s))[:k]
+        assert np.array_equal(idx, ref)
+        assert np.array_equal(top, s[ref])
+
+
+def test_recall_bounds():
+    assert oracle.recall([1, 2, 3], [3, 2, 1]) == 1.0
+    assert oracle.recall([1, 2, 3], [4, 5, 6]) == 0.0
+    assert oracle.recall([1, 2, 9], [1, 2, 3, 4]) == 0.5
+
+
+def test_tiny_workload_planted_keys_rank_high():
+    """Sanity (reported, not a pin): the 16 planted keys close to the query
+    land in the top-64 at 64 bits/key."""
+    ses = synth.tiny_4k()
+    ix = oracle.build_index(ses.keys)
+    t, T, nb = oracle.plan_session(ix, ses.q_bf16, ses.budgets, 1)
+    idx, _, _ = oracle.scan_query(ix, ses.q_bf16[0], t[0], 0, 64)
+    assert len(set(ses.planted[0].tolist()) & set(idx.tolist())) >= 12
