@@ -1,0 +1,296 @@
+// C ABI of the Fathom sm_100a library: argument validation, residency
+// resolution, workspace accounting, device status and instrumentation.
+// The operations themselves are documented in include/fathom.h.
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace fathom {
+
+// First device-side error since the last fathom_last_device_status() call
+// (one word per device: a module-scope __device__ variable).
+__device__ int g_device_status;
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+std::mutex g_mu;
+int *g_status_ptr[64] = {nullptr};
+struct EventPair {
+    cudaEvent_t begin, end;
+};
+std::vector<EventPair> g_recorded;   // profiled scan launches not read yet
+std::vector<EventPair> g_free_events;
+}  // namespace
+
+int *device_status_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+}  // namespace fathom
+
+using namespace fathom;
+
+namespace {
+
+fathom_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FATHOM_OK : FATHOM_ERR_CUDA; }
+
+bool index_shape_ok(const fathom_index *ix)
+{
+    if (!ix) return false;
+    if (ix->n_kv_heads < 1 || ix->group < 1 || ix->group > kMaxGroup) return false;
+    if (ix->head_dim < 32 || ix->head_dim > kMaxHeadDim || ix->head_dim % 32) return false;
+    if (ix->n_keys < 1 || ix->n_words < 4 || ix->n_words % 4) return false;
+    if ((long long)ix->n_words * 32 < (long long)ix->n_keys) return false;
+    if (ix->residency != FATHOM_RES_DEVICE && ix->residency != FATHOM_RES_HOST_MAPPED) return false;
+    // global plane row indices must fit in 32 bits
+    if ((long long)ix->n_kv_heads * ix->head_dim * kBits >= (1ll << 31)) return false;
+    return true;
+}
+
+// Resolve the planes pointer to a device address for the residency mode.
+fathom_status resolve_planes(const fathom_index *ix, uint32_t **out)
+{
+    // plane rows are copied 16 bytes at a time
+    if (!ix->planes || (reinterpret_cast<uintptr_t>(ix->planes) & 15u)) return FATHOM_ERR_INVALID_ARG;
+    if (ix->residency == FATHOM_RES_HOST_MAPPED) {
+        void *dptr = nullptr;
+        if (cudaHostGetDevicePointer(&dptr, ix->planes, 0) != cudaSuccess || !dptr) {
+            cudaGetLastError();
+            return FATHOM_ERR_INVALID_ARG;
+        }
+        *out = static_cast<uint32_t *>(dptr);
+        return FATHOM_OK;
+    }
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, ix->planes) != cudaSuccess) {
+        cudaGetLastError();
+        return FATHOM_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return FATHOM_ERR_INVALID_ARG;
+    *out = ix->planes;
+    return FATHOM_OK;
+}
+
+bool stats_ok(const fathom_index *ix)
+{
+    return ix->mn && ix->scale && ix->sigma2 && ix->sum_code && ix->sum_code2;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+EventPair take_event_pair()
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_free_events.empty()) {
+        EventPair p = g_free_events.back();
+        g_free_events.pop_back();
+        return p;
+    }
+    EventPair p{};
+    cudaEventCreate(&p.begin);
+    cudaEventCreate(&p.end);
+    return p;
+}
+
+fathom_status scan_common(const fathom_index *sessions, int n_sessions,
+                          const uint16_t *const *q, const uint8_t *const *t,
+                          const uint8_t *const *tu, int32_t k, int32_t *const *out_idx,
+                          float *const *out_score, void *ws, size_t ws_bytes, uint32_t flags,
+                          cudaStream_t stream)
+{
+    if (!sessions || n_sessions < 1 || n_sessions > kMaxSessions) return FATHOM_ERR_INVALID_ARG;
+    if (!q || !t || !tu || !out_idx || !out_score) return FATHOM_ERR_INVALID_ARG;
+    if (flags & ~(FATHOM_SCAN_FORCE_EXACT | FATHOM_SCAN_PROFILE)) return FATHOM_ERR_INVALID_ARG;
+    if (k < 1 || k > kMaxK) return FATHOM_ERR_INVALID_ARG;
+    std::vector<fathom_index> resolved(n_sessions);
+    std::vector<ScanSessionArgs> args(n_sessions);
+    for (int s = 0; s < n_sessions; ++s) {
+        const fathom_index *ix = &sessions[s];
+        if (!index_shape_ok(ix) || !ix->mn || !ix->scale) return FATHOM_ERR_INVALID_ARG;
+        if (ix->head_dim != sessions[0].head_dim || ix->group != sessions[0].group)
+            return FATHOM_ERR_INVALID_ARG;
+        if (k > ix->n_keys) return FATHOM_ERR_INVALID_ARG;
+        if (!q[s] || !t[s] || !tu[s] || !out_idx[s] || !out_score[s]) return FATHOM_ERR_INVALID_ARG;
+        resolved[s] = *ix;
+        fathom_status st = resolve_planes(ix, &resolved[s].planes);
+        if (st != FATHOM_OK) return st;
+        args[s] = ScanSessionArgs{&resolved[s], q[s], t[s], tu[s], out_idx[s], out_score[s]};
+    }
+    const size_t need = scan_workspace_bytes(sessions, n_sessions, k);
+    if (!ws || !aligned16(ws) || ws_bytes < need) return FATHOM_ERR_WORKSPACE;
+
+    ScanProfileHook hook{false, nullptr, nullptr, false};
+    EventPair ev{};
+    if (flags & FATHOM_SCAN_PROFILE) {
+        ev = take_event_pair();
+        hook = ScanProfileHook{true, ev.begin, ev.end, false};
+    }
+    cudaError_t e = launch_scan(args.data(), n_sessions, k, ws, ws_bytes, flags, stream, &hook);
+    if (flags & FATHOM_SCAN_PROFILE) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (hook.recorded)
+            g_recorded.push_back(ev);
+        else
+            g_free_events.push_back(ev);
+    }
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t fathom_n_words(int32_t n_keys)
+{
+    if (n_keys < 1) return 0;
+    return (int32_t)(((long long)n_keys + 127) / 128 * 4);
+}
+
+const char *fathom_status_str(fathom_status status)
+{
+    switch (status) {
+    case FATHOM_OK: return "ok";
+    case FATHOM_ERR_INVALID_ARG: return "invalid argument";
+    case FATHOM_ERR_CUDA: return "CUDA error";
+    case FATHOM_ERR_NONFINITE: return "non-finite key, query or importance";
+    case FATHOM_ERR_TIMEOUT: return "device wait timed out";
+    case FATHOM_ERR_WORKSPACE: return "workspace missing or too small";
+    case FATHOM_ERR_UNIMPLEMENTED: return "unimplemented";
+    }
+    return "unknown status";
+}
+
+size_t fathom_pack_workspace_bytes(const fathom_index *index)
+{
+    if (!index_shape_ok(index)) return 0;
+    return (size_t)8 * index->n_kv_heads * index->head_dim;
+}
+
+fathom_status fathom_pack_keys(const float *keys, const fathom_index *index, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!keys || !index_shape_ok(index) || !stats_ok(index)) return FATHOM_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fathom_pack_workspace_bytes(index))
+        return FATHOM_ERR_WORKSPACE;
+    fathom_index ix = *index;
+    fathom_status st = resolve_planes(index, &ix.planes);
+    if (st != FATHOM_OK) return st;
+    return cuda_status(launch_pack(keys, ix, static_cast<uint32_t *>(workspace), stream));
+}
+
+fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
+                          const int32_t *budget, uint8_t *t, uint8_t *t_union, uint64_t *bytes,
+                          cudaStream_t stream)
+{
+    if (!index_shape_ok(index) || !index->sigma2) return FATHOM_ERR_INVALID_ARG;
+    if (!q_bf16 || !budget || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
+    return cuda_status(launch_plan(*index, q_bf16, budget, 0, false, t, t_union, bytes, stream));
+}
+
+fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf16, int32_t r,
+                                uint8_t *t, uint8_t *t_union, uint64_t *bytes,
+                                cudaStream_t stream)
+{
+    if (!index_shape_ok(index)) return FATHOM_ERR_INVALID_ARG;
+    if (!q_bf16 || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
+    if (r < 0 || r > index->head_dim) return FATHOM_ERR_INVALID_ARG;
+    return cuda_status(launch_plan(*index, q_bf16, nullptr, r, true, t, t_union, bytes, stream));
+}
+
+size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k)
+{
+    if (!index_shape_ok(index) || k < 1 || k > kMaxK) return 0;
+    return scan_workspace_bytes(index, 1, k);
+}
+
+fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,
+                               const uint8_t *t, const uint8_t *t_union, int32_t k,
+                               int32_t *out_idx, float *out_score, void *workspace,
+                               size_t workspace_bytes, uint32_t flags, cudaStream_t stream)
+{
+    return scan_common(index, 1, &q_bf16, &t, &t_union, k, &out_idx, &out_score, workspace,
+                       workspace_bytes, flags, stream);
+}
+
+size_t fathom_scan_batched_workspace_bytes(const fathom_index *sessions, int32_t n_sessions,
+                                           int32_t k)
+{
+    if (!sessions || n_sessions < 1 || n_sessions > kMaxSessions || k < 1 || k > kMaxK) return 0;
+    for (int s = 0; s < n_sessions; ++s)
+        if (!index_shape_ok(&sessions[s])) return 0;
+    return scan_workspace_bytes(sessions, n_sessions, k);
+}
+
+fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_sessions,
+                                       const uint16_t *const *q_bf16, const uint8_t *const *t,
+                                       const uint8_t *const *t_union, int32_t k,
+                                       int32_t *const *out_idx, float *const *out_score,
+                                       void *workspace, size_t workspace_bytes, uint32_t flags,
+                                       cudaStream_t stream)
+{
+    return scan_common(sessions, n_sessions, q_bf16, t, t_union, k, out_idx, out_score,
+                       workspace, workspace_bytes, flags, stream);
+}
+
+fathom_status fathom_last_device_status(cudaStream_t stream)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  stream) != cudaSuccess)
+        return FATHOM_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FATHOM_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                stream) != cudaSuccess)
+        return FATHOM_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FATHOM_ERR_CUDA;
+    return static_cast<fathom_status>(v);
+}
+
+uint64_t fathom_launch_count(void) { return (uint64_t)g_launches.load(); }
+
+fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_launches)
+{
+    std::vector<EventPair> recs;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        recs.swap(g_recorded);
+    }
+    double total = 0.0;
+    fathom_status st = FATHOM_OK;
+    for (const EventPair &p : recs) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(p.end) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, p.begin, p.end) != cudaSuccess) {
+            cudaGetLastError();
+            st = FATHOM_ERR_CUDA;
+            continue;
+        }
+        total += ms;
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        g_free_events.insert(g_free_events.end(), recs.begin(), recs.end());
+    }
+    if (scan_kernel_ms) *scan_kernel_ms = total;
+    if (scan_kernel_launches) *scan_kernel_launches = recs.size();
+    return st;
+}
+
+}  // extern "C"

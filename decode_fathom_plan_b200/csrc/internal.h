@@ -1,0 +1,50 @@
+// Host-side interfaces between the C-ABI layer and the kernel launchers
+// (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fathom.h"
+
+namespace fathom {
+
+// Address of this device's status word (a __device__ int).
+int *device_status_ptr();
+// Count one kernel launch (for fathom_launch_count).
+void note_launch(int n = 1);
+
+// ---- pack.cu
+cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_minmax,
+                        cudaStream_t stream);
+
+// ---- plan.cu
+cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
+                        int32_t fixed_r, bool fixed, uint8_t *t, uint8_t *t_union,
+                        uint64_t *bytes, cudaStream_t stream);
+
+// ---- scan.cu
+struct ScanSessionArgs {
+    const fathom_index *ix;
+    const uint16_t *q;
+    const uint8_t *t;
+    const uint8_t *t_union;
+    int32_t *out_idx;
+    float *out_score;
+};
+
+// Workspace bytes for a batch of sessions (single call = batch of one).
+size_t scan_workspace_bytes(const fathom_index *sessions, int n_sessions, int k);
+
+// Profiling events around the main scan kernel (FATHOM_SCAN_PROFILE).
+struct ScanProfileHook {
+    bool enabled;
+    cudaEvent_t begin, end;
+    bool recorded;   // set when the main scan kernel was launched and timed
+};
+
+cudaError_t launch_scan(const ScanSessionArgs *sessions, int n_sessions, int k,
+                        void *ws, size_t ws_bytes, uint32_t flags, cudaStream_t stream,
+                        ScanProfileHook *hook);
+
+}  // namespace fathom

@@ -1,0 +1,216 @@
+/*
+ * fathom.h -- C ABI of the B200 (sm_100a) Fathom per-query read-depth
+ * top-k key scan.
+ *
+ * The method: "Fathom：面向卸载 KV 缓存稀疏解码的每查询读取深度" (the
+ * papers.ananclaw.com explainer of arXiv 2609.17652), section 核心方法:
+ *   storage side (存储侧) -- the K cache is quantised to 4 bits and stored
+ *     channel-major as bit planes; the first t planes of a channel are its
+ *     t-bit quantiser;
+ *   read side (读侧) -- each query spends a per-key bit budget B over the
+ *     channels by reverse water-filling on the importance w_c, up to 4 bits
+ *     per channel, letting unimportant channels take 0 bits; bytes read =
+ *     sum_c t_c * bytes_per_plane;
+ * and section 解决什么真问题: every decode step ranks n keys and keeps the
+ * top-k.
+ *
+ * Conventions for every call:
+ *   - All buffers are owned by the caller.  The library allocates no device
+ *     or host memory; scratch space is a caller-supplied workspace sized by
+ *     the matching *_workspace_bytes call (16-byte aligned).
+ *   - Calls are stream-ordered and asynchronous: they validate what the host
+ *     can see, enqueue kernels on `stream` and return.  Argument errors are
+ *     returned at once and enqueue nothing.  Errors that only the device can
+ *     see (a non-finite key or importance, a budget out of range) are
+ *     recorded in a per-device status word read by
+ *     fathom_last_device_status().
+ *   - Layouts (H = KV heads, G = query heads per KV head, Q = H*G,
+ *     d = head_dim, n = keys, n_words = words per plane):
+ *       keys      float32 [H][n][d]            (token-major, as a K cache)
+ *       planes    uint32  [H][d][4][n_words]   slot s holds bit 3-s of the
+ *                 4-bit code (slot 0 = most significant); bit i of word w
+ *                 belongs to key 32*w+i; words past the last key are zero
+ *       mn, scale, sigma2  float32 [H][d]; sum_code, sum_code2 int64 [H][d]
+ *       q         bfloat16 bits (uint16) [Q][d], query q served by KV head
+ *                 q / G
+ *       budget    int32 [Q] bits per key, 0 <= B <= 4*d
+ *       t         uint8 [Q][d] bits read per channel; t_union uint8 [H][d]
+ *       bytes     uint64 [Q + H]: per query, then per KV head (union)
+ *       out_idx   int32 [Q][k], out_score float32 [Q][k]: the k keys of
+ *                 largest score, ordered by score descending and then key
+ *                 index ascending
+ *   - head_dim is a multiple of 32 and at most 256; G is 1..8;
+ *     n_words is a multiple of 4 (16-byte plane rows) with 32*n_words >= n;
+ *     1 <= k <= min(n, 4096).
+ */
+#ifndef FATHOM_H
+#define FATHOM_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FATHOM_OK = 0,
+    FATHOM_ERR_INVALID_ARG = 1,   /* bad pointer, size or layout            */
+    FATHOM_ERR_CUDA = 2,          /* a CUDA runtime call failed             */
+    FATHOM_ERR_NONFINITE = 3,     /* non-finite key, query or importance    */
+    FATHOM_ERR_TIMEOUT = 4,       /* a bounded device wait ran out          */
+    FATHOM_ERR_WORKSPACE = 5,     /* workspace missing or too small         */
+    FATHOM_ERR_UNIMPLEMENTED = 6  /* a mode this build does not provide     */
+} fathom_status;
+
+/* Where the planes live.  DEVICE: HBM.  HOST_MAPPED: pinned host memory
+ * that the scan reads zero-copy over the host link (the explainer's
+ * setting: the 4-bit K index is offloaded to host memory). */
+typedef enum {
+    FATHOM_RES_DEVICE = 0,
+    FATHOM_RES_HOST_MAPPED = 1
+} fathom_residency;
+
+/* A packed K index of one session (one layer).  Plain descriptor; every
+ * pointer is caller-owned.  planes is a device pointer (DEVICE) or a pinned,
+ * device-mapped host pointer (HOST_MAPPED); the statistics are device
+ * pointers. */
+typedef struct {
+    int32_t n_kv_heads;       /* H */
+    int32_t group;            /* G query heads per KV head */
+    int32_t head_dim;         /* d */
+    int32_t n_keys;           /* n */
+    int32_t n_words;          /* words per plane */
+    int32_t residency;        /* fathom_residency */
+    uint32_t *planes;         /* [H][d][4][n_words] */
+    float *mn;                /* [H][d] channel minimum */
+    float *scale;             /* [H][d] (max - min) / 15, 0 if max == min */
+    float *sigma2;            /* [H][d] variance of the dequantised keys */
+    int64_t *sum_code;        /* [H][d] sum of codes */
+    int64_t *sum_code2;       /* [H][d] sum of squared codes */
+} fathom_index;
+
+/* Scan flags. */
+#define FATHOM_SCAN_DEFAULT 0u
+/* Skip the sampled candidate threshold and select every query's top-k with
+ * the exact multi-pass radix select (the path the fast path falls back to). */
+#define FATHOM_SCAN_FORCE_EXACT 1u
+/* Record CUDA events around the main scan kernel (benchmarking only). */
+#define FATHOM_SCAN_PROFILE 2u
+
+/* Words per plane for n keys: n rounded up to 128 keys, i.e. 16-byte rows. */
+int32_t fathom_n_words(int32_t n_keys);
+
+/* Human-readable name of a status. */
+const char *fathom_status_str(fathom_status status);
+
+/* ---------------------------------------------------------------------- */
+/* Storage side.                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes fathom_pack_keys needs for `index` (8*H*d). */
+size_t fathom_pack_workspace_bytes(const fathom_index *index);
+
+/* Quantise keys to 4 bits per (KV head, channel) and write the bit planes
+ * and channel statistics into `index` (explainer, 核心方法 / 存储侧).
+ * Per (h, c) over all n keys: mn = min, scale = (max-min)/15 (0 if the
+ * channel is constant), code = clamp(floor((k-mn)/scale + 0.5), 0, 15) in
+ * IEEE float32; sum_code, sum_code2 exact; sigma2 = scale^2*(n*S2-S1^2)/n^2
+ * in fp64 rounded to float32 (the variance of the stored 4-bit keys, the
+ * importance weight the read side uses).
+ * keys: device float32 [H][n][d].  Every output array of `index` is
+ * written; planes may be a mapped host pointer (written zero-copy).
+ * A non-finite key sets FATHOM_ERR_NONFINITE in the device status. */
+fathom_status fathom_pack_keys(const float *keys, const fathom_index *index,
+                               void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Read side: plans.                                                      */
+/* ---------------------------------------------------------------------- */
+
+/* Reverse water-filling (explainer, 核心方法 / 读侧): for each query,
+ * w_c = (q_c*q_c)*sigma2_c in float32; channels are visited by w descending
+ * (ties to the lower channel) and each takes min(4, remaining budget) bits,
+ * so t_c = min(4, max(0, B - 4*rank_c)) and sum_c t_c = B.  Also writes the
+ * GQA union t_union[h][c] = max over the G queries of KV head h, and the
+ * bytes each query (and each KV head's union) reads: sum_c t_c * 4*n_words.
+ * q_bf16, budget, t, t_union, bytes: device pointers.
+ * A budget outside [0, 4d] sets FATHOM_ERR_INVALID_ARG in the device status
+ * (that query reads nothing); a non-finite w sets FATHOM_ERR_NONFINITE. */
+fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
+                          const int32_t *budget, uint8_t *t, uint8_t *t_union,
+                          uint64_t *bytes, cudaStream_t stream);
+
+/* Fixed-width baseline plan (the 136-bit / 68-bit key scans the explainer
+ * compares against): the r channels of largest |q_c| (ties to the lower
+ * channel) are read at 4 bits, the rest at 0.  Same outputs as
+ * fathom_plan.  0 <= r <= d. */
+fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf16,
+                                int32_t r, uint8_t *t, uint8_t *t_union,
+                                uint64_t *bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Read side: scan and select.                                            */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes fathom_scan_topk needs for `index` and k. */
+size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k);
+
+/* Score every key for every query from only the planes its plan selects,
+ * and select the top-k (explainer, 核心方法 and 解决什么真问题).
+ * Each KV head reads the union of its G queries' planes once; query g's
+ * score of key j is
+ *   s_gj = sum_c q_gc * (mn_c + scale_c*(2^(4-t)*u + (2^(4-t)-1)/2)),
+ *   t = t_gc, u = code_cj >> (4-t)
+ * (the key rebuilt at the middle of its coarse t-bit bin), accumulated in
+ * float32.  Outputs the k keys of largest s, ties to the lower index.
+ * q_bf16, t, t_union, out_idx, out_score, workspace: device pointers.
+ * flags: FATHOM_SCAN_* bits. */
+fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,
+                               const uint8_t *t, const uint8_t *t_union, int32_t k,
+                               int32_t *out_idx, float *out_score,
+                               void *workspace, size_t workspace_bytes,
+                               uint32_t flags, cudaStream_t stream);
+
+/* Workspace bytes fathom_scan_topk_batched needs. */
+size_t fathom_scan_batched_workspace_bytes(const fathom_index *sessions,
+                                           int32_t n_sessions, int32_t k);
+
+/* The same scan over many independent sessions (concurrent agent sessions
+ * of the explainer's setting) in one launch per phase.  sessions: host
+ * array of n_sessions (1..64) descriptors sharing head_dim and group;
+ * q_bf16, t, t_union, out_idx, out_score: host arrays of n_sessions device
+ * pointers laid out as for fathom_scan_topk. */
+fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_sessions,
+                                       const uint16_t *const *q_bf16,
+                                       const uint8_t *const *t,
+                                       const uint8_t *const *t_union, int32_t k,
+                                       int32_t *const *out_idx, float *const *out_score,
+                                       void *workspace, size_t workspace_bytes,
+                                       uint32_t flags, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Status and instrumentation.                                            */
+/* ---------------------------------------------------------------------- */
+
+/* Synchronise `stream`, return the first device-side error recorded on the
+ * current device since the last call (FATHOM_OK if none) and clear it.
+ * A failed synchronisation returns FATHOM_ERR_CUDA. */
+fathom_status fathom_last_device_status(cudaStream_t stream);
+
+/* Kernels this library has launched in this process. */
+uint64_t fathom_launch_count(void);
+
+/* Time of the main scan kernel, recorded with CUDA events by calls made
+ * with FATHOM_SCAN_PROFILE: synchronises on the recorded events and
+ * returns the summed milliseconds and the number of launches timed, then
+ * forgets them.  Not thread-safe; benchmarking only. */
+fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATHOM_H */

@@ -1,0 +1,102 @@
+"""The C-ABI library loads and exports every symbol include/fathom.h declares;
+host-side validation rejects bad arguments before touching the GPU.  CPU only:
+no call here reaches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_fathom_plan_b200 as fp
+from decode_fathom_plan_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "fathom.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fathom_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build()
+    return fp.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(fp.EXPORTED)
+
+
+def test_n_words_rounds_to_16_byte_rows(lib):
+    for n, w in ((1, 4), (32, 4), (128, 4), (129, 8), (4096, 128), (131072, 4096),
+                 (1 << 20, 32768)):
+        assert fp.fathom_n_words(n) == w
+    assert fp.fathom_n_words(0) == 0
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert fp.status_str(code)
+    assert "workspace" in fp.status_str(fp.FATHOM_ERR_WORKSPACE)
+
+
+def _desc(H=2, G=4, d=128, n=4096, residency=0, fake=0x1000):
+    return fp.fathom_index(H, G, d, n, fp.fathom_n_words(n), residency,
+                           fake, fake, fake, fake, fake, fake)
+
+
+def test_workspace_sizes_are_host_computable(lib):
+    ix = _desc()
+    assert fp.fathom_pack_workspace_bytes(ix) == 8 * 2 * 128
+    ws = fp.fathom_scan_workspace_bytes(ix, 64)
+    assert ws > 0 and ws % 256 == 0
+    # larger k needs a larger candidate buffer
+    big = _desc(n=1 << 20)
+    assert fp.fathom_scan_workspace_bytes(big, 2048) > fp.fathom_scan_workspace_bytes(big, 64)
+    assert fp.fathom_scan_batched_workspace_bytes([ix, big], 64) == \
+        fp.fathom_scan_workspace_bytes(ix, 64) + fp.fathom_scan_workspace_bytes(big, 64)
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 48), ("head_dim", 512), ("group", 9),
+                                         ("group", 0), ("n_words", 6), ("n_keys", 0),
+                                         ("residency", 7)])
+def test_bad_index_shapes_are_rejected(lib, field, value):
+    ix = _desc()
+    setattr(ix, field, value)
+    assert fp.fathom_scan_workspace_bytes(ix, 64) == 0
+    assert fp.fathom_pack_workspace_bytes(ix) == 0
+    rc = lib.fathom_plan(ctypes.byref(ix), 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0)
+    assert rc == fp.FATHOM_ERR_INVALID_ARG
+
+
+def test_null_pointers_are_rejected(lib):
+    ix = _desc()
+    assert lib.fathom_plan(ctypes.byref(ix), 0, 0x1000, 0x1000, 0x1000, 0x1000, 0) == \
+        fp.FATHOM_ERR_INVALID_ARG
+    assert lib.fathom_fixed_plan(ctypes.byref(ix), 0x1000, 200, 0x1000, 0x1000, 0x1000, 0) == \
+        fp.FATHOM_ERR_INVALID_ARG
+    assert lib.fathom_scan_topk(ctypes.byref(ix), 0, 0x1000, 0x1000, 64, 0x1000, 0x1000,
+                                0x1000, 1 << 30, 0, 0) == fp.FATHOM_ERR_INVALID_ARG
+    assert lib.fathom_pack_keys(0, ctypes.byref(ix), 0x1000, 1 << 20, 0) == \
+        fp.FATHOM_ERR_INVALID_ARG
+
+
+def test_bad_k_and_flags_are_rejected(lib):
+    ix = _desc(n=100)
+    for k in (0, 101, 5000):
+        assert lib.fathom_scan_topk(ctypes.byref(ix), 0x1000, 0x1000, 0x1000, k, 0x1000, 0x1000,
+                                    0x1000, 1 << 30, 0, 0) == fp.FATHOM_ERR_INVALID_ARG
+    assert lib.fathom_scan_topk(ctypes.byref(ix), 0x1000, 0x1000, 0x1000, 8, 0x1000, 0x1000,
+                                0x1000, 1 << 30, 1 << 7, 0) == fp.FATHOM_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(fp, "_lib", None)
+    with pytest.raises(ImportError):
+        fp.load_library(str(tmp_path / "missing.so"))
