@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the Fathom per-query read-depth top-k key scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
+                    [--workload qwen3_8b_layer_128k|host_1m]
+
+A step is one decode-step scan of a whole layer through the hot path, once
+per bit budget of the workload: plan (reverse water-filling, GQA union) then
+scan + top-k, for every KV head and query head.  Default workload: a
+Qwen3-8B-shaped layer resident in HBM (8 KV heads x 4 query heads,
+head_dim 128, 131072 keys, B in {68, 92, 136}, k = 2048).  Inputs are
+synthetic (seeded, see synth/); each step gets fresh queries and the L2 is
+flushed (256 MiB write) between timed steps, outside the step's events.
+
+Prints one JSON line (rank 0).  value = Gkeys/s over all ranks (keys per KV
+head x KV heads x budgets x steps / the slowest rank's summed step time).
+For N > 1 each rank scans its own independent layer (weak scaling; the path
+needs no collective).  --impl reference times the CPU oracle instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "Gkeys/s per decode-step scan; achieved GB/s vs HBM / PCIe roofline"
+UNIT = "Gkeys/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+WORKLOADS = {
+    "qwen3_8b_layer_128k": dict(H=8, G=4, n=131072, d=128, budgets=(68, 92, 136), k=2048,
+                                residency="device"),
+    "host_1m": dict(H=8, G=4, n=1 << 20, d=128, budgets=(18, 68, 92, 136), k=2048,
+                    residency="host_mapped"),
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
+    p.add_argument("--workload", choices=tuple(WORKLOADS), default="qwen3_8b_layer_128k")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--heat-seconds", type=float, default=1.0,
+                   help="minimum warm-up duration (load for the clock sampler); 0 for "
+                        "profiler runs, which then see exactly --warmup warm-up steps")
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def config_of(wl_name, wl, flush_note):
+    return {"workload": wl_name, "kv_heads": wl["H"], "query_heads_per_kv": wl["G"],
+            "head_dim": wl["d"], "n_keys": wl["n"], "budgets_bits_per_key": list(wl["budgets"]),
+            "k": wl["k"], "residency": "hbm" if wl["residency"] == "device" else "host_pinned_mapped",
+            "l2": flush_note}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample(ses, budgets, k, heads, ref=None):
+    """Time the oracle (plan + fp64 score + full-sort top-k per query) on the
+    given KV heads at every budget.  The index build (storage side, off the
+    decode path) is not timed.  Returns (seconds, head-scans, keys)."""
+    import oracle
+    if ref is None:
+        ref = oracle.build_index(ses.keys[list(heads)])
+    G = ses.group
+    t0 = time.perf_counter()
+    scans = 0
+    for hi, h in enumerate(heads):
+        for B in budgets:
+            for g in range(G):
+                qrow = ses.q_bf16[h * G + g]
+                tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), B)
+                s = oracle.score_planes(ref["planes"][hi], ref["mn"][hi], ref["scale"][hi],
+                                        qrow, tq, ses.n_keys)
+                oracle.topk(s, k)
+            scans += 1
+    return time.perf_counter() - t0, scans, scans * ses.n_keys
+
+
+def cpu_baseline(ses, wl):
+    # about 10-30 s of single-thread oracle work
+    heads = tuple(range(max(1, min(4, wl["H"], (4 * 131072) // wl["n"]))))
+    secs, scans, keys = oracle_sample(ses, wl["budgets"], wl["k"], heads)
+    return {"value": keys / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"KV heads {list(heads)} x budgets {list(wl['budgets'])}: {scans} head "
+                      f"scans of {ses.n_keys} keys (4 query heads each), single thread, "
+                      f"{secs:.1f} s"}
+
+
+def run_reference(args, wl_name, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    n = wl["n"] if wl["residency"] == "device" else min(wl["n"], 1 << 18)
+    ses = synth.make_session(0, 1, wl["G"], n, wl["budgets"][0], head_dim=wl["d"])
+    budgets = wl["budgets"]
+    import oracle
+    ref = oracle.build_index(ses.keys[:1])
+    times = []
+    for i in range(args.warmup + args.steps):
+        secs, _, _ = oracle_sample(ses, (budgets[i % len(budgets)],), wl["k"], (0,), ref)
+        if i >= args.warmup:
+            times.append(secs)
+    keys_per_step = n                      # one KV head, one budget, per step
+    total = sum(times)
+    value = keys_per_step * len(times) / total / 1e9
+    sample = (f"each step: 1 of {wl['H']} KV heads ({wl['G']} query heads), one budget "
+              f"(cycling {list(budgets)}), {n} keys, single thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl_name, wl, "n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU path
+def run_fathom(args, wl_name, wl):
+    import torch
+    import decode_fathom_plan_b200 as fp
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    fp.load_library()
+    H, G, n, d, k = wl["H"], wl["G"], wl["n"], wl["d"], wl["k"]
+    budgets = wl["budgets"]
+    Q = H * G
+    ses = synth.make_session(rank, H, G, n, budgets[0], head_dim=d)
+    keys_dev = torch.from_numpy(ses.keys).cuda()
+    index = fp.KeyIndex(H, G, n, d, wl["residency"])
+    index.pack(keys_dev)
+    torch.cuda.synchronize()
+    assert fp.fathom_last_device_status() == fp.FATHOM_OK
+
+    W, K = max(3, args.warmup), args.steps
+    qsets = synth.draw_queries(10_000 + rank, Q, d, count=W + K)
+    q_dev = torch.from_numpy(qsets.view(np.int16)).cuda()
+    bvec = [torch.full((Q,), B, dtype=torch.int32, device="cuda") for B in budgets]
+    bufs = [fp.ScanBuffers(index, k) for _ in budgets]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step(i, flags=0):
+        for bi in range(len(budgets)):
+            fp.plan_and_scan(index, q_dev[i], bvec[bi], bufs[bi], flags=flags)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_heat = time.perf_counter()
+    i = 0
+    while i < W or time.perf_counter() - t_heat < args.heat_seconds:   # warm-up + clock load
+        step(i % W)
+        flush.fill_(i & 0xFF)
+        i += 1
+    torch.cuda.synchronize()
+    fp.fathom_profile_read()
+    status = fp.fathom_last_device_status()
+    assert status == fp.FATHOM_OK, fp.status_str(status)
+
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = fp.fathom_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for s in range(K):
+        flush.fill_(s & 0xFF)
+        ev[s][0].record()
+        step(W + s, fp.FATHOM_SCAN_PROFILE)
+        ev[s][1].record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = fp.fathom_launch_count() - launches0
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    scan_ms, scan_launches = fp.fathom_profile_read()
+    status = fp.fathom_last_device_status()
+    assert status == fp.FATHOM_OK, fp.status_str(status)
+
+    # plan byte counts of the last step (identical structure every step)
+    per_budget = []
+    union_bytes_total = 0
+    for bi, B in enumerate(budgets):
+        nb = bufs[bi].nbytes.cpu().numpy()
+        qb, ub = nb[:Q].astype(np.float64), nb[Q:].astype(np.float64)
+        union_bytes_total += ub.sum()
+        per_budget.append({"B": B, "bytes_per_query": float(qb.mean()),
+                           "union_bytes_per_kv_head": float(ub.mean()),
+                           "union_factor": float(ub.sum() / (qb.sum() / G))})
+
+    # quality: recall against the exact fp32 top-k (torch, outside the path)
+    with torch.no_grad():
+        qf = q_dev[W + K - 1].view(torch.bfloat16).float().reshape(H, G, d)
+        for bi, pb in enumerate(per_budget):
+            got = bufs[bi].idx.reshape(H, G, k).long()
+            rec = []
+            for h in range(H):
+                exact = (keys_dev[h] @ qf[h].T).topk(k, dim=0).indices.T     # [G][k]
+                for g in range(G):
+                    inter = np.intersect1d(exact[g].cpu().numpy(), got[h, g].cpu().numpy())
+                    rec.append(len(inter) / k)
+            pb["recall_vs_exact_fp32"] = float(np.mean(rec))
+
+    # end to end through the public API with host buffers
+    q_host = torch.from_numpy(qsets[W:W + K].view(np.int16)).pin_memory()
+    b_host = [torch.full((Q,), B, dtype=torch.int32).pin_memory() for B in budgets]
+    q_stage = torch.empty((Q, d), dtype=torch.int16, device="cuda")
+    idx_host = [torch.empty((Q, k), dtype=torch.int32).pin_memory() for _ in budgets]
+    sc_host = [torch.empty((Q, k), dtype=torch.float32).pin_memory() for _ in budgets]
+    e2e_s = []
+    for s in range(K):
+        flush.fill_(s & 0xFF)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for bi in range(len(budgets)):
+            q_stage.copy_(q_host[s], non_blocking=True)
+            bvec[bi].copy_(b_host[bi], non_blocking=True)
+            fp.plan_and_scan(index, q_stage, bvec[bi], bufs[bi])
+            idx_host[bi].copy_(bufs[bi].idx, non_blocking=True)
+            sc_host[bi].copy_(bufs[bi].score, non_blocking=True)
+        torch.cuda.synchronize()
+        e2e_s.append(time.perf_counter() - t0)
+    h2d = len(budgets) * (Q * d * 2 + Q * 4)
+    d2h = len(budgets) * (Q * k * 8)
+
+    keys_per_step = H * n * len(budgets)
+    if dist:
+        t = torch.tensor([total_ms, sum(e2e_s)], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_total = float(t[0]), float(t[1])
+    else:
+        e2e_total = sum(e2e_s)
+    value = keys_per_step * K * world / (total_ms / 1e3) / 1e9
+    e2e_value = keys_per_step * K * world / e2e_total / 1e9
+
+    peak, peak_src = load_peaks()
+    bytes_per_launch = union_bytes_total / len(budgets)
+    avg_launch_ms = scan_ms / max(1, scan_launches)
+    achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm" if wl["residency"] == "device" else "host_link",
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "scan_kernel (filter pass)",
+                "peak_source": f"{peak_src} hbm_gbs", "avg_launch_us": avg_launch_ms * 1e3,
+                "algorithmic_bytes_per_launch": bytes_per_launch}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_of(wl_name, wl, "flushed between steps (256 MiB write)"),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches), "roofline": roofline, "clocks": clk,
+            "per_budget": per_budget,
+            "step_ms_median": statistics.median(step_ms)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(ses, wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, args.workload, wl)
+    else:
+        run_fathom(args, args.workload, wl)
+
+
+if __name__ == "__main__":
+    main()

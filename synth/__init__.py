@@ -165,3 +165,11 @@ WORKLOADS = {
     "fixed_vs_wf_1m": dict(H=8, G=4, n=1 << 20, budgets=(68, 92), fixed_r=(34, 17),
                            k=2048, residency="host_mapped"),
 }
+
+
+def draw_queries(seed: int, n_queries: int, head_dim: int = HEAD_DIM, count: int = 1) -> np.ndarray:
+    """`count` further query sets (one per decode step) with the recipe's
+    query distribution: N(0, 1) rounded to bfloat16.  -> uint16 [count][Q][d]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    q = rng.standard_normal((count, n_queries, head_dim)).astype(np.float32)
+    return f32_to_bf16_bits(q).reshape(count, n_queries, head_dim)
