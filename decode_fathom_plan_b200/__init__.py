@@ -37,6 +37,7 @@ EXPORTED = (
     "fathom_plan", "fathom_fixed_plan", "fathom_scan_workspace_bytes", "fathom_scan_topk",
     "fathom_scan_batched_workspace_bytes", "fathom_scan_topk_batched",
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
+    "fathom_scan_topk_static",
 )
 
 
@@ -81,6 +82,7 @@ def load_library(path: str = LIB_PATH):
         "fathom_fixed_plan": ([IX, P, I32, P, P, P, P], ctypes.c_int),
         "fathom_scan_workspace_bytes": ([IX, I32], SZ),
         "fathom_scan_topk": ([IX, P, P, P, I32, P, P, P, SZ, U32, P], ctypes.c_int),
+        "fathom_scan_topk_static": ([IX, P, P, P, I32, P, P, U32, P], ctypes.c_int),
         "fathom_scan_batched_workspace_bytes": ([IX, I32, I32], SZ),
         "fathom_scan_topk_batched": ([IX, I32, P, P, P, I32, P, P, P, SZ, U32, P], ctypes.c_int),
         "fathom_last_device_status": ([P], ctypes.c_int),
@@ -165,6 +167,17 @@ def fathom_scan_topk(index: fathom_index, q_bf16, t, t_union, k: int, out_idx, o
                                            _ptr(t_union), int(k), _ptr(out_idx), _ptr(out_score),
                                            _ptr(workspace), ws_bytes, int(flags),
                                            _stream(stream)), "fathom_scan_topk")
+
+
+def fathom_scan_topk_static(index: fathom_index, q_bf16, t, t_union, k: int, out_idx,
+                            out_score, flags: int = 0, stream=None):
+    """fathom_scan_topk without a workspace argument, for callers that cannot
+    allocate device memory: runs on the library's fixed 8 MiB per-GPU scratch
+    array (see include/fathom.h for the limits and the sharing rule)."""
+    _check(load_library().fathom_scan_topk_static(ctypes.byref(index), _ptr(q_bf16), _ptr(t),
+                                                  _ptr(t_union), int(k), _ptr(out_idx),
+                                                  _ptr(out_score), int(flags), _stream(stream)),
+           "fathom_scan_topk_static")
 
 
 def _index_array(sessions: Sequence[fathom_index]):

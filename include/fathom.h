@@ -17,7 +17,8 @@
  * Conventions for every call:
  *   - All buffers are owned by the caller.  The library allocates no device
  *     or host memory; scratch space is a caller-supplied workspace sized by
- *     the matching *_workspace_bytes call (16-byte aligned).
+ *     the matching *_workspace_bytes call (16-byte aligned).  The one
+ *     exception is the fixed scratch array behind fathom_scan_topk_static.
  *   - Calls are stream-ordered and asynchronous: they validate what the host
  *     can see, enqueue kernels on `stream` and return.  Argument errors are
  *     returned at once and enqueue nothing.  Errors that only the device can
@@ -173,6 +174,30 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
                                int32_t *out_idx, float *out_score,
                                void *workspace, size_t workspace_bytes,
                                uint32_t flags, cudaStream_t stream);
+
+/* fathom_scan_topk for callers that cannot allocate device memory (the
+ * paper has no counterpart: this is an interface convenience).  Some callers
+ * are handed only their inputs and outputs and have no allocator to call --
+ * e.g. a plugin inside an engine whose memory pool already owns the free HBM,
+ * or a decode loop that must not call cudaMalloc because it can synchronise
+ * the device.  This call takes no workspace: it runs on an 8 MiB scratch
+ * array that the library reserves as a static __device__ variable on every
+ * GPU that loads it, held until the process exits.
+ *   - Same arguments and results as fathom_scan_topk, minus the workspace.
+ *   - A problem needing more than 8 MiB of scratch (about one Qwen3-8B-shaped
+ *     layer, 32 query heads, at up to 1,048,576 keys with k <= 2048) is
+ *     rejected with FATHOM_ERR_WORKSPACE before anything is enqueued; use
+ *     fathom_scan_topk for it.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the one array.  Calls whose kernels overlap
+ *     on the GPU (e.g. on two streams at once) race on it: order them.
+ *   - Calls or frees no device memory. */
+fathom_status fathom_scan_topk_static(const fathom_index *index, const uint16_t *q_bf16,
+                                      const uint8_t *t, const uint8_t *t_union, int32_t k,
+                                      int32_t *out_idx, float *out_score, uint32_t flags,
+                                      cudaStream_t stream);
 
 /* Workspace bytes fathom_scan_topk_batched needs. */
 size_t fathom_scan_batched_workspace_bytes(const fathom_index *sessions,
