@@ -1,6 +1,8 @@
 // C ABI of the Fathom sm_100a library: argument validation, residency
 // resolution, workspace accounting, device status and instrumentation.
 // The operations themselves are documented in include/fathom.h.
+#include <stdio.h>
+
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -40,6 +42,14 @@ int *device_status_ptr()
 }
 
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+cudaError_t note_error(cudaError_t e, const char *site)
+{
+    if (e != cudaSuccess)
+        fprintf(stderr, "fathom: %s failed: %s (%s)\n", site, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+    return e;
+}
 
 }  // namespace fathom
 

@@ -13,6 +13,9 @@ namespace fathom {
 int *device_status_ptr();
 // Count one kernel launch (for fathom_launch_count).
 void note_launch(int n = 1);
+// Record the CUDA error of a failed step (reported on stderr once per site
+// by the C-ABI layer) and return it.
+cudaError_t note_error(cudaError_t e, const char *site);
 
 // ---- pack.cu
 cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_minmax,

@@ -9,91 +9,145 @@
 // sharing across a GQA group; here a KV head reads the union of its
 // queries' planes.
 //
-// One CTA per KV head, one warp per query head; d <= 256 channels, so each
-// lane owns d/32 channels.  Ranks come from counting (w' > w, or w' == w and
-// c' < c) over the d importances in shared memory, which gives
-// t_c = min(4, max(0, B - 4*rank_c)) without a sort.
+// One CTA per KV head, one warp per query head: the warp sorts the query's
+// channels by (w descending, channel ascending) in registers, so channel
+// c's position is rank_c and t_c = min(4, max(0, B - 4*rank_c)).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace fathom {
 namespace {
 
-template <bool kFixed>
-__global__ void plan_kernel(const uint16_t *__restrict__ q, const int32_t *__restrict__ budget,
-                            int32_t fixed_r, const float *__restrict__ sigma2, int G, int d,
-                            int n_words, uint8_t *t, uint8_t *t_union, uint64_t *bytes, int Q,
-                            int *status)
+// Sort N composite keys held E = N/32 per lane (element e = lane*E + i)
+// in descending order: bitonic network, strides below E inside the lane,
+// the rest by warp shuffles.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(unsigned long long (&key)[E])
 {
-    __shared__ float key[kMaxGroup][kMaxHeadDim];
+    const int lane = threadIdx.x & 31;
+    constexpr int N = 32 * E;
+#pragma unroll
+    for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+        for (int j = size >> 1; j > 0; j >>= 1) {
+            if (j < E) {
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    if ((i & j) == 0) {
+                        const int e = lane * E + i;
+                        const bool desc = (e & size) == 0;
+                        const unsigned long long a = key[i], b = key[i ^ j];
+                        if ((a < b) == desc) {
+                            key[i] = b;
+                            key[i ^ j] = a;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, key[i], j / E);
+                    const int e = lane * E + i;
+                    const bool desc = (e & size) == 0, low = (e & j) == 0;
+                    key[i] = (low == desc) ? max(key[i], other) : min(key[i], other);
+                }
+            }
+        }
+    }
+}
+
+// One CTA per KV head, one warp per query head.  Each warp sorts its
+// query's channels by (key descending, channel ascending) with a warp
+// bitonic network; a channel's position in that order is its rank, and
+// t_c = min(4, max(0, B - 4*rank)) (or 4 for the first r under the fixed
+// plan).  E = padded head_dim / 32.
+template <bool kFixed, int E>
+__global__ void __launch_bounds__(kMaxGroup * 32)
+plan_kernel(const uint16_t *__restrict__ q, const int32_t *__restrict__ budget, int32_t fixed_r,
+            const float *__restrict__ sigma2, int G, int d, int n_words, uint8_t *t,
+            uint8_t *t_union, uint64_t *bytes, int Q, int *status)
+{
     __shared__ uint8_t tt[kMaxGroup][kMaxHeadDim];
-    __shared__ unsigned long long union_bytes;
     const int h = blockIdx.x;
     const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qi = h * G + g;
-    const int per = d >> 5;
     const unsigned long long plane_bytes = 4ull * (unsigned long long)n_words;
-    if (threadIdx.x == 0) union_bytes = 0;
-
+    const int qi = h * G + g;
+    unsigned long long key[E];
     bool bad = false;
-    for (int i = 0; i < per; ++i) {
-        const int c = lane + 32 * i;
-        const float qf = bf16_to_float(q[(size_t)qi * d + c]);
-        float k;
-        if (kFixed) {
-            k = fabsf(qf);
-            bad |= !isfinite(qf);
-        } else {
-            k = __fmul_rn(__fmul_rn(qf, qf), sigma2[h * d + c]);
-            bad |= !isfinite(k);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = lane * E + i;
+        key[i] = 0ull;                                   // padding sorts last
+        if (c < d) {
+            const float qf = bf16_to_float(q[(size_t)qi * d + c]);
+            float k;
+            if (kFixed) {
+                k = fabsf(qf);
+                bad |= !isfinite(qf);
+            } else {
+                k = __fmul_rn(__fmul_rn(qf, qf), sigma2[h * d + c]);
+                bad |= !isfinite(k);
+            }
+            key[i] = ((unsigned long long)order_key(k) << 32) | (0xFFFFFFFFu - (uint32_t)c);
         }
-        key[g][c] = k;
     }
     bad = __any_sync(0xFFFFFFFFu, bad);
     int B = 0;
     if (!kFixed) {
         B = budget[qi];
         if (B < 0 || B > kBits * d) {
-            set_status(status, FATHOM_ERR_INVALID_ARG);
+            if (lane == 0) set_status(status, FATHOM_ERR_INVALID_ARG);
             B = 0;
         }
     }
-    if (bad) set_status(status, FATHOM_ERR_NONFINITE);
-    __syncwarp();
-
+    if (bad && lane == 0) set_status(status, FATHOM_ERR_NONFINITE);
+    warp_sort_desc<E>(key);
     unsigned long long my_bytes = 0;
-    for (int i = 0; i < per; ++i) {
-        const int c = lane + 32 * i;
-        const float kc = key[g][c];
-        int rank = 0;
-        for (int c2 = 0; c2 < d; ++c2) {
-            const float k2 = key[g][c2];
-            rank += (k2 > kc) || (k2 == kc && c2 < c);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int rank = lane * E + i;
+        const uint32_t c = 0xFFFFFFFFu - (uint32_t)(key[i] & 0xFFFFFFFFull);
+        if (key[i] != 0ull && c < (uint32_t)d) {
+            int tc = kFixed ? (rank < fixed_r ? kBits : 0) : min(kBits, max(0, B - kBits * rank));
+            if (bad) tc = 0;
+            tt[g][c] = (uint8_t)tc;
+            t[(size_t)qi * d + c] = (uint8_t)tc;
+            my_bytes += (unsigned long long)tc * plane_bytes;
         }
-        int tc;
-        if (kFixed)
-            tc = rank < fixed_r ? kBits : 0;
-        else
-            tc = min(kBits, max(0, B - kBits * rank));
-        if (bad) tc = 0;
-        tt[g][c] = (uint8_t)tc;
-        t[(size_t)qi * d + c] = (uint8_t)tc;
-        my_bytes += (unsigned long long)tc * plane_bytes;
     }
+#pragma unroll
     for (int off = 16; off > 0; off >>= 1) my_bytes += __shfl_xor_sync(0xFFFFFFFFu, my_bytes, off);
     if (lane == 0) bytes[qi] = my_bytes;
     __syncthreads();
-
-    unsigned long long ub = 0;
-    for (int c = threadIdx.x; c < d; c += blockDim.x) {
-        uint8_t m = 0;
-        for (int gg = 0; gg < G; ++gg) m = max(m, tt[gg][c]);
-        t_union[h * d + c] = m;
-        ub += (unsigned long long)m * plane_bytes;
+    // GQA union, one warp per 32 channels
+    if (g == 0) {
+        unsigned long long ub = 0;
+        for (int c = lane; c < d; c += 32) {
+            uint8_t m = 0;
+            for (int gg = 0; gg < G; ++gg) m = max(m, tt[gg][c]);
+            t_union[h * d + c] = m;
+            ub += (unsigned long long)m * plane_bytes;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ub += __shfl_xor_sync(0xFFFFFFFFu, ub, off);
+        if (lane == 0) bytes[Q + h] = ub;
     }
-    atomicAdd(&union_bytes, ub);
-    __syncthreads();
-    if (threadIdx.x == 0) bytes[Q + h] = union_bytes;
+}
+
+template <bool kFixed>
+void launch_plan_kernel(int E, dim3 grid, int threads, cudaStream_t stream, const uint16_t *q,
+                        const int32_t *budget, int32_t fixed_r, const float *sigma2, int G, int d,
+                        int n_words, uint8_t *t, uint8_t *t_union, uint64_t *bytes, int Q,
+                        int *status)
+{
+    switch (E) {
+    case 1: plan_kernel<kFixed, 1><<<grid, threads, 0, stream>>>(q, budget, fixed_r, sigma2, G, d, n_words, t, t_union, bytes, Q, status); break;
+    case 2: plan_kernel<kFixed, 2><<<grid, threads, 0, stream>>>(q, budget, fixed_r, sigma2, G, d, n_words, t, t_union, bytes, Q, status); break;
+    case 4: plan_kernel<kFixed, 4><<<grid, threads, 0, stream>>>(q, budget, fixed_r, sigma2, G, d, n_words, t, t_union, bytes, Q, status); break;
+    default: plan_kernel<kFixed, 8><<<grid, threads, 0, stream>>>(q, budget, fixed_r, sigma2, G, d, n_words, t, t_union, bytes, Q, status); break;
+    }
 }
 
 }  // namespace
@@ -105,12 +159,14 @@ cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t
     const int H = ix.n_kv_heads, G = ix.group, d = ix.head_dim;
     const int Q = H * G;
     int *status = device_status_ptr();
+    int E = 1;
+    while (32 * E < d) E <<= 1;   // head_dim padded to a power of two
     if (fixed)
-        plan_kernel<true><<<H, G * 32, 0, stream>>>(q, budget, fixed_r, ix.sigma2, G, d,
-                                                    ix.n_words, t, t_union, bytes, Q, status);
+        launch_plan_kernel<true>(E, dim3(H), G * 32, stream, q, budget, fixed_r, ix.sigma2, G, d,
+                                 ix.n_words, t, t_union, bytes, Q, status);
     else
-        plan_kernel<false><<<H, G * 32, 0, stream>>>(q, budget, fixed_r, ix.sigma2, G, d,
-                                                     ix.n_words, t, t_union, bytes, Q, status);
+        launch_plan_kernel<false>(E, dim3(H), G * 32, stream, q, budget, fixed_r, ix.sigma2, G, d,
+                                  ix.n_words, t, t_union, bytes, Q, status);
     note_launch(1);
     return cudaGetLastError();
 }

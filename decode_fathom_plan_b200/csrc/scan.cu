@@ -16,23 +16,30 @@
 // v is an integer 0..15, so the hot loop is "nibble -> float, then one fma
 // per query head", with no per-bit work.
 //
-// Data path (one CTA = one KV head x one 2048-key tile):
-//   * the union plan T_c = max_g t_gc of the KV head's G query heads decides
-//     which plane rows are read; each row slice is 256 contiguous bytes
-//     (64 words) and is copied into shared memory with 16-byte cp.async,
-//     three stages of up to 8 channels (32 rows) in flight;
-//   * thread (column, row r) owns keys 32*column + 4m + r, m = 0..7: a
-//     funnel-shift rotate and a mask move bit 4m+r of each plane word to bit
-//     4m+p, so one register holds the thread's 8 nibbles; each nibble
-//     becomes a float by OR-ing it under the mantissa of a power of two and
-//     subtracting that power (exact), two at a time with __fadd2_rn;
-//   * each query head reading the channel adds W*v with __ffma2_rn (two keys
-//     per instruction); a head reading fewer planes than the union masks
-//     its nibbles first.
+// Data path.  A KV head reads the union plan T_c = max_g t_gc of its G query
+// heads once.  Union channels are ordered by the set of query heads reading
+// them (stable counting sort), so the fma pattern is chosen once per run of
+// equal sets instead of once per channel.  A stage is 8 union channels x 4
+// plane rows x a chunk of up to 64 plane words (2048 keys); rows past a
+// channel's depth are zero-filled by cp.async without a global read, so every
+// channel is processed the same way.  Stages are copied into shared memory
+// with 16-byte cp.async, STAGES buffers deep.  Thread (column, row r) owns
+// keys 32*column + 4m + r, m = 0..7: a funnel-shift rotate and a mask move
+// bit 4m+r of each plane word to bit 4m+p, so one register holds the
+// thread's 8 nibbles; each nibble becomes a float by OR-ing it under the
+// mantissa of a power of two and subtracting that power (exact), two at a
+// time with __fadd2_rn; each query head reading the channel adds W*v with
+// __ffma2_rn (two keys per instruction).
+//
+// Work distribution: persistent CTAs (as many as are resident) each take an
+// equal contiguous range of 4-word column groups of the (session, KV head)
+// sequence, so there is no partial last wave; a CTA rebuilds its per-head
+// tables only when its range crosses into the next head.
+//
 // No tensor cores: this is a sparse binary-weighted reduction.
 //
 // Selection without materialising n scores per query:
-//   1. sample:   score a few evenly spaced tiles (about 3% of the keys) and
+//   1. sample:   score evenly strided whole tiles (about 3% of the keys) and
 //                write their order keys to the workspace;
 //   2. theta:    per query, theta = the r-th largest sampled key, with r
 //                about 2*k*m/n, so ~2k keys are expected to pass;
@@ -44,8 +51,8 @@
 //   5. fallback: a flagged query is redone exactly by one CTA that
 //                recomputes its scores once per radix digit (no score
 //                buffer), so results never depend on the sample.
-// Every key of the sampled pass is recomputed by the full scan with the same
-// arithmetic, so a key's score is the same in both passes.
+// Correctness needs only that every key scoring at least the k-th largest
+// score is a candidate, which "count >= k" guarantees for any theta.
 #include <math.h>
 
 #include <algorithm>
@@ -56,6 +63,10 @@
 
 namespace fathom {
 namespace {
+
+constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-word chunk
+constexpr int kMainStages = 3;
+constexpr int kSampleStages = 8;
 
 struct SessionDesc {
     const uint32_t *planes;      // device address of [H][d][4][n_words]
@@ -69,9 +80,9 @@ struct SessionDesc {
     uint32_t *qstate;            // [Q][4]: theta, count, fallback flag, spare
     uint32_t *sample;            // [Q][m_keys]
     unsigned long long *cand;    // [Q][cap]
-    int H, n, n_words, n_cols, n_tiles;
+    int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int item_begin, sample_item_begin, q_begin;
+    int group_begin, sample_group_begin, q_begin;
 };
 
 template <int NS>
@@ -80,19 +91,24 @@ struct Batch {
     SessionDesc s[NS];
 };
 
+// Per-head tables of a scanning CTA (the stage buffers live in dynamic
+// shared memory).
 template <int GP>
-struct alignas(16) ScanSmem {
-    alignas(16) uint32_t stage[kStages][kStageRows][kTileCols];   // cp.async needs 16-byte rows
-    uint32_t row_g[kBits * kMaxHeadDim];         // global plane row of each union row
-    float W[kMaxHeadDim][GP];                    // q*scale per (union channel, query)
-    uint8_t tq[kMaxHeadDim][GP];                 // planes read per (union channel, query)
-    uint8_t uT[kMaxHeadDim];                     // union depth
-    uint8_t uro[kMaxHeadDim];                    // first row of the channel inside its stage
-    uint16_t stage_row0[kMaxHeadDim / kStageChannels + 1];
+struct alignas(16) ScanMeta {
+    alignas(16) float2 W2[kMaxHeadDim][GP];   // (w, w), w = q*scale if the query reads all T
+                                              // planes of the union channel, else (0, 0)
+    float Wp[kMaxHeadDim][GP];                // w = q*scale (partial-depth readers)
+    uint32_t row_g[kBits * kMaxHeadDim];      // plane row of (union channel, slot); ~0u = zero fill
+    uint32_t meta[kMaxHeadDim];               // bits 0-7: queries reading all T planes;
+                                              // bits 16-23: queries reading 0 < t < T planes
+    uint8_t tq[kMaxHeadDim][GP];              // planes read per (union channel, query)
+    uint8_t stage_partial[kMaxHeadDim / kStageChannels];   // a query reads 0 < t < T in the stage
     float bias[GP];
-    int U, P, n_stages;
-    int part[2][kScanThreads / 32];
+    int U, n_stages;
+    int part[kScanThreads / 32];
 };
+
+typedef uint32_t (*StageBuf)[kStageRows][kTileCols];
 
 // ------------------------------------------------------------ small helpers
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
@@ -115,23 +131,47 @@ __device__ __forceinline__ void cp_async_wait()
 // 8 nibbles of a word -> 8 exact floats, paired (m, m+4).  A nibble at bit
 // 4m is OR-ed under the mantissa of 2^(23-4m), whose unit in the last place
 // there is 1, so the float is 2^(23-4m) + v; subtracting the power leaves v.
-// Nibbles 5..7 are shifted down by 20 bits first (bits 20..31 would reach
-// the exponent).
-__device__ __forceinline__ void nibbles_to_floats(uint32_t nib, float2 (&v)[4])
+// Nibble m+4 sits at bit 4m of nib >> 16, so both halves of the 64-bit word
+// {nib, nib >> 16} use the same mask and power, and each pair is one
+// 64-bit and/or plus one paired add (add.rn.f32x2) with no repacking.
+// neg[m] holds -2^(23-4m) in both halves.
+__device__ __forceinline__ void nibbles_to_floats(uint32_t nib, const unsigned long long (&neg)[4],
+                                                  float2 (&v)[4])
 {
-    const uint32_t hi = nib >> 20;
-    const float f0 = __uint_as_float((nib & 0x0000000Fu) | 0x4B000000u);   // 2^23
-    const float f1 = __uint_as_float((nib & 0x000000F0u) | 0x49000000u);   // 2^19
-    const float f2 = __uint_as_float((nib & 0x00000F00u) | 0x47000000u);   // 2^15
-    const float f3 = __uint_as_float((nib & 0x0000F000u) | 0x45000000u);   // 2^11
-    const float f4 = __uint_as_float((nib & 0x000F0000u) | 0x43000000u);   // 2^7
-    const float f5 = __uint_as_float((hi & 0x0000000Fu) | 0x4B000000u);
-    const float f6 = __uint_as_float((hi & 0x000000F0u) | 0x49000000u);
-    const float f7 = __uint_as_float((hi & 0x00000F00u) | 0x47000000u);
-    v[0] = __fadd2_rn(make_float2(f0, f4), make_float2(-8388608.0f, -128.0f));
-    v[1] = __fadd2_rn(make_float2(f1, f5), make_float2(-524288.0f, -8388608.0f));
-    v[2] = __fadd2_rn(make_float2(f2, f6), make_float2(-32768.0f, -524288.0f));
-    v[3] = __fadd2_rn(make_float2(f3, f7), make_float2(-2048.0f, -32768.0f));
+    unsigned long long r0, r1, r2, r3;
+    asm("{\n"
+        ".reg .b64 p, t;\n"
+        ".reg .b32 h;\n"
+        "shr.b32 h, %4, 16;\n"
+        "mov.b64 p, {%4, h};\n"
+        "and.b64 t, p, 0x0000000F0000000F;\n"
+        "or.b64 t, t, 0x4B0000004B000000;\n"
+        "add.rn.f32x2 %0, t, %5;\n"
+        "and.b64 t, p, 0x000000F0000000F0;\n"
+        "or.b64 t, t, 0x4900000049000000;\n"
+        "add.rn.f32x2 %1, t, %6;\n"
+        "and.b64 t, p, 0x00000F0000000F00;\n"
+        "or.b64 t, t, 0x4700000047000000;\n"
+        "add.rn.f32x2 %2, t, %7;\n"
+        "and.b64 t, p, 0x0000F0000000F000;\n"
+        "or.b64 t, t, 0x4500000045000000;\n"
+        "add.rn.f32x2 %3, t, %8;\n"
+        "}"
+        : "=l"(r0), "=l"(r1), "=l"(r2), "=l"(r3)
+        : "r"(nib), "l"(neg[0]), "l"(neg[1]), "l"(neg[2]), "l"(neg[3]));
+    v[0] = make_float2(__uint_as_float((uint32_t)r0), __uint_as_float((uint32_t)(r0 >> 32)));
+    v[1] = make_float2(__uint_as_float((uint32_t)r1), __uint_as_float((uint32_t)(r1 >> 32)));
+    v[2] = make_float2(__uint_as_float((uint32_t)r2), __uint_as_float((uint32_t)(r2 >> 32)));
+    v[3] = make_float2(__uint_as_float((uint32_t)r3), __uint_as_float((uint32_t)(r3 >> 32)));
+}
+
+// -2^(23-4m) in both halves, m = 0..3.
+__constant__ unsigned long long c_neg_magic[4] = {0xCB000000CB000000ull, 0xC9000000C9000000ull,
+                                                  0xC7000000C7000000ull, 0xC5000000C5000000ull};
+__device__ __forceinline__ void magic_negatives(unsigned long long (&neg)[4])
+{
+#pragma unroll
+    for (int m = 0; m < 4; ++m) neg[m] = c_neg_magic[m];
 }
 
 // Offset of the coarse-bin middle: (2^(4-t) - 1) / 2.
@@ -141,66 +181,71 @@ __device__ __forceinline__ double bin_offset(int t)
 }
 
 // ------------------------------------------------------- per-head set-up
-// Builds the union channel list, plane-row table, weights and biases for
-// query heads q_rows[0..G) of KV head h.  tu_row: the union plan to read;
-// t_rows: each query's own plan.  256 threads, d <= 256.
+// Builds the union channel list (channel order), plane-row table, weights
+// (zero for a query that does not read the channel at full union depth) and
+// biases for query heads q_rows[0..G) of KV head h.
+// tu_row: the union plan to read; t_rows: each query's own plan.
+// 256 threads, d <= 256.  Ends with a barrier.
 template <int GP>
-__device__ void setup_head(ScanSmem<GP> &sm, int h, int G, int d, const uint8_t *tu_row,
+__device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t *tu_row,
                            const uint8_t *t_rows, const uint16_t *q_rows, const float *mn_h,
                            const float *sc_h)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int T = (tid < d) ? min((int)tu_row[tid], kBits) : 0;
-    const int has = T > 0;
-    int inc_u = has, inc_p = T;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int a = __shfl_up_sync(0xFFFFFFFFu, inc_u, off);
-        const int b = __shfl_up_sync(0xFFFFFFFFu, inc_p, off);
-        if (lane >= off) { inc_u += a; inc_p += b; }
-    }
-    if (lane == 31) { sm.part[0][warp] = inc_u; sm.part[1][warp] = inc_p; }
+    const int c = tid;
+    const int T = (c < d) ? min((int)tu_row[c], kBits) : 0;
+    const bool has = T > 0;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
+    if (lane == 0) sm.part[warp] = __popc(bal);
+    if (tid < kMaxHeadDim / kStageChannels) sm.stage_partial[tid] = 0;
     __syncthreads();
-    int base_u = 0, base_p = 0, U = 0, P = 0;
+    int base = 0, U = 0;
 #pragma unroll
     for (int w = 0; w < kScanThreads / 32; ++w) {
-        if (w < warp) { base_u += sm.part[0][w]; base_p += sm.part[1][w]; }
-        U += sm.part[0][w];
-        P += sm.part[1][w];
+        const int p = sm.part[w];
+        base += (w < warp) ? p : 0;
+        U += p;
     }
-    const int u = base_u + inc_u - has;
-    const int prow = base_p + inc_p - T;
+    const int n_stages = (U + kStageChannels - 1) / kStageChannels;
     if (has) {
-        const int c = tid;
-        sm.uT[u] = (uint8_t)T;
-        if ((u % kStageChannels) == 0) sm.stage_row0[u / kStageChannels] = (uint16_t)prow;
-        for (int s = 0; s < T; ++s) sm.row_g[prow + s] = (uint32_t)((h * d + c) * kBits + s);
+        const int u = base + __popc(bal & ((1u << lane) - 1u));
         const float sc = sc_h[c];
+        unsigned full = 0, partial = 0;
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
+            int tg = 0;
+            float w = 0.0f;
             if (g < G) {
-                sm.W[u][g] = __fmul_rn(bf16_to_float(q_rows[g * d + c]), sc);
-                sm.tq[u][g] = (uint8_t)min((int)t_rows[g * d + c], T);
-            } else {
-                sm.W[u][g] = 0.0f;
-                sm.tq[u][g] = 0;
+                tg = min((int)t_rows[g * d + c], T);
+                w = __fmul_rn(bf16_to_float(q_rows[g * d + c]), sc);
             }
+            if (tg == T) full |= 1u << g;
+            else if (tg > 0) partial |= 1u << g;
+            // full-depth readers use W2 in the unconditional fma; others add 0
+            // there and, if partial, their own masked term
+            sm.W2[u][g] = (tg == T) ? make_float2(w, w) : make_float2(0.0f, 0.0f);
+            sm.Wp[u][g] = w;
+            sm.tq[u][g] = (uint8_t)tg;
         }
+        sm.meta[u] = full | (partial << 16);
+        if (partial) sm.stage_partial[u / kStageChannels] = 1;
+#pragma unroll
+        for (int s2 = 0; s2 < kBits; ++s2)
+            sm.row_g[u * kBits + s2] = (s2 < T) ? (uint32_t)((h * d + c) * kBits + s2) : 0xFFFFFFFFu;
     }
+    for (int i = U * kBits + tid; i < n_stages * kStageRows; i += blockDim.x) sm.row_g[i] = 0xFFFFFFFFu;
     if (tid == 0) {
         sm.U = U;
-        sm.P = P;
-        sm.n_stages = (U + kStageChannels - 1) / kStageChannels;
-        sm.stage_row0[(U + kStageChannels - 1) / kStageChannels] = (uint16_t)P;
+        sm.n_stages = n_stages;
     }
     // bias_g over every channel, each at its own (clamped) depth
     if (warp < GP) {
         double acc = 0.0;
         if (warp < G) {
-            for (int c = lane; c < d; c += 32) {
-                const int tg = min((int)t_rows[warp * d + c], min((int)tu_row[c], kBits));
-                const double qf = (double)bf16_to_float(q_rows[warp * d + c]);
-                acc += qf * ((double)mn_h[c] + (double)sc_h[c] * bin_offset(tg));
+            for (int cc = lane; cc < d; cc += 32) {
+                const int tg = min((int)t_rows[warp * d + cc], min((int)tu_row[cc], kBits));
+                const double qf = (double)bf16_to_float(q_rows[warp * d + cc]);
+                acc += qf * ((double)mn_h[cc] + (double)sc_h[cc] * bin_offset(tg));
             }
         }
 #pragma unroll
@@ -208,93 +253,147 @@ __device__ void setup_head(ScanSmem<GP> &sm, int h, int G, int d, const uint8_t 
         if (lane == 0) sm.bias[warp] = (float)acc;
     }
     __syncthreads();
-    if (has) sm.uro[u] = (uint8_t)(prow - sm.stage_row0[u / kStageChannels]);
-    __syncthreads();
 }
 
-// ------------------------------------------------------------- tile scan
+// ------------------------------------------------------------- chunk scan
+// Copy stage st (32 plane rows x the chunk's 16-byte column groups in
+// [col_lo, col_hi)) into stage buffer buf.  Rows past a channel's depth and
+// columns past col_hi are zero-filled with no global read.
 template <int GP>
-__device__ __forceinline__ void load_stage(ScanSmem<GP> &sm, int st, int buf,
-                                           const uint32_t *planes, int n_words, int n_cols,
-                                           int col0)
+__device__ __forceinline__ void load_stage(const ScanMeta<GP> &sm, StageBuf stage, int st,
+                                           int buf, const uint32_t *planes, int n_words,
+                                           int col_lo, int col_hi)
 {
-    const int r0 = sm.stage_row0[st];
-    const int R = sm.stage_row0[st + 1] - r0;
     const int chunk = threadIdx.x & 15;
-    const int col = col0 + chunk * 4;
-    const bool ok = col < n_cols;
-    for (int row = threadIdx.x >> 4; row < R; row += kScanThreads / 16) {
-        const uint32_t *src = planes + (size_t)sm.row_g[r0 + row] * (size_t)n_words + (ok ? col : 0);
-        cp_async16(&sm.stage[buf][row][chunk * 4], src, ok ? 16 : 0);
+    const int col = col_lo + chunk * 4;
+    const bool ok = col < col_hi;
+    const uint32_t *rows = &sm.row_g[st * kStageRows];
+#pragma unroll
+    for (int row = threadIdx.x >> 4; row < kStageRows; row += kScanThreads / 16) {
+        const uint32_t g = rows[row];
+        const bool live = ok && g != 0xFFFFFFFFu;
+        const uint32_t *src = live ? planes + (size_t)g * (size_t)n_words + col : planes;
+        cp_async16(&stage[buf][row][chunk * 4], src, live ? 16 : 0);
     }
 }
 
-template <int GP>
-__device__ __forceinline__ void compute_stage(const ScanSmem<GP> &sm, int st, int buf, int col,
-                                              int r, float2 (&acc)[GP][4])
+// The thread's 8 nibbles of one channel: bit 4m+r of the word in slot s
+// (bit 3-s of the code) moves to bit 4m+(3-s) by a rotate and a mask.
+// sh[p] = (r - p) mod 32.
+template <int COLS = kTileCols>
+__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t (*rows)[COLS], int col,
+                                                   const uint32_t (&sh)[4])
 {
-    const int u0 = st * kStageChannels;
-    const int u1 = min(u0 + kStageChannels, sm.U);
-    for (int u = u0; u < u1; ++u) {
-        const int T = sm.uT[u];
-        const int ro = sm.uro[u];
-        uint32_t nib = 0;
+    const uint32_t x0 = rows[0][col], x1 = rows[1][col], x2 = rows[2][col], x3 = rows[3][col];
+    uint32_t nib = __funnelshift_r(x0, x0, sh[3]) & 0x88888888u;
+    nib |= __funnelshift_r(x1, x1, sh[2]) & 0x44444444u;
+    nib |= __funnelshift_r(x2, x2, sh[1]) & 0x22222222u;
+    nib |= __funnelshift_r(x3, x3, sh[0]) & 0x11111111u;
+    return nib;
+}
+
+// Queries reading fewer planes than the union drop the low bits first.
+template <int GP>
+__device__ __forceinline__ void fma_partial(unsigned pmask, uint32_t nib, int u,
+                                            const ScanMeta<GP> &sm,
+                                            const unsigned long long (&neg)[4],
+                                            float2 (&acc)[GP][4])
+{
 #pragma unroll
-        for (int s = 0; s < kBits; ++s) {
-            if (s < T) {
-                const uint32_t x = sm.stage[buf][ro + s][col];
-                const int p = kBits - 1 - s;   // slot s holds bit 3-s
-                nib |= __funnelshift_r(x, x, (r - p) & 31) & (0x11111111u << p);
-            }
-        }
-        float2 v[4];
-        nibbles_to_floats(nib, v);
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
+    for (int g = 0; g < GP; ++g) {
+        if (pmask & (1u << g)) {
             const int tg = sm.tq[u][g];
-            if (tg == 0) continue;
-            const float w = sm.W[u][g];
+            const uint32_t keep = ((0xFu << (kBits - tg)) & 0xFu) * 0x11111111u;
+            float2 vm[4];
+            nibbles_to_floats(nib & keep, neg, vm);
+            const float w = sm.Wp[u][g];
             const float2 w2 = make_float2(w, w);
-            if (tg == T) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[g][i] = __ffma2_rn(v[i], w2, acc[g][i]);
-            } else {
-                const uint32_t keep = ((0xFu << (kBits - tg)) & 0xFu) * 0x11111111u;
-                float2 vm[4];
-                nibbles_to_floats(nib & keep, vm);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[g][i] = __ffma2_rn(vm[i], w2, acc[g][i]);
-            }
+            for (int i = 0; i < 4; ++i) acc[g][i] = __ffma2_rn(vm[i], w2, acc[g][i]);
         }
     }
 }
 
-// Scores of the thread's 8 keys of tile `tile` for every query head:
+// One union channel: gather the thread's 8 nibbles, convert, and add
+// W2[u][g] * v for every query head (W2 is zero for heads that do not read
+// the channel at full union depth).
+template <int GP, bool kPartial, int COLS = kTileCols>
+__device__ __forceinline__ void channel(const ScanMeta<GP> &sm, const uint32_t (*rows)[COLS],
+                                        int u, int col, const uint32_t (&sh)[4],
+                                        const unsigned long long (&neg)[4], float2 (&acc)[GP][4])
+{
+    const uint32_t nib = gather_nibbles<COLS>(rows, col, sh);
+    float2 v[4];
+    nibbles_to_floats(nib, neg, v);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        const float2 w = sm.W2[u][g];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[g][i] = __ffma2_rn(v[i], w, acc[g][i]);
+    }
+    if (kPartial) {
+        const uint32_t meta = sm.meta[u];
+        if (meta >> 16) fma_partial<GP>(meta >> 16, nib, u, sm, neg, acc);
+    }
+}
+
+// Channels [u0, u1) of the stage held in `rows` (channel u0 in rows 0..3).
+template <int GP, int COLS = kTileCols>
+__device__ __forceinline__ void compute_stage(const ScanMeta<GP> &sm, int st,
+                                              const uint32_t (*rows)[COLS], int u0, int u1,
+                                              int col, const uint32_t (&sh)[4],
+                                              const unsigned long long (&neg)[4],
+                                              float2 (&acc)[GP][4])
+{
+    if (u1 - u0 == kStageChannels && !sm.stage_partial[st]) {
+#pragma unroll
+        for (int j = 0; j < kStageChannels; ++j)
+            channel<GP, false, COLS>(sm, rows + kBits * j, u0 + j, col, sh, neg, acc);
+    } else {
+        for (int u = u0; u < u1; ++u)
+            channel<GP, true, COLS>(sm, rows + kBits * (u - u0), u, col, sh, neg, acc);
+    }
+}
+
+// Scores of the thread's 8 keys of the chunk of plane words [col_lo, col_hi)
+// (at most 64 words) for every query head:
 // score(g, m) = bias_g + acc[g][m % 4].{x if m < 4 else y}.
-template <int GP>
-__device__ void scan_tile(ScanSmem<GP> &sm, const uint32_t *planes, int n_words, int n_cols,
-                          int tile, float2 (&acc)[GP][4])
+// Warps whose 8 columns lie past col_hi only take part in the copies and
+// barriers.  Starts with a barrier (stage buffers may still be in use).
+template <int GP, int STAGES>
+__device__ void scan_chunk(const ScanMeta<GP> &sm, StageBuf stage, const uint32_t *planes,
+                           int n_words, int col_lo, int col_hi, float2 (&acc)[GP][4])
 {
     const int col = threadIdx.x >> 2, r = threadIdx.x & 3;
-    const int col0 = tile * kTileCols;
+    const bool busy = col_lo + ((threadIdx.x >> 5) << 3) < col_hi;   // warp-uniform
+    uint32_t sh[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
+    unsigned long long neg[4];
+    magic_negatives(neg);
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[g][i] = make_float2(0.0f, 0.0f);
     const int n_stages = sm.n_stages;
-    __syncthreads();   // stage buffers may still be read by a previous tile
+    const int U = sm.U;
+    __syncthreads();
 #pragma unroll
-    for (int st = 0; st < kStages - 1; ++st) {
-        if (st < n_stages) load_stage(sm, st, st, planes, n_words, n_cols, col0);
+    for (int st = 0; st < STAGES - 1; ++st) {
+        if (st < n_stages) load_stage(sm, stage, st, st, planes, n_words, col_lo, col_hi);
         cp_async_commit();
     }
     for (int st = 0; st < n_stages; ++st) {
-        cp_async_wait<kStages - 2>();
+        cp_async_wait<STAGES - 2>();
         __syncthreads();
-        const int nx = st + kStages - 1;
-        if (nx < n_stages) load_stage(sm, nx, nx % kStages, planes, n_words, n_cols, col0);
+        const int nx = st + STAGES - 1;
+        if (nx < n_stages) load_stage(sm, stage, nx, nx % STAGES, planes, n_words, col_lo, col_hi);
         cp_async_commit();
-        compute_stage(sm, st, st % kStages, col, r, acc);
+        if (busy) {
+            const int u0 = st * kStageChannels;
+            compute_stage<GP>(sm, st, stage[st % STAGES], u0, min(u0 + kStageChannels, U), col, sh,
+                              neg, acc);
+        }
     }
     cp_async_wait<0>();
 }
@@ -306,11 +405,11 @@ __device__ __forceinline__ float score_of(const float2 (&a)[4], int m, float bia
 }
 
 template <int NS>
-__device__ __forceinline__ int find_session_by_item(const Batch<NS> &b, int item, bool sample)
+__device__ __forceinline__ int find_session_by_group(const Batch<NS> &b, int g, bool sample)
 {
     int si = 0;
     for (int s = 1; s < b.n_sessions; ++s)
-        if ((sample ? b.s[s].sample_item_begin : b.s[s].item_begin) <= item) si = s;
+        if ((sample ? b.s[s].sample_group_begin : b.s[s].group_begin) <= g) si = s;
     return si;
 }
 
@@ -323,77 +422,215 @@ __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
     return si;
 }
 
-// ------------------------------------------------- sampled / filtered scan
-// kSample: grid over (session, head, sample tile); writes order keys of the
-// sampled keys.  Otherwise grid over (session, head, tile); appends keys
-// scoring >= theta to the candidate buffer.
-template <int NS, int GP, bool kSample>
-__global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 3)
-scan_kernel(const __grid_constant__ Batch<NS> b)
-{
-    __shared__ ScanSmem<GP> sm;
-    const int item = blockIdx.x;
-    const int si = find_session_by_item(b, item, kSample);
-    const SessionDesc &S = b.s[si];
-    const int local = item - (kSample ? S.sample_item_begin : S.item_begin);
-    const int per_head = kSample ? S.m_tiles : S.n_tiles;
-    const int h = local / per_head;
-    const int ti = local - h * per_head;
-    const int tile = kSample ? ti * S.sample_stride : ti;
-    const int G = b.G, d = b.d;
-    const int q0 = h * G;
+// ----------------------------------------------------------- sampled pass
+// Scores of the sampled keys, latency-first: a CTA takes 16 plane words
+// (512 keys) of one sampled tile, copies every selected plane row of them
+// into shared memory at once, and splits the union channels over four
+// groups of 64 threads (stage st goes to group st % 4); the groups' partial
+// sums are added in group order.  The order keys of all 512 keys (0 past the
+// last key) go to the sample buffer.
+constexpr int kSampleCols = 16;
+constexpr int kSampleGroups = kScanThreads / (kSampleCols * 4);   // 4
+constexpr int kSampleChunks = kTileCols / kSampleCols;            // per sampled tile
+constexpr int kMaxStages = kMaxHeadDim / kStageChannels;          // 32
+typedef uint32_t (*SampleBuf)[kStageRows][kSampleCols];
+constexpr size_t kSampleSmem = (size_t)kMaxStages * kStageRows * kSampleCols * sizeof(uint32_t);
 
+template <int NS, int GP>
+__global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_constant__ Batch<NS> b)
+{
+    __shared__ ScanMeta<GP> sm;
+    extern __shared__ __align__(16) uint32_t sample_dyn[];
+    SampleBuf buf = reinterpret_cast<SampleBuf>(sample_dyn);
+    const int item = blockIdx.x;
+    int si = 0;
+    for (int s2 = 1; s2 < b.n_sessions; ++s2)
+        if (b.s[s2].sample_group_begin <= item) si = s2;     // here: sampled-chunk index
+    const SessionDesc &S = b.s[si];
+    const int per_head = S.m_tiles * kSampleChunks;
+    const int local = item - S.sample_group_begin;
+    const int h = local / per_head;
+    const int ci = local - h * per_head;
+    const int tile_i = ci / kSampleChunks, chunk = ci - tile_i * kSampleChunks;
+    const int col_lo = tile_i * S.sample_stride * kTileCols + chunk * kSampleCols;
+    const int col_hi = min(S.n_cols, col_lo + kSampleCols);
+    const int G = b.G, d = b.d, q0 = h * G;
     setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
                    S.mn + h * d, S.scale + h * d);
-    float2 acc[GP][4];
-    scan_tile<GP>(sm, S.planes, S.n_words, S.n_cols, tile, acc);
+    // every plane row of every stage, 4 x 16 bytes per row
+    const int n_stages = sm.n_stages;
+    const int n_chunks = n_stages * kStageRows * (kSampleCols / 4);
+    for (int e = threadIdx.x; e < n_chunks; e += kScanThreads) {
+        const int row = e >> 2, part = e & 3;          // row over all stages
+        const int col = col_lo + part * 4;
+        const uint32_t g = sm.row_g[row];
+        const bool live = col < col_hi && g != 0xFFFFFFFFu;
+        const uint32_t *src = live ? S.planes + (size_t)g * (size_t)S.n_words + col : S.planes;
+        cp_async16(&buf[row / kStageRows][row % kStageRows][part * 4], src, live ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
 
+    const int grp = threadIdx.x / (kSampleCols * 4);
+    const int lt = threadIdx.x - grp * kSampleCols * 4;
+    const int col = lt >> 2, r = lt & 3;
+    uint32_t sh[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
+    unsigned long long neg[4];
+    magic_negatives(neg);
+    float2 acc[GP][4];
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[g][i] = make_float2(0.0f, 0.0f);
+    for (int st = grp; st < n_stages; st += kSampleGroups) {
+        const int u0 = st * kStageChannels;
+        compute_stage<GP, kSampleCols>(sm, st, buf[st], u0, min(u0 + kStageChannels, sm.U), col,
+                                       sh, neg, acc);
+    }
+    __syncthreads();   // the stage buffer becomes the reduction buffer
+    float2 *red = reinterpret_cast<float2 *>(sample_dyn);    // [groups-1][64][GP*4]
+    if (grp > 0) {
+#pragma unroll
+        for (int g = 0; g < GP; ++g)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                red[((grp - 1) * kSampleCols * 4 + lt) * GP * 4 + g * 4 + i] = acc[g][i];
+    }
+    __syncthreads();
+    if (grp == 0) {
+#pragma unroll
+        for (int o = 1; o < kSampleGroups; ++o)
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 pv = red[((o - 1) * kSampleCols * 4 + lt) * GP * 4 + g * 4 + i];
+                    acc[g][i].x += pv.x;
+                    acc[g][i].y += pv.y;
+                }
+        const int key0 = (col_lo + col) * 32 + r;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+            if (g >= G) break;
+            const float bias = sm.bias[g];
+            uint32_t *dst = S.sample + (size_t)(q0 + g) * S.m_keys + (size_t)tile_i * kTileKeys +
+                            (chunk * kSampleCols + col) * 32 + r;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int j = key0 + 4 * m;
+                dst[4 * m] = (j < S.n && col_lo + col < col_hi)
+                                 ? order_key(score_of(acc[g], m, bias)) : 0u;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------- sampled / filtered scan
+// Persistent: CTA i owns column groups [i*per_cta, (i+1)*per_cta) of the
+// linear (session, KV head, column group) space.  kSample: the space is the
+// sampled tiles' groups and the scores go to the sample buffer; otherwise
+// keys scoring >= theta are appended to the candidate buffer.
+template <int NS, int GP, bool kSample, int STAGES>
+__global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
+scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
+{
+    __shared__ ScanMeta<GP> sm;
+    extern __shared__ __align__(16) uint32_t scan_dyn[];
+    StageBuf stage = reinterpret_cast<StageBuf>(scan_dyn);
+    const int G = b.G, d = b.d;
     const int col = threadIdx.x >> 2, r = threadIdx.x & 3, lane = threadIdx.x & 31;
-    const int key0 = (tile * kTileCols + col) * 32 + r;
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-        if (g >= G) break;
-        const int qq = q0 + g;
-        const float bias = sm.bias[g];
+    int g = blockIdx.x * per_cta;
+    const int g_end = min(total_groups, g + per_cta);
+    int cur_si = -1, cur_h = -1;
+    while (g < g_end) {
+        const int si = find_session_by_group(b, g, kSample);
+        const SessionDesc &S = b.s[si];
+        const int per_head = kSample ? S.m_tiles * kTileGroups : S.col_groups;
+        const int local = g - (kSample ? S.sample_group_begin : S.group_begin);
+        const int h = local / per_head;
+        const int gi = local - h * per_head;
+        // this chunk: balanced split of what is left of the range in this head
+        // (and, when sampling, in this sampled tile), at most 16 groups
+        int avail = min(g_end - g, per_head - gi);
+        int tile_i = 0, tile_off = 0, col_lo;
         if (kSample) {
-            uint32_t *dst = S.sample + (size_t)qq * S.m_keys + (size_t)ti * kTileKeys + col * 32 + r;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int j = key0 + 4 * m;
-                dst[4 * m] = (j < S.n) ? order_key(score_of(acc[g], m, bias)) : 0u;
-            }
+            tile_i = gi / kTileGroups;
+            tile_off = gi - tile_i * kTileGroups;
+            avail = min(avail, kTileGroups - tile_off);
+            col_lo = (tile_i * S.sample_stride) * kTileCols + tile_off * 4;
         } else {
-            const uint32_t theta = S.qstate[qq * kQueryStateWords + 0];
-            uint32_t ok[8];
-            unsigned pass = 0;
+            col_lo = gi * 4;
+        }
+        const int pieces = (avail + kTileGroups - 1) / kTileGroups;
+        const int lim = (avail + pieces - 1) / pieces;
+        const int width = lim * 4;                     // plane words owned by this chunk
+        const int col_hi = min(S.n_cols, col_lo + width);
+        const int q0 = h * G;
+        if (si != cur_si || h != cur_h) {
+            __syncthreads();   // the previous chunk's epilogue may still read sm
+            setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
+                           S.mn + h * d, S.scale + h * d);
+            cur_si = si;
+            cur_h = h;
+        }
+        float2 acc[GP][4];
+        scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
+
+        const bool mine = col < width;
+        const int key0 = (col_lo + col) * 32 + r;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int j = key0 + 4 * m;
-                ok[m] = order_key(score_of(acc[g], m, bias));
-                if (j < S.n && ok[m] >= theta) pass |= 1u << m;
-            }
-            const int cnt = __popc(pass);
-            int inc = cnt;
+        for (int gg = 0; gg < GP; ++gg) {
+            if (gg >= G) break;
+            const int qq = q0 + gg;
+            const float bias = sm.bias[gg];
+            if (kSample) {
+                if (mine) {
+                    uint32_t *dst = S.sample + (size_t)qq * S.m_keys + (size_t)tile_i * kTileKeys +
+                                    (tile_off * 4 + col) * 32 + r;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
-                if (lane >= off) inc += y;
-            }
-            const int total = __shfl_sync(0xFFFFFFFFu, inc, 31);
-            if (total == 0) continue;
-            unsigned base = 0;
-            if (lane == 31) base = atomicAdd(&S.qstate[qq * kQueryStateWords + 1], (unsigned)total);
-            base = __shfl_sync(0xFFFFFFFFu, base, 31);
-            unsigned pos = base + (unsigned)(inc - cnt);
-            unsigned long long *cq = S.cand + (size_t)qq * b.cap;
+                    for (int m = 0; m < 8; ++m) {
+                        const int j = key0 + 4 * m;
+                        dst[4 * m] = (j < S.n && col_lo + col < col_hi)
+                                         ? order_key(score_of(acc[gg], m, bias)) : 0u;
+                    }
+                }
+            } else {
+                const uint32_t theta = S.qstate[qq * kQueryStateWords + 0];
+                uint32_t ok[8];
+                unsigned pass = 0;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                if (pass & (1u << m)) {
-                    if (pos < (unsigned)b.cap) cq[pos] = composite(ok[m], (uint32_t)(key0 + 4 * m));
-                    ++pos;
+                for (int m = 0; m < 8; ++m) {
+                    const int j = key0 + 4 * m;
+                    ok[m] = order_key(score_of(acc[gg], m, bias));
+                    if (mine && col_lo + col < col_hi && j < S.n && ok[m] >= theta) pass |= 1u << m;
+                }
+                const int cnt = __popc(pass);
+                int inc = cnt;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                    if (lane >= off) inc += y;
+                }
+                const int total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+                if (total == 0) continue;
+                unsigned base = 0;
+                if (lane == 31) base = atomicAdd(&S.qstate[qq * kQueryStateWords + 1], (unsigned)total);
+                base = __shfl_sync(0xFFFFFFFFu, base, 31);
+                unsigned pos = base + (unsigned)(inc - cnt);
+                unsigned long long *cq = S.cand + (size_t)qq * b.cap;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    if (pass & (1u << m)) {
+                        if (pos < (unsigned)b.cap) cq[pos] = composite(ok[m], (uint32_t)(key0 + 4 * m));
+                        ++pos;
+                    }
                 }
             }
         }
+        g += lim;
     }
 }
 
@@ -504,16 +741,198 @@ __device__ void write_outputs(const unsigned long long *sel, int k, int32_t *out
     }
 }
 
+// ------------------------------------------------- range-relative radix select
+// Selection over a set held in shared memory by a CTA of kSelThreads threads.
+// Values are composites x = ((okey - lo) << 32) | low, where lo is the set's
+// smallest order key, so the first 11-bit digit already splits the set's own
+// range instead of the fixed sign/exponent bits (and bins stay sparse, so
+// plain shared-memory atomics rarely collide).
+constexpr int kSelThreads = 512;
+constexpr int kSelBits = 11;
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelBinsPerThread = kSelBins / kSelThreads;   // 4
+constexpr int kBitmapMaxKeys = 1 << 20;                     // index-order output via a bitmap
+constexpr int kChunkWords = 8;                              // bitmap words per prefix entry
+
+struct SelShared {
+    unsigned hist[kSelBins];
+    unsigned wsum[kSelThreads / 32];
+    unsigned long long prefix;
+    unsigned krem, above;
+    int bin, cut, done;
+    uint32_t lo, hi;
+};
+
+__device__ __forceinline__ bool high_bits_match(unsigned long long x, unsigned long long p, int top)
+{
+    return top >= 64 || ((x ^ p) >> top) == 0ull;
+}
+
+// Block-wide min / max of order keys (all kSelThreads threads call it).
+__device__ __forceinline__ void sel_range(SelShared &ss, uint32_t lo, uint32_t hi)
+{
+    lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+    hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+    if (threadIdx.x == 0) { ss.lo = 0xFFFFFFFFu; ss.hi = 0u; }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) { atomicMin(&ss.lo, lo); atomicMax(&ss.hi, hi); }
+    __syncthreads();
+}
+
+// Exclusive prefix sum of one value per thread over the block; returns the
+// thread's prefix and writes the total to *total (all threads).
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned *wsum, unsigned *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+        if (lane >= off) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    unsigned before = inc - v, all = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        const unsigned ws = wsum[w];
+        before += (w < warp) ? ws : 0u;
+        all += ws;
+    }
+    __syncthreads();
+    *total = all;
+    return before;
+}
+
+// Which bin (counting from the top) holds the krem-th largest element:
+// above = elements in higher bins < krem <= above + hist[bin].  Thread t
+// owns the kSelBinsPerThread bins just below 2048 - t*kSelBinsPerThread.
+__device__ __forceinline__ void sel_pick(SelShared &ss)
+{
+    const int tid = threadIdx.x;
+    unsigned h[kSelBinsPerThread], mine = 0;
+#pragma unroll
+    for (int i = 0; i < kSelBinsPerThread; ++i) {
+        h[i] = ss.hist[kSelBins - 1 - kSelBinsPerThread * tid - i];
+        mine += h[i];
+    }
+    unsigned total;
+    const unsigned before = block_exclusive_scan(mine, ss.wsum, &total);
+    const unsigned krem = ss.krem;
+    if (before < krem && krem <= before + mine) {
+        unsigned run = before;
+#pragma unroll
+        for (int i = 0; i < kSelBinsPerThread; ++i) {
+            if (run < krem && krem <= run + h[i]) {
+                ss.bin = kSelBins - 1 - kSelBinsPerThread * tid - i;
+                ss.above = run;
+            }
+            run += h[i];
+        }
+    }
+    __syncthreads();
+}
+
+// Runs the digit passes over `count` elements produced by get(i) until the
+// selected set is determined.  Afterwards: selected iff
+// (x >> ss.cut) >= (ss.prefix >> ss.cut).  stop_bit: lowest bit examined.
+template <class Get>
+__device__ void sel_run(SelShared &ss, unsigned count, unsigned k, int top, int stop_bit, Get get)
+{
+    if (threadIdx.x == 0) {
+        ss.prefix = 0ull;
+        ss.krem = k;
+        ss.done = 0;
+        ss.cut = stop_bit;
+    }
+    for (int hi_bit = top; hi_bit > stop_bit; hi_bit -= kSelBits) {
+        const int shift = max(stop_bit, hi_bit - kSelBits);
+        const unsigned width_mask = (1u << (hi_bit - shift)) - 1u;
+#pragma unroll
+        for (int i = 0; i < kSelBinsPerThread; ++i) ss.hist[threadIdx.x + i * kSelThreads] = 0;
+        if (threadIdx.x == 0) { ss.bin = 0; ss.above = 0; }
+        __syncthreads();
+        const unsigned long long pf = ss.prefix;
+        for (unsigned i = threadIdx.x; i < count; i += kSelThreads) {
+            const unsigned long long x = get(i);
+            if (high_bits_match(x, pf, hi_bit)) atomicAdd(&ss.hist[(unsigned)(x >> shift) & width_mask], 1u);
+        }
+        __syncthreads();
+        sel_pick(ss);
+        if (threadIdx.x == 0) {
+            const unsigned b = (unsigned)ss.bin & (kSelBins - 1);
+            ss.krem -= ss.above;
+            ss.prefix |= (unsigned long long)b << shift;
+            if (ss.hist[b] == ss.krem) {
+                ss.done = 1;
+                ss.cut = shift;
+            }
+        }
+        __syncthreads();
+        if (ss.done) break;
+    }
+}
+
+__device__ __forceinline__ int bit_length(uint32_t v) { return v ? 32 - __clz(v) : 0; }
+
+// Writes the k selected composites `sel` (okey << 32 | ~index) to the
+// outputs in ascending key index: a bitmap of the selected indices in
+// shared memory (n_keys <= kBitmapMaxKeys) and one prefix count per
+// kChunkWords bitmap words give each key its output position.  `bm` holds
+// ceil(n/32) words followed by the prefixes.
+__device__ void emit_in_index_order(const unsigned long long *sel, int k, int n, uint32_t *bm,
+                                    unsigned *wsum, int32_t *out_idx, float *out_score)
+{
+    const int words = (n + 31) >> 5;
+    const int chunks = (words + kChunkWords - 1) / kChunkWords;
+    uint32_t *pre = bm + chunks * kChunkWords;
+    for (int w = threadIdx.x; w < chunks * kChunkWords; w += kSelThreads) bm[w] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < k; i += kSelThreads) {
+        const uint32_t j = ~(uint32_t)(sel[i] & 0xFFFFFFFFull);
+        atomicOr(&bm[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    // prefix over chunks: each thread sums a contiguous run of chunks
+    const int per = (chunks + kSelThreads - 1) / kSelThreads;
+    const int c0 = threadIdx.x * per, c1 = min(chunks, c0 + per);
+    unsigned mine = 0;
+    for (int c = c0; c < c1; ++c) {
+        unsigned cc = 0;
+#pragma unroll
+        for (int w = 0; w < kChunkWords; ++w) cc += __popc(bm[c * kChunkWords + w]);
+        pre[c] = cc;
+        mine += cc;
+    }
+    unsigned total;
+    unsigned run = block_exclusive_scan(mine, wsum, &total);
+    for (int c = c0; c < c1; ++c) {
+        const unsigned cc = pre[c];
+        pre[c] = run;
+        run += cc;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < k; i += kSelThreads) {
+        const unsigned long long v = sel[i];
+        const uint32_t j = ~(uint32_t)(v & 0xFFFFFFFFull);
+        const int wj = (int)(j >> 5), c = wj / kChunkWords;
+        unsigned pos = pre[c];
+        for (int w = c * kChunkWords; w < wj; ++w) pos += __popc(bm[w]);
+        pos += __popc(bm[wj] & ((1u << (j & 31)) - 1u));
+        out_idx[pos] = (int32_t)j;
+        out_score[pos] = order_key_to_float((uint32_t)(v >> 32));
+    }
+}
+
 // ---------------------------------------------------------------- theta
-// One CTA per query: theta = the sample_rank-th largest sampled order key
-// (4 radix passes over the sample held in shared memory), and reset the
-// candidate count and fallback flag.
+// One CTA per query: theta = the sample_rank-th largest sampled order key,
+// and reset the candidate count and fallback flag.
 template <int NS>
-__global__ void __launch_bounds__(1024) theta_kernel(const __grid_constant__ Batch<NS> b,
-                                                     uint32_t force_exact)
+__global__ void __launch_bounds__(kSelThreads) theta_kernel(const __grid_constant__ Batch<NS> b,
+                                                            uint32_t force_exact)
 {
     extern __shared__ uint32_t vals[];
-    __shared__ SelectState ss;
+    __shared__ SelShared ss;
     const int gq = blockIdx.x;
     const int si = find_session_by_query(b, gq);
     const SessionDesc &S = b.s[si];
@@ -528,31 +947,35 @@ __global__ void __launch_bounds__(1024) theta_kernel(const __grid_constant__ Bat
         return;
     }
     const int m = S.m_keys;
-    const uint32_t *src = S.sample + (size_t)qq * m;
-    for (int i = threadIdx.x; i < m; i += blockDim.x) vals[i] = src[i];
-    select_reset(ss, (unsigned)S.sample_rank);
-    __syncthreads();
-    for (int digit = 3; digit >= 0; --digit) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) ss.hist[i] = 0;
-        __syncthreads();
-        const uint32_t pm = (uint32_t)ss.pmask, pf = (uint32_t)ss.prefix;
-        for (int i = threadIdx.x; i < m; i += blockDim.x) {
-            const uint32_t v = vals[i];
-            if ((v & pm) == pf) atomicAdd(&ss.hist[(v >> (8 * digit)) & 0xFFu], 1u);
-        }
-        __syncthreads();
-        select_step(ss, digit);
+    const uint4 *src = reinterpret_cast<const uint4 *>(S.sample + (size_t)qq * m);
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = threadIdx.x; i < m / 4; i += kSelThreads) {
+        const uint4 v = src[i];
+        reinterpret_cast<uint4 *>(vals)[i] = v;
+        lo = min(min(lo, min(v.x, v.y)), min(v.z, v.w));
+        hi = max(max(hi, max(v.x, v.y)), max(v.z, v.w));
     }
-    if (threadIdx.x == 0) { st[0] = (uint32_t)ss.prefix; st[1] = 0; st[2] = 0; }
+    sel_range(ss, lo, hi);
+    const uint32_t base = ss.lo;
+    const int top = 32 + bit_length(ss.hi - base);
+    sel_run(ss, (unsigned)m, (unsigned)S.sample_rank, top, 32,
+            [&](unsigned i) { return (unsigned long long)(vals[i] - base) << 32; });
+    if (threadIdx.x == 0) {
+        st[0] = base + (uint32_t)(ss.prefix >> 32);
+        st[1] = 0;
+        st[2] = 0;
+    }
 }
 
 // ---------------------------------------------------------------- final
-// One CTA per query: exact top-k of the candidates when k <= count <= cap.
+// One CTA per query: exact top-k of the candidates when k <= count <= cap,
+// written in ascending key index.  Shared memory: the selected k (kMaxFastK
+// composites), then the candidates, later reused for the index bitmap.
 template <int NS>
-__global__ void __launch_bounds__(1024) final_kernel(const __grid_constant__ Batch<NS> b)
+__global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constant__ Batch<NS> b)
 {
     extern __shared__ unsigned long long dyn[];
-    __shared__ SelectState ss;
+    __shared__ SelShared ss;
     const int gq = blockIdx.x;
     const int si = find_session_by_query(b, gq);
     const SessionDesc &S = b.s[si];
@@ -566,37 +989,49 @@ __global__ void __launch_bounds__(1024) final_kernel(const __grid_constant__ Bat
         if (threadIdx.x == 0) st[2] = 1;
         return;
     }
-    unsigned long long *x = dyn;              // [cap]
-    unsigned long long *sel = dyn + b.cap;    // [kpad]
+    unsigned long long *sel = dyn;                  // [kMaxFastK]
+    unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the bitmap
     const unsigned long long *cq = S.cand + (size_t)qq * b.cap;
-    for (unsigned i = threadIdx.x; i < cnt; i += blockDim.x) x[i] = cq[i];
-    select_reset(ss, (unsigned)k);
-    __syncthreads();
-    for (int digit = 7; digit >= 0; --digit) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) ss.hist[i] = 0;
-        __syncthreads();
-        const unsigned long long pm = ss.pmask, pf = ss.prefix;
-        for (unsigned i = threadIdx.x; i < cnt; i += blockDim.x) {
-            const unsigned long long v = x[i];
-            if ((v & pm) == pf) atomicAdd(&ss.hist[(unsigned)(v >> (8 * digit)) & 0xFFu], 1u);
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (unsigned i = 2 * threadIdx.x; i < cnt; i += 2 * kSelThreads) {
+        unsigned long long v0, v1 = 0ull;
+        if (i + 1 < cnt) {
+            const ulonglong2 p = *reinterpret_cast<const ulonglong2 *>(cq + i);
+            v0 = p.x;
+            v1 = p.y;
+            x[i + 1] = v1;
+            lo = min(lo, (uint32_t)(v1 >> 32));
+            hi = max(hi, (uint32_t)(v1 >> 32));
+        } else {
+            v0 = cq[i];
         }
-        __syncthreads();
-        select_step(ss, digit);
-        if (ss.done) break;
+        x[i] = v0;
+        lo = min(lo, (uint32_t)(v0 >> 32));
+        hi = max(hi, (uint32_t)(v0 >> 32));
     }
-    const int shift = ss.shift;
-    const unsigned long long lim = ss.prefix >> shift;
-    for (unsigned i = threadIdx.x; i < cnt; i += blockDim.x) {
+    sel_range(ss, lo, hi);
+    const unsigned long long base = (unsigned long long)ss.lo << 32;
+    const int top = 32 + bit_length(ss.hi - ss.lo);
+    sel_run(ss, cnt, (unsigned)k, top, 0, [&](unsigned i) { return x[i] - base; });
+    // compact exactly the k selected, in candidate order (block scan)
+    const int cut = ss.cut;
+    const unsigned long long lim = ss.prefix >> cut;
+    const unsigned per = (cnt + kSelThreads - 1) / kSelThreads;
+    const unsigned i0 = threadIdx.x * per, i1 = min(cnt, i0 + per);
+    unsigned mine = 0;
+    for (unsigned i = i0; i < i1; ++i) mine += ((x[i] - base) >> cut) >= lim;
+    unsigned total;
+    unsigned pos = block_exclusive_scan(mine, ss.wsum, &total);
+    for (unsigned i = i0; i < i1; ++i) {
         const unsigned long long v = x[i];
-        if ((v >> shift) >= lim) {
-            const unsigned slot = atomicAdd(&ss.nsel, 1u);
-            if (slot < (unsigned)k) sel[slot] = v;
+        if (((v - base) >> cut) >= lim) {
+            if (pos < (unsigned)k) sel[pos] = v;
+            ++pos;
         }
     }
-    for (int i = k + threadIdx.x; i < b.kpad; i += blockDim.x) sel[i] = 0ull;
     __syncthreads();
-    bitonic_sort_desc(sel, b.kpad);
-    write_outputs(sel, k, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
+    emit_in_index_order(sel, k, S.n, reinterpret_cast<uint32_t *>(x), ss.wsum,
+                        S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
 }
 
 // ------------------------------------------------------------- fallback
@@ -606,9 +1041,12 @@ __global__ void __launch_bounds__(1024) final_kernel(const __grid_constant__ Bat
 template <int NS>
 __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_constant__ Batch<NS> b)
 {
-    __shared__ ScanSmem<1> sm;
+    __shared__ ScanMeta<1> sm;
     __shared__ SelectState ss;
-    extern __shared__ unsigned long long sel[];   // [kpad]
+    extern __shared__ __align__(16) uint32_t fb_dyn[];
+    StageBuf stage = reinterpret_cast<StageBuf>(fb_dyn);
+    unsigned long long *sel =
+        reinterpret_cast<unsigned long long *>(fb_dyn + kMainStages * kStageRows * kTileCols);
     const int gq = blockIdx.x;
     const int si = find_session_by_query(b, gq);
     const SessionDesc &S = b.s[si];
@@ -626,13 +1064,14 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
         for (int i = threadIdx.x; i < 256; i += blockDim.x) ss.hist[i] = 0;
         __syncthreads();
         const unsigned long long pm = ss.pmask, pf = ss.prefix;
-        for (int tile = 0; tile < S.n_tiles; ++tile) {
-            scan_tile<1>(sm, S.planes, S.n_words, S.n_cols, tile, acc);
-            const int key0 = (tile * kTileCols + col) * 32 + r;
+        for (int c0 = 0; c0 < S.n_cols; c0 += kTileCols) {
+            const int c1 = min(S.n_cols, c0 + kTileCols);
+            scan_chunk<1, kMainStages>(sm, stage, S.planes, S.n_words, c0, c1, acc);
+            const int key0 = (c0 + col) * 32 + r;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int j = key0 + 4 * m;
-                if (j < S.n) {
+                if (c0 + col < c1 && j < S.n) {
                     const unsigned long long v =
                         composite(order_key(score_of(acc[0], m, bias)), (uint32_t)j);
                     if ((v & pm) == pf) atomicAdd(&ss.hist[(unsigned)(v >> (8 * digit)) & 0xFFu], 1u);
@@ -645,13 +1084,14 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
     }
     const int shift = ss.shift;
     const unsigned long long lim = ss.prefix >> shift;
-    for (int tile = 0; tile < S.n_tiles; ++tile) {
-        scan_tile<1>(sm, S.planes, S.n_words, S.n_cols, tile, acc);
-        const int key0 = (tile * kTileCols + col) * 32 + r;
+    for (int c0 = 0; c0 < S.n_cols; c0 += kTileCols) {
+        const int c1 = min(S.n_cols, c0 + kTileCols);
+        scan_chunk<1, kMainStages>(sm, stage, S.planes, S.n_words, c0, c1, acc);
+        const int key0 = (c0 + col) * 32 + r;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int j = key0 + 4 * m;
-            if (j < S.n) {
+            if (c0 + col < c1 && j < S.n) {
                 const unsigned long long v = composite(order_key(score_of(acc[0], m, bias)), (uint32_t)j);
                 if ((v >> shift) >= lim) {
                     const unsigned slot = atomicAdd(&ss.nsel, 1u);
@@ -660,10 +1100,17 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
             }
         }
     }
+    // ascending key index: sort the k selected by ~index, descending
+    __syncthreads();   // every selected composite has been written
+    for (int i = threadIdx.x; i < k; i += blockDim.x) sel[i] = (sel[i] << 32) | (sel[i] >> 32);
     for (int i = k + threadIdx.x; i < b.kpad; i += blockDim.x) sel[i] = 0ull;
     __syncthreads();
     bitonic_sort_desc(sel, b.kpad);
-    write_outputs(sel, k, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
+    for (int i = threadIdx.x; i < k; i += blockDim.x) {
+        const unsigned long long v = sel[i];
+        S.out_idx[(size_t)qq * k + i] = (int32_t)(~(uint32_t)(v >> 32));
+        S.out_score[(size_t)qq * k + i] = order_key_to_float((uint32_t)(v & 0xFFFFFFFFull));
+    }
 }
 
 // ------------------------------------------------------------- host side
@@ -692,7 +1139,7 @@ Sizing size_session(int n, int n_words, int k)
     z.n_cols = std::min(n_words, ceil_div(ceil_div(n, 32), 4) * 4);
     z.n_tiles = ceil_div(z.n_cols, kTileCols);
     const int cap = capacity_for(std::min(k, kMaxFastK));
-    z.exact_only = (k > kMaxFastK) ? 1 : 0;
+    z.exact_only = (k > kMaxFastK || n > kBitmapMaxKeys) ? 1 : 0;
     if (z.exact_only || n <= cap) return z;
     const double target = (double)kSampleTargetRank * (double)n / (2.0 * (double)k);
     int m = (int)std::min<double>(std::max<double>(target, kSampleMinKeys), kSampleMaxKeys);
@@ -728,46 +1175,141 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     return L;
 }
 
+// Per-device cache of one kernel's resident CTAs (after raising its dynamic
+// shared-memory limit once).
+struct LaunchCache {
+    int slots[64] = {0};
+};
+
+template <class Kernel>
+cudaError_t resident_slots(LaunchCache &cache, Kernel kernel, size_t dyn_smem, int *slots)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (cache.slots[dev] == 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0, n_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanThreads, dyn_smem);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        cache.slots[dev] = std::max(1, per_sm) * std::max(1, n_sm);
+    }
+    *slots = cache.slots[dev];
+    return cudaSuccess;
+}
+
+// Raise a kernel's dynamic shared-memory limit to its largest possible need,
+// once per device.  `done` must belong to that kernel alone.
+template <class Kernel>
+cudaError_t ensure_smem(int (&done)[64], Kernel kernel, size_t max_bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)max_bytes);
+        if (e != cudaSuccess) return e;
+        done[dev] = 1;
+    }
+    return cudaSuccess;
+}
+
+// One set of "limit raised" flags per kernel instantiation.
+template <int NS>
+struct SmemFlags {
+    static int theta[64], final_[64], fallback[64];
+};
+template <int NS> int SmemFlags<NS>::theta[64];
+template <int NS> int SmemFlags<NS>::final_[64];
+template <int NS> int SmemFlags<NS>::fallback[64];
+
+constexpr size_t kStageBytes = (size_t)kStageRows * kTileCols * sizeof(uint32_t);
+
+// Shared-memory bytes of the index-order bitmap and its chunk prefixes.
+inline size_t bitmap_bytes_for(int n)
+{
+    const size_t words = ((size_t)n + 31) / 32;
+    const size_t chunks = (words + kChunkWords - 1) / kChunkWords;
+    return (chunks * kChunkWords + chunks) * sizeof(uint32_t);
+}
+
+template <int NS>
+size_t final_bitmap_bytes(const Batch<NS> &bt)
+{
+    size_t m = 0;
+    for (int s = 0; s < bt.n_sessions; ++s) m = std::max(m, bitmap_bytes_for(bt.s[s].n));
+    return m;
+}
+
 template <int NS, int GP>
-cudaError_t run_batch(const Batch<NS> &bt, int total_items, int total_sample_items,
+cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_groups,
                       int total_queries, int max_m_keys, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
 {
+    static LaunchCache sample_cache, main_cache;   // these kernels depend on GP too
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
     int launches = 0;
-    if (!force && total_sample_items > 0) {
-        scan_kernel<NS, GP, true><<<total_sample_items, kScanThreads, 0, stream>>>(bt);
+    if (!force && total_sample_groups > 0) {
+        static int sample_smem_set[64];
+        if ((e = ensure_smem(sample_smem_set, sample_kernel<NS, GP>, kSampleSmem)) != cudaSuccess)
+            return note_error(e, "sample set-up");
+        const int ctas = total_sample_groups;   // one CTA per sampled 16-word chunk
+        sample_kernel<NS, GP><<<ctas, kScanThreads, kSampleSmem, stream>>>(bt);
+        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "sample launch");
         ++launches;
     }
     const size_t theta_smem = (size_t)max_m_keys * sizeof(uint32_t);
-    e = cudaFuncSetAttribute(theta_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max<size_t>(theta_smem, 1));
-    if (e != cudaSuccess) return e;
-    theta_kernel<NS><<<total_queries, 1024, theta_smem, stream>>>(bt, force ? 1u : 0u);
+    if ((e = ensure_smem(SmemFlags<NS>::theta, theta_kernel<NS>,
+                         (size_t)kSampleMaxKeys * sizeof(uint32_t))) != cudaSuccess)
+        return note_error(e, "theta set-up");
+    theta_kernel<NS><<<total_queries, kSelThreads, theta_smem, stream>>>(bt, force ? 1u : 0u);
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "theta launch");
     ++launches;
-    if (!force && total_items > 0) {
+    if (!force && total_groups > 0) {
+        auto kern = scan_kernel<NS, GP, false, kMainStages>;
+        const size_t dyn = kMainStages * kStageBytes;
+        int slots = 0;
+        if ((e = resident_slots(main_cache, kern, dyn, &slots)) != cudaSuccess)
+            return note_error(e, "scan set-up");
+        (void)slots;
+        const int per_cta = kTileGroups;   // one 64-word chunk per CTA (4 resident per SM)
+        const int ctas = (total_groups + per_cta - 1) / per_cta;
         if (hook && hook->enabled) cudaEventRecord(hook->begin, stream);
-        scan_kernel<NS, GP, false><<<total_items, kScanThreads, 0, stream>>>(bt);
+        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, per_cta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
         if (hook && hook->enabled) {
             cudaEventRecord(hook->end, stream);
             hook->recorded = true;
         }
         ++launches;
     }
-    const size_t final_smem = ((size_t)bt.cap + bt.kpad) * sizeof(unsigned long long);
-    e = cudaFuncSetAttribute(final_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)final_smem);
-    if (e != cudaSuccess) return e;
-    final_kernel<NS><<<total_queries, 1024, final_smem, stream>>>(bt);
-    const size_t fb_smem = (size_t)bt.kpad * sizeof(unsigned long long);
-    e = cudaFuncSetAttribute(fallback_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)fb_smem);
-    if (e != cudaSuccess) return e;
+    const size_t bitmap_bytes = final_bitmap_bytes(bt);
+    const size_t final_smem = kMaxFastK * sizeof(unsigned long long) +
+                              std::max((size_t)bt.cap * sizeof(unsigned long long), bitmap_bytes);
+    if ((e = ensure_smem(SmemFlags<NS>::final_, final_kernel<NS>,
+                         kMaxFastK * sizeof(unsigned long long) +
+                             std::max((size_t)capacity_for(kMaxFastK) * sizeof(unsigned long long),
+                                      bitmap_bytes_for(kBitmapMaxKeys)))) != cudaSuccess)
+        return note_error(e, "final set-up");
+    final_kernel<NS><<<total_queries, kSelThreads, final_smem, stream>>>(bt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "final launch");
+    const size_t fb_smem = kMainStages * kStageBytes + (size_t)bt.kpad * sizeof(unsigned long long);
+    if ((e = ensure_smem(SmemFlags<NS>::fallback, fallback_kernel<NS>,
+                         kMainStages * kStageBytes + (size_t)kMaxK * sizeof(unsigned long long))) !=
+        cudaSuccess)
+        return note_error(e, "fallback set-up");
     fallback_kernel<NS><<<total_queries, kScanThreads, fb_smem, stream>>>(bt);
     launches += 2;
     note_launch(launches);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "fallback launch");
+    return cudaSuccess;
 }
 
 template <int NS>
@@ -783,7 +1325,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int items = 0, sitems = 0, queries = 0, max_m = 0;
+    int groups = 0, sgroups = 0, queries = 0, max_m = 0;
     size_t at = 0;
     char *base = static_cast<char *>(ws);
     for (int s = 0; s < n_sessions; ++s) {
@@ -807,25 +1349,25 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.n = ix.n_keys;
         D.n_words = ix.n_words;
         D.n_cols = z.n_cols;
-        D.n_tiles = z.n_tiles;
+        D.col_groups = z.n_cols / 4;
         D.m_tiles = z.m_tiles;
         D.sample_stride = z.stride;
         D.m_keys = z.m_keys;
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
-        D.item_begin = items;
-        D.sample_item_begin = sitems;
+        D.group_begin = groups;
+        D.sample_group_begin = sgroups;
         D.q_begin = queries;
-        items += D.H * D.n_tiles;
-        sitems += D.H * D.m_tiles;
+        groups += D.H * D.col_groups;
+        sgroups += D.H * D.m_tiles * kSampleChunks;   // sampled 16-word chunks
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, items, sitems, queries, max_m, flags, stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, items, sitems, queries, max_m, flags, stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, items, sitems, queries, max_m, flags, stream, hook);
-    return run_batch<NS, 8>(bt, items, sitems, queries, max_m, flags, stream, hook);
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
+    return run_batch<NS, 8>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
 }
 
 }  // namespace

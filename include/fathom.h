@@ -38,8 +38,9 @@
  *       t         uint8 [Q][d] bits read per channel; t_union uint8 [H][d]
  *       bytes     uint64 [Q + H]: per query, then per KV head (union)
  *       out_idx   int32 [Q][k], out_score float32 [Q][k]: the k keys of
- *                 largest score, ordered by score descending and then key
- *                 index ascending
+ *                 largest score (ties to the lower key index), listed in
+ *                 ascending key index (the order a gather of their K/V rows
+ *                 wants), each with its score
  *   - head_dim is a multiple of 32 and at most 256; G is 1..8;
  *     n_words is a multiple of 4 (16-byte plane rows) with 32*n_words >= n;
  *     1 <= k <= min(n, 4096).
@@ -166,7 +167,8 @@ size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k);
  *   s_gj = sum_c q_gc * (mn_c + scale_c*(2^(4-t)*u + (2^(4-t)-1)/2)),
  *   t = t_gc, u = code_cj >> (4-t)
  * (the key rebuilt at the middle of its coarse t-bit bin), accumulated in
- * float32.  Outputs the k keys of largest s, ties to the lower index.
+ * float32.  Outputs the k keys of largest s, ties to the lower index,
+ * listed in ascending key index.
  * q_bf16, t, t_union, out_idx, out_score, workspace: device pointers.
  * flags: FATHOM_SCAN_* bits. */
 fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,

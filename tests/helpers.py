@@ -29,7 +29,7 @@ def check_topk(gpu_idx, gpu_score, s, a, k, rtol=SCORE_RTOL):
     * every returned score within rtol * A_j of the oracle's score of that key;
     * the set equals the oracle's top-k except for keys whose oracle score is
       within rtol * A of the oracle's k-th score (both sides, equal size);
-    * order: scores non-increasing, equal scores by ascending index.
+    * order: ascending key index.
     Returns the number of keys that differ (inside the tie band)."""
     gpu_idx = np.asarray(gpu_idx, dtype=np.int64)
     gpu_score = np.asarray(gpu_score, dtype=np.float64)
@@ -49,7 +49,5 @@ def check_topk(gpu_idx, gpu_score, s, a, k, rtol=SCORE_RTOL):
         band = rtol * max(a[j], a[ref_idx[-1]])
         assert abs(s[j] - kth) <= band, (f"key {j} (oracle score {s[j]}) differs from the "
                                          f"oracle top-{k} outside the tie band (k-th {kth})")
-    assert np.all(np.diff(gpu_score) <= 0), "scores not in descending order"
-    same = np.diff(gpu_score) == 0
-    assert np.all(np.diff(gpu_idx)[same] > 0), "equal scores not in ascending index order"
+    assert np.all(np.diff(gpu_idx) > 0), "indices not in ascending order"
     return len(diff) // 2
