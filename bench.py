@@ -58,6 +58,8 @@ def parse_args():
     p.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
     p.add_argument("--workload", choices=tuple(WORKLOADS), default="qwen3_8b_layer_128k")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--graph", type=int, default=1,
+                   help="replay the timed steps as one CUDA graph (1) or launch them eagerly (0)")
     p.add_argument("--heat-seconds", type=float, default=1.0,
                    help="minimum warm-up duration (load for the clock sampler); 0 for "
                         "profiler runs, which then see exactly --warmup warm-up steps")
@@ -134,6 +136,34 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+# ------------------------------------------------------------ host link
+def measure_host_link(fp, torch, nbytes=1 << 30, reps=10):
+    """Host->device link peaks measured in this run: a pinned host->device
+    copy of `nbytes` and a zero-copy read kernel over the same pinned buffer
+    (best of `reps` each, CUDA events)."""
+    host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dev = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best_copy = best_zero = 0.0
+    for _ in range(reps):
+        a.record()
+        dev.copy_(host, non_blocking=True)
+        b.record()
+        b.synchronize()
+        best_copy = max(best_copy, nbytes / (a.elapsed_time(b) / 1e3) / 1e9)
+    for _ in range(reps):
+        a.record()
+        fp.fathom_link_probe(host, nbytes, sink)
+        b.record()
+        b.synchronize()
+        best_zero = max(best_zero, nbytes / (a.elapsed_time(b) / 1e3) / 1e9)
+    del host, dev
+    return {"h2d_memcpy_gbs": best_copy, "zero_copy_read_gbs": best_zero,
+            "how": f"pinned host->device copy and zero-copy read kernel over {nbytes >> 20} MiB, "
+                   f"best of {reps}, CUDA events"}
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -224,6 +254,7 @@ def run_fathom(args, wl_name, wl):
     torch.cuda.synchronize()
     assert fp.fathom_last_device_status() == fp.FATHOM_OK
 
+    link = measure_host_link(fp, torch) if wl["residency"] != "device" else None
     W, K = max(3, args.warmup), args.steps
     qsets = synth.draw_queries(10_000 + rank, Q, d, count=W + K)
     q_dev = torch.from_numpy(qsets.view(np.int16)).cuda()
@@ -248,25 +279,47 @@ def run_fathom(args, wl_name, wl):
     status = fp.fathom_last_device_status()
     assert status == fp.FATHOM_OK, fp.status_str(status)
 
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K)]
+
+    def timed_steps():
+        for s in range(K):
+            flush.fill_(s & 0xFF)               # L2 flush, outside the step's events
+            ev[s][0].record()
+            step(W + s, fp.FATHOM_SCAN_PROFILE)
+            ev[s][1].record()
+
     launches0 = fp.fathom_launch_count()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    for s in range(K):
-        flush.fill_(s & 0xFF)
-        ev[s][0].record()
-        step(W + s, fp.FATHOM_SCAN_PROFILE)
-        ev[s][1].record()
+    graph = None
+    if args.graph:
+        # the K timed steps as one CUDA graph (kernels, flushes and events are
+        # all nodes; every step still runs all of its work)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+                timed_steps()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+    launches = fp.fathom_launch_count() - launches0
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if graph is not None:
+        graph.replay()
+    else:
+        timed_steps()
+        launches = fp.fathom_launch_count() - launches0
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    launches = fp.fathom_launch_count() - launches0
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
     scan_ms, scan_launches = fp.fathom_profile_read()
+    if graph is not None:
+        del graph
     status = fp.fathom_last_device_status()
     assert status == fp.FATHOM_OK, fp.status_str(status)
 
@@ -326,14 +379,18 @@ def run_fathom(args, wl_name, wl):
     value = keys_per_step * K * world / (total_ms / 1e3) / 1e9
     e2e_value = keys_per_step * K * world / e2e_total / 1e9
 
-    peak, peak_src = load_peaks()
     bytes_per_launch = union_bytes_total / len(budgets)
     avg_launch_ms = scan_ms / max(1, scan_launches)
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm" if wl["residency"] == "device" else "host_link",
-                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None, "kernel": "scan_kernel (filter pass)",
-                "peak_source": f"{peak_src} hbm_gbs", "avg_launch_us": avg_launch_ms * 1e3,
+    if wl["residency"] == "device":
+        peak, peak_src = load_peaks()
+        bound, peak_note = "hbm", f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"
+    else:
+        peak = max(link["h2d_memcpy_gbs"], link["zero_copy_read_gbs"])
+        bound, peak_note = "host_link", "measured in this run: max(pinned copy, zero-copy read)"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None, "kernel": "scan_kernel (filter pass)",
+                "peak_source": peak_note, "avg_launch_us": avg_launch_ms * 1e3,
                 "algorithmic_bytes_per_launch": bytes_per_launch}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -342,9 +399,12 @@ def run_fathom(args, wl_name, wl):
             "config": config_of(wl_name, wl, "flushed between steps (256 MiB write)"),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": int(launches), "roofline": roofline, "clocks": clk,
+            "gpu_launches": int(launches), "launch_mode": "cuda_graph" if args.graph else "eager",
+            "roofline": roofline, "clocks": clk,
             "per_budget": per_budget,
             "step_ms_median": statistics.median(step_ms)}
+    if link is not None:
+        line["host_link"] = link
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(ses, wl)
     if rank == 0:

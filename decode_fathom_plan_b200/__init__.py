@@ -37,7 +37,7 @@ EXPORTED = (
     "fathom_plan", "fathom_fixed_plan", "fathom_scan_workspace_bytes", "fathom_scan_topk",
     "fathom_scan_batched_workspace_bytes", "fathom_scan_topk_batched",
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
-    "fathom_scan_topk_static",
+    "fathom_scan_topk_static", "fathom_link_probe",
 )
 
 
@@ -87,6 +87,7 @@ def load_library(path: str = LIB_PATH):
         "fathom_scan_topk_batched": ([IX, I32, P, P, P, I32, P, P, P, SZ, U32, P], ctypes.c_int),
         "fathom_last_device_status": ([P], ctypes.c_int),
         "fathom_launch_count": ([], ctypes.c_uint64),
+        "fathom_link_probe": ([P, SZ, P, P], ctypes.c_int),
         "fathom_profile_read": ([ctypes.POINTER(ctypes.c_double),
                                  ctypes.POINTER(ctypes.c_uint64)], ctypes.c_int),
     }
@@ -207,6 +208,12 @@ def fathom_scan_topk_batched(sessions: Sequence[fathom_index], q_bf16, t, t_unio
 
 def fathom_last_device_status(stream=None) -> int:
     return int(load_library().fathom_last_device_status(_stream(stream)))
+
+
+def fathom_link_probe(buffer, nbytes: int, sink, stream=None):
+    """Zero-copy read of `nbytes` of a pinned host (or device) buffer."""
+    _check(load_library().fathom_link_probe(_ptr(buffer), int(nbytes), _ptr(sink),
+                                            _stream(stream)), "fathom_link_probe")
 
 
 def fathom_launch_count() -> int:

@@ -1281,11 +1281,12 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
         (void)slots;
         const int per_cta = kTileGroups;   // one 64-word chunk per CTA (4 resident per SM)
         const int ctas = (total_groups + per_cta - 1) / per_cta;
-        if (hook && hook->enabled) cudaEventRecord(hook->begin, stream);
+        // external records stay timing records when the stream is being captured
+        if (hook && hook->enabled) cudaEventRecordWithFlags(hook->begin, stream, cudaEventRecordExternal);
         kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, per_cta);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
         if (hook && hook->enabled) {
-            cudaEventRecord(hook->end, stream);
+            cudaEventRecordWithFlags(hook->end, stream, cudaEventRecordExternal);
             hook->recorded = true;
         }
         ++launches;

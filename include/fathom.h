@@ -236,6 +236,15 @@ uint64_t fathom_launch_count(void);
  * forgets them.  Not thread-safe; benchmarking only. */
 fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_launches);
 
+/* Instrumentation: read `bytes` (>= 16, a multiple of 16 is read in full)
+ * of `buffer` -- a pinned, device-mapped host buffer, or device memory --
+ * with 16-byte loads from every SM, the access pattern of the host-resident
+ * scan, so the zero-copy read bandwidth of the host link can be measured
+ * with events around the call.  `sink` is a device word the kernel may
+ * increment (keeps the loads).  buffer must be 16-byte aligned. */
+fathom_status fathom_link_probe(const void *buffer, size_t bytes, unsigned long long *sink,
+                                cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
