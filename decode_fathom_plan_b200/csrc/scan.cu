@@ -66,6 +66,7 @@ namespace {
 
 constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-word chunk
 constexpr int kMainStages = 3;
+constexpr int kHostStages = 6;   // host-resident planes: more bytes in flight per CTA
 constexpr int kSampleStages = 8;
 
 struct SessionDesc {
@@ -81,7 +82,7 @@ struct SessionDesc {
     uint32_t *sample;            // [Q][m_keys]
     unsigned long long *cand;    // [Q][cap]
     int H, n, n_words, n_cols, col_groups;
-    int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
+    int m_tiles, sample_stride, m_keys, sample_rank, exact_only, host_resident;
     int group_begin, sample_group_begin, q_begin;
 };
 
@@ -111,12 +112,22 @@ struct alignas(16) ScanMeta {
 typedef uint32_t (*StageBuf)[kStageRows][kTileCols];
 
 // ------------------------------------------------------------ small helpers
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
+// Plain 16-byte copy (no source-size operand).
+__device__ __forceinline__ void cp_async16_full(void *smem, const void *gmem)
 {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
-                 "r"(src_bytes)
-                 : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+// 16 bytes of plane data, or zeros where there is none (a row past the
+// channel's depth, or a column past the chunk): a plain copy for live data,
+// a shared-memory store of zeros otherwise, so no global request is issued
+// for zero rows.  The zeros are visible after the stage's barrier.
+__device__ __forceinline__ void copy_or_zero16(void *smem, const void *gmem, bool live)
+{
+    if (live)
+        cp_async16_full(smem, gmem);
+    else
+        *reinterpret_cast<uint4 *>(smem) = make_uint4(0u, 0u, 0u, 0u);
 }
 __device__ __forceinline__ void cp_async_commit()
 {
@@ -272,8 +283,7 @@ __device__ __forceinline__ void load_stage(const ScanMeta<GP> &sm, StageBuf stag
     for (int row = threadIdx.x >> 4; row < kStageRows; row += kScanThreads / 16) {
         const uint32_t g = rows[row];
         const bool live = ok && g != 0xFFFFFFFFu;
-        const uint32_t *src = live ? planes + (size_t)g * (size_t)n_words + col : planes;
-        cp_async16(&stage[buf][row][chunk * 4], src, live ? 16 : 0);
+        copy_or_zero16(&stage[buf][row][chunk * 4], planes + (size_t)g * (size_t)n_words + col, live);
     }
 }
 
@@ -465,8 +475,8 @@ __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_const
         const int col = col_lo + part * 4;
         const uint32_t g = sm.row_g[row];
         const bool live = col < col_hi && g != 0xFFFFFFFFu;
-        const uint32_t *src = live ? S.planes + (size_t)g * (size_t)S.n_words + col : S.planes;
-        cp_async16(&buf[row / kStageRows][row % kStageRows][part * 4], src, live ? 16 : 0);
+        copy_or_zero16(&buf[row / kStageRows][row % kStageRows][part * 4],
+                       S.planes + (size_t)g * (size_t)S.n_words + col, live);
     }
     cp_async_commit();
     cp_async_wait<0>();
@@ -1175,33 +1185,6 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     return L;
 }
 
-// Per-device cache of one kernel's resident CTAs (after raising its dynamic
-// shared-memory limit once).
-struct LaunchCache {
-    int slots[64] = {0};
-};
-
-template <class Kernel>
-cudaError_t resident_slots(LaunchCache &cache, Kernel kernel, size_t dyn_smem, int *slots)
-{
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (cache.slots[dev] == 0) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
-        if (e != cudaSuccess) return e;
-        int per_sm = 0, n_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanThreads, dyn_smem);
-        if (e != cudaSuccess) return e;
-        e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        cache.slots[dev] = std::max(1, per_sm) * std::max(1, n_sm);
-    }
-    *slots = cache.slots[dev];
-    return cudaSuccess;
-}
-
 // Raise a kernel's dynamic shared-memory limit to its largest possible need,
 // once per device.  `done` must belong to that kernel alone.
 template <class Kernel>
@@ -1231,6 +1214,17 @@ template <int NS> int SmemFlags<NS>::fallback[64];
 
 constexpr size_t kStageBytes = (size_t)kStageRows * kTileCols * sizeof(uint32_t);
 
+// Record a timing event; inside a stream capture it must be an external
+// record to stay a timing record in the graph (the flag is invalid outside).
+inline void record_timing_event(cudaEvent_t ev, cudaStream_t stream)
+{
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, stream);
+}
+
 // Shared-memory bytes of the index-order bitmap and its chunk prefixes.
 inline size_t bitmap_bytes_for(int n)
 {
@@ -1252,7 +1246,6 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
                       int total_queries, int max_m_keys, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
 {
-    static LaunchCache sample_cache, main_cache;   // these kernels depend on GP too
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
     int launches = 0;
@@ -1273,20 +1266,27 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "theta launch");
     ++launches;
     if (!force && total_groups > 0) {
-        auto kern = scan_kernel<NS, GP, false, kMainStages>;
-        const size_t dyn = kMainStages * kStageBytes;
-        int slots = 0;
-        if ((e = resident_slots(main_cache, kern, dyn, &slots)) != cudaSuccess)
-            return note_error(e, "scan set-up");
-        (void)slots;
-        const int per_cta = kTileGroups;   // one 64-word chunk per CTA (4 resident per SM)
-        const int ctas = (total_groups + per_cta - 1) / per_cta;
-        // external records stay timing records when the stream is being captured
-        if (hook && hook->enabled) cudaEventRecordWithFlags(hook->begin, stream, cudaEventRecordExternal);
-        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, per_cta);
+        // host-resident planes wait on the host link: keep more stages in flight
+        bool host = false;
+        for (int s = 0; s < bt.n_sessions; ++s) host |= bt.s[s].host_resident != 0;
+        const int ctas = (total_groups + kTileGroups - 1) / kTileGroups;   // one 64-word chunk each
+        if (hook && hook->enabled) record_timing_event(hook->begin, stream);
+        if (host) {
+            static int host_smem_set[64];
+            auto kern = scan_kernel<NS, GP, false, kHostStages>;
+            const size_t dyn = kHostStages * kStageBytes;
+            if ((e = ensure_smem(host_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
+            kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
+        } else {
+            static int main_smem_set[64];
+            auto kern = scan_kernel<NS, GP, false, kMainStages>;
+            const size_t dyn = kMainStages * kStageBytes;
+            if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
+            kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
         if (hook && hook->enabled) {
-            cudaEventRecordWithFlags(hook->end, stream, cudaEventRecordExternal);
+            record_timing_event(hook->end, stream);
             hook->recorded = true;
         }
         ++launches;
@@ -1356,6 +1356,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.m_keys = z.m_keys;
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
+        D.host_resident = ix.residency == FATHOM_RES_HOST_MAPPED ? 1 : 0;
         D.group_begin = groups;
         D.sample_group_begin = sgroups;
         D.q_begin = queries;

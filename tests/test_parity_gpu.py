@@ -3,7 +3,7 @@ the oracle, spanning several tiles and ragged tails.
 
 Bars: pack outputs, plans and byte counts bit-exact; scores within
 1e-4 * sum_c |q_c khat_cj|; top-k sets equal up to keys inside that band
-around the k-th score; output order by score then index."""
+around the k-th score; outputs listed in ascending key index."""
 import numpy as np
 import pytest
 import torch
@@ -261,3 +261,35 @@ def test_scan_rejects_small_workspace():
     with pytest.raises(fp.FathomError) as e:
         fp.fathom_scan_topk(ix.desc, q, t, tu, 8, oi, os_, ws)
     assert e.value.status == fp.FATHOM_ERR_WORKSPACE
+
+
+def test_scan_profile_flag_times_the_scan_kernel():
+    """FATHOM_SCAN_PROFILE records events around the main scan kernel, both
+    when launched eagerly and inside a CUDA graph capture."""
+    ses = synth.make_session(77, 2, 4, 30000, 92)
+    ix = gpu_index(ses)
+    q, t, tu, _ = run_plan(ix, ses, ses.budgets)
+    buf = fp.ScanBuffers(ix, 128)
+    fp.fathom_profile_read()
+    fp.fathom_scan_topk(ix.desc, q, t, tu, 128, buf.idx, buf.score, buf.workspace,
+                        fp.FATHOM_SCAN_PROFILE)
+    torch.cuda.synchronize()
+    ms, n = fp.fathom_profile_read()
+    assert n == 1 and ms > 0
+    ref_idx = buf.idx.clone()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+            fp.fathom_scan_topk(ix.desc, q, t, tu, 128, buf.idx, buf.score, buf.workspace,
+                                fp.FATHOM_SCAN_PROFILE)
+    torch.cuda.current_stream().wait_stream(side)
+    buf.idx.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    ms, n = fp.fathom_profile_read()
+    assert n == 1 and ms > 0
+    assert torch.equal(buf.idx, ref_idx)
+    assert fp.fathom_last_device_status() == fp.FATHOM_OK
+    del g
