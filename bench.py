@@ -385,11 +385,13 @@ def run_fathom(args, wl_name, wl):
     if wl["residency"] == "device":
         peak, peak_src = load_peaks()
         bound, peak_note = "hbm", f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"
+        kernel = "scan_kernel (filter pass)"
     else:
         peak = max(link["h2d_memcpy_gbs"], link["zero_copy_read_gbs"])
         bound, peak_note = "host_link", "measured in this run: max(pinned copy, zero-copy read)"
+        kernel = "fetch_kernel (union planes, host -> device mirror)"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "kernel": "scan_kernel (filter pass)",
+                "frac": achieved / peak, "traffic": None, "kernel": kernel,
                 "peak_source": peak_note, "avg_launch_us": avg_launch_ms * 1e3,
                 "algorithmic_bytes_per_launch": bytes_per_launch}
 

@@ -26,6 +26,18 @@ cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t
                         int32_t fixed_r, bool fixed, uint8_t *t, uint8_t *t_union,
                         uint64_t *bytes, cudaStream_t stream);
 
+// ---- fetch.cu
+// One host-resident index to fetch: for each of its n_channels = H*d
+// (head, channel) pairs, the first t_union[hc] slots of n_words words.
+struct FetchJob {
+    const uint32_t *src;       // device-mapped host planes [H][d][4][n_words]
+    uint32_t *dst;             // device mirror, same layout
+    const uint8_t *t_union;    // [H][d]
+    int n_channels;
+    int n_words;
+};
+cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream);
+
 // ---- scan.cu
 struct ScanSessionArgs {
     const fathom_index *ix;
@@ -39,11 +51,13 @@ struct ScanSessionArgs {
 // Workspace bytes for a batch of sessions (single call = batch of one).
 size_t scan_workspace_bytes(const fathom_index *sessions, int n_sessions, int k);
 
-// Profiling events around the main scan kernel (FATHOM_SCAN_PROFILE).
+// Profiling events around the dominant kernel of a scan call
+// (FATHOM_SCAN_PROFILE): the fetch when any index is host-resident, else
+// the main scan.
 struct ScanProfileHook {
     bool enabled;
     cudaEvent_t begin, end;
-    bool recorded;   // set when the main scan kernel was launched and timed
+    bool recorded;   // set when that kernel was launched and timed
 };
 
 cudaError_t launch_scan(const ScanSessionArgs *sessions, int n_sessions, int k,

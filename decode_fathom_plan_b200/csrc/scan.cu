@@ -66,8 +66,6 @@ namespace {
 
 constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-word chunk
 constexpr int kMainStages = 3;
-constexpr int kHostStages = 6;   // host-resident planes: more bytes in flight per CTA
-constexpr int kSampleStages = 8;
 
 struct SessionDesc {
     const uint32_t *planes;      // device address of [H][d][4][n_words]
@@ -82,8 +80,8 @@ struct SessionDesc {
     uint32_t *sample;            // [Q][m_keys]
     unsigned long long *cand;    // [Q][cap]
     int H, n, n_words, n_cols, col_groups;
-    int m_tiles, sample_stride, m_keys, sample_rank, exact_only, host_resident;
-    int group_begin, sample_group_begin, q_begin;
+    int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
+    int group_begin, sample_group_begin, q_begin;   // sample_group_begin: sampled-chunk index
 };
 
 template <int NS>
@@ -415,11 +413,11 @@ __device__ __forceinline__ float score_of(const float2 (&a)[4], int m, float bia
 }
 
 template <int NS>
-__device__ __forceinline__ int find_session_by_group(const Batch<NS> &b, int g, bool sample)
+__device__ __forceinline__ int find_session_by_group(const Batch<NS> &b, int g)
 {
     int si = 0;
     for (int s = 1; s < b.n_sessions; ++s)
-        if ((sample ? b.s[s].sample_group_begin : b.s[s].group_begin) <= g) si = s;
+        if (b.s[s].group_begin <= g) si = s;
     return si;
 }
 
@@ -455,7 +453,7 @@ __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_const
     const int item = blockIdx.x;
     int si = 0;
     for (int s2 = 1; s2 < b.n_sessions; ++s2)
-        if (b.s[s2].sample_group_begin <= item) si = s2;     // here: sampled-chunk index
+        if (b.s[s2].sample_group_begin <= item) si = s2;
     const SessionDesc &S = b.s[si];
     const int per_head = S.m_tiles * kSampleChunks;
     const int local = item - S.sample_group_begin;
@@ -538,12 +536,12 @@ __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_const
     }
 }
 
-// ------------------------------------------------- sampled / filtered scan
-// Persistent: CTA i owns column groups [i*per_cta, (i+1)*per_cta) of the
-// linear (session, KV head, column group) space.  kSample: the space is the
-// sampled tiles' groups and the scores go to the sample buffer; otherwise
-// keys scoring >= theta are appended to the candidate buffer.
-template <int NS, int GP, bool kSample, int STAGES>
+// ------------------------------------------------------- filtered scan
+// CTA i owns column groups [i*per_cta, (i+1)*per_cta) of the linear
+// (session, KV head, column group) space (one 64-word chunk, or two pieces
+// where the range crosses a KV head's end) and appends the keys scoring
+// >= theta to their query's candidate buffer.
+template <int NS, int GP, int STAGES>
 __global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
 scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
 {
@@ -556,24 +554,15 @@ scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
     const int g_end = min(total_groups, g + per_cta);
     int cur_si = -1, cur_h = -1;
     while (g < g_end) {
-        const int si = find_session_by_group(b, g, kSample);
+        const int si = find_session_by_group(b, g);
         const SessionDesc &S = b.s[si];
-        const int per_head = kSample ? S.m_tiles * kTileGroups : S.col_groups;
-        const int local = g - (kSample ? S.sample_group_begin : S.group_begin);
-        const int h = local / per_head;
-        const int gi = local - h * per_head;
-        // this chunk: balanced split of what is left of the range in this head
-        // (and, when sampling, in this sampled tile), at most 16 groups
-        int avail = min(g_end - g, per_head - gi);
-        int tile_i = 0, tile_off = 0, col_lo;
-        if (kSample) {
-            tile_i = gi / kTileGroups;
-            tile_off = gi - tile_i * kTileGroups;
-            avail = min(avail, kTileGroups - tile_off);
-            col_lo = (tile_i * S.sample_stride) * kTileCols + tile_off * 4;
-        } else {
-            col_lo = gi * 4;
-        }
+        const int local = g - S.group_begin;
+        const int h = local / S.col_groups;
+        const int gi = local - h * S.col_groups;
+        // this chunk: balanced split of what is left of the range in this
+        // head, at most 16 groups
+        const int avail = min(g_end - g, S.col_groups - gi);
+        const int col_lo = gi * 4;
         const int pieces = (avail + kTileGroups - 1) / kTileGroups;
         const int lim = (avail + pieces - 1) / pieces;
         const int width = lim * 4;                     // plane words owned by this chunk
@@ -589,54 +578,41 @@ scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
 
-        const bool mine = col < width;
+        const bool mine = col < width && col_lo + col < col_hi;
         const int key0 = (col_lo + col) * 32 + r;
 #pragma unroll
         for (int gg = 0; gg < GP; ++gg) {
             if (gg >= G) break;
             const int qq = q0 + gg;
             const float bias = sm.bias[gg];
-            if (kSample) {
-                if (mine) {
-                    uint32_t *dst = S.sample + (size_t)qq * S.m_keys + (size_t)tile_i * kTileKeys +
-                                    (tile_off * 4 + col) * 32 + r;
+            const uint32_t theta = S.qstate[qq * kQueryStateWords + 0];
+            uint32_t ok[8];
+            unsigned pass = 0;
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const int j = key0 + 4 * m;
-                        dst[4 * m] = (j < S.n && col_lo + col < col_hi)
-                                         ? order_key(score_of(acc[gg], m, bias)) : 0u;
-                    }
-                }
-            } else {
-                const uint32_t theta = S.qstate[qq * kQueryStateWords + 0];
-                uint32_t ok[8];
-                unsigned pass = 0;
+            for (int m = 0; m < 8; ++m) {
+                const int j = key0 + 4 * m;
+                ok[m] = order_key(score_of(acc[gg], m, bias));
+                if (mine && j < S.n && ok[m] >= theta) pass |= 1u << m;
+            }
+            const int cnt = __popc(pass);
+            int inc = cnt;
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int j = key0 + 4 * m;
-                    ok[m] = order_key(score_of(acc[gg], m, bias));
-                    if (mine && col_lo + col < col_hi && j < S.n && ok[m] >= theta) pass |= 1u << m;
-                }
-                const int cnt = __popc(pass);
-                int inc = cnt;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                if (lane >= off) inc += y;
+            }
+            const int total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+            if (total == 0) continue;
+            unsigned base = 0;
+            if (lane == 31) base = atomicAdd(&S.qstate[qq * kQueryStateWords + 1], (unsigned)total);
+            base = __shfl_sync(0xFFFFFFFFu, base, 31);
+            unsigned pos = base + (unsigned)(inc - cnt);
+            unsigned long long *cq = S.cand + (size_t)qq * b.cap;
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
-                    if (lane >= off) inc += y;
-                }
-                const int total = __shfl_sync(0xFFFFFFFFu, inc, 31);
-                if (total == 0) continue;
-                unsigned base = 0;
-                if (lane == 31) base = atomicAdd(&S.qstate[qq * kQueryStateWords + 1], (unsigned)total);
-                base = __shfl_sync(0xFFFFFFFFu, base, 31);
-                unsigned pos = base + (unsigned)(inc - cnt);
-                unsigned long long *cq = S.cand + (size_t)qq * b.cap;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    if (pass & (1u << m)) {
-                        if (pos < (unsigned)b.cap) cq[pos] = composite(ok[m], (uint32_t)(key0 + 4 * m));
-                        ++pos;
-                    }
+            for (int m = 0; m < 8; ++m) {
+                if (pass & (1u << m)) {
+                    if (pos < (unsigned)b.cap) cq[pos] = composite(ok[m], (uint32_t)(key0 + 4 * m));
+                    ++pos;
                 }
             }
         }
@@ -738,16 +714,6 @@ __device__ void bitonic_sort_desc(unsigned long long *x, int kpad)
             }
             __syncthreads();
         }
-    }
-}
-
-__device__ void write_outputs(const unsigned long long *sel, int k, int32_t *out_idx,
-                              float *out_score)
-{
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        const unsigned long long x = sel[i];
-        out_idx[i] = (int32_t)(~(uint32_t)(x & 0xFFFFFFFFull));
-        out_score[i] = order_key_to_float((uint32_t)(x >> 32));
     }
 }
 
@@ -1166,8 +1132,16 @@ Sizing size_session(int n, int n_words, int k)
 }
 
 struct WsLayout {
-    size_t qstate, sample, cand, total;
+    size_t qstate, sample, cand, mirror, total;
 };
+
+// A host-resident index is fetched into a device mirror of its planes
+// before the scoring passes (fetch.cu); the mirror is part of the workspace.
+inline bool host_resident(const fathom_index &ix) { return ix.residency == FATHOM_RES_HOST_MAPPED; }
+inline size_t plane_bytes(const fathom_index &ix)
+{
+    return (size_t)ix.n_kv_heads * (size_t)ix.head_dim * kBits * (size_t)ix.n_words * sizeof(uint32_t);
+}
 
 WsLayout layout_session(const fathom_index &ix, int k, size_t at)
 {
@@ -1181,6 +1155,8 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     at += align256((size_t)Q * z.m_keys * sizeof(uint32_t));
     L.cand = at;
     at += align256((size_t)Q * cap * sizeof(unsigned long long));
+    L.mirror = at;
+    if (host_resident(ix)) at += align256(plane_bytes(ix));
     L.total = at;
     return L;
 }
@@ -1243,12 +1219,21 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 
 template <int NS, int GP>
 cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_groups,
-                      int total_queries, int max_m_keys, uint32_t flags, cudaStream_t stream,
-                      ScanProfileHook *hook)
+                      int total_queries, int max_m_keys, const FetchJob *fetch, int n_fetch,
+                      uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
 {
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
     int launches = 0;
+    if (n_fetch > 0) {
+        // host-resident planes: bring the union plan's planes into the mirror
+        if (hook && hook->enabled) record_timing_event(hook->begin, stream);
+        if ((e = launch_fetch(fetch, n_fetch, stream)) != cudaSuccess) return note_error(e, "fetch launch");
+        if (hook && hook->enabled) {
+            record_timing_event(hook->end, stream);
+            hook->recorded = true;
+        }
+    }
     if (!force && total_sample_groups > 0) {
         static int sample_smem_set[64];
         if ((e = ensure_smem(sample_smem_set, sample_kernel<NS, GP>, kSampleSmem)) != cudaSuccess)
@@ -1266,26 +1251,16 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "theta launch");
     ++launches;
     if (!force && total_groups > 0) {
-        // host-resident planes wait on the host link: keep more stages in flight
-        bool host = false;
-        for (int s = 0; s < bt.n_sessions; ++s) host |= bt.s[s].host_resident != 0;
+        const bool timed = hook && hook->enabled && n_fetch == 0;
         const int ctas = (total_groups + kTileGroups - 1) / kTileGroups;   // one 64-word chunk each
-        if (hook && hook->enabled) record_timing_event(hook->begin, stream);
-        if (host) {
-            static int host_smem_set[64];
-            auto kern = scan_kernel<NS, GP, false, kHostStages>;
-            const size_t dyn = kHostStages * kStageBytes;
-            if ((e = ensure_smem(host_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
-            kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
-        } else {
-            static int main_smem_set[64];
-            auto kern = scan_kernel<NS, GP, false, kMainStages>;
-            const size_t dyn = kMainStages * kStageBytes;
-            if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
-            kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
-        }
+        static int main_smem_set[64];
+        auto kern = scan_kernel<NS, GP, kMainStages>;
+        const size_t dyn = kMainStages * kStageBytes;
+        if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
+        if (timed) record_timing_event(hook->begin, stream);
+        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
-        if (hook && hook->enabled) {
+        if (timed) {
             record_timing_event(hook->end, stream);
             hook->recorded = true;
         }
@@ -1326,7 +1301,8 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, sgroups = 0, queries = 0, max_m = 0;
+    int groups = 0, sgroups = 0, queries = 0, max_m = 0, n_fetch = 0;
+    FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
     for (int s = 0; s < n_sessions; ++s) {
@@ -1336,6 +1312,12 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         at = L.total;
         SessionDesc &D = bt.s[s];
         D.planes = ix.planes;
+        if (host_resident(ix)) {
+            uint32_t *mirror = reinterpret_cast<uint32_t *>(base + L.mirror);
+            fetch[n_fetch++] = FetchJob{ix.planes, mirror, ss[s].t_union,
+                                        ix.n_kv_heads * ix.head_dim, ix.n_words};
+            D.planes = mirror;
+        }
         D.mn = ix.mn;
         D.scale = ix.scale;
         D.q = ss[s].q;
@@ -1356,7 +1338,6 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.m_keys = z.m_keys;
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
-        D.host_resident = ix.residency == FATHOM_RES_HOST_MAPPED ? 1 : 0;
         D.group_begin = groups;
         D.sample_group_begin = sgroups;
         D.q_begin = queries;
@@ -1366,10 +1347,14 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
-    return run_batch<NS, 8>(bt, groups, sgroups, queries, max_m, flags, stream, hook);
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+                                           stream, hook);
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+                                           stream, hook);
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+                                           stream, hook);
+    return run_batch<NS, 8>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+                                           stream, hook);
 }
 
 }  // namespace

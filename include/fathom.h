@@ -66,9 +66,12 @@ typedef enum {
     FATHOM_ERR_UNIMPLEMENTED = 6  /* a mode this build does not provide     */
 } fathom_status;
 
-/* Where the planes live.  DEVICE: HBM.  HOST_MAPPED: pinned host memory
- * that the scan reads zero-copy over the host link (the explainer's
- * setting: the 4-bit K index is offloaded to host memory). */
+/* Where the planes live.  DEVICE: HBM.  HOST_MAPPED: pinned, device-mapped
+ * host memory (the explainer's setting: the 4-bit K index is offloaded to
+ * host memory).  A scan of a HOST_MAPPED index first fetches the planes its
+ * union plan selects over the host link into a device mirror held in the
+ * workspace (so its workspace includes H*d*4*n_words*4 bytes), then scores
+ * from the mirror. */
 typedef enum {
     FATHOM_RES_DEVICE = 0,
     FATHOM_RES_HOST_MAPPED = 1
@@ -98,7 +101,9 @@ typedef struct {
 /* Skip the sampled candidate threshold and select every query's top-k with
  * the exact multi-pass radix select (the path the fast path falls back to). */
 #define FATHOM_SCAN_FORCE_EXACT 1u
-/* Record CUDA events around the main scan kernel (benchmarking only). */
+/* Record CUDA events around the dominant kernel of the call (benchmarking
+ * only): the fetch of host-resident planes when the index is HOST_MAPPED,
+ * else the main scan kernel. */
 #define FATHOM_SCAN_PROFILE 2u
 
 /* Words per plane for n keys: n rounded up to 128 keys, i.e. 16-byte rows. */
@@ -230,10 +235,11 @@ fathom_status fathom_last_device_status(cudaStream_t stream);
 /* Kernels this library has launched in this process. */
 uint64_t fathom_launch_count(void);
 
-/* Time of the main scan kernel, recorded with CUDA events by calls made
- * with FATHOM_SCAN_PROFILE: synchronises on the recorded events and
- * returns the summed milliseconds and the number of launches timed, then
- * forgets them.  Not thread-safe; benchmarking only. */
+/* Time of the kernel FATHOM_SCAN_PROFILE times (the fetch for a
+ * host-resident index, else the main scan), recorded with CUDA events:
+ * synchronises on the recorded events and returns the summed milliseconds
+ * and the number of launches timed, then forgets them.  Not thread-safe;
+ * benchmarking only. */
 fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_launches);
 
 /* Instrumentation: read `bytes` (>= 16, a multiple of 16 is read in full)

@@ -63,6 +63,16 @@ def test_workspace_sizes_are_host_computable(lib):
         fp.fathom_scan_workspace_bytes(ix, 64) + fp.fathom_scan_workspace_bytes(big, 64)
 
 
+def test_host_resident_workspace_holds_a_plane_mirror(lib):
+    # a HOST_MAPPED index is fetched into a device mirror of its planes
+    # [H][d][4][n_words] uint32 held in the workspace
+    for H, d, n in ((2, 128, 4096), (8, 128, 1 << 20), (1, 64, 1000)):
+        dev = fp.fathom_scan_workspace_bytes(_desc(H=H, d=d, n=n, residency=0), 64)
+        host = fp.fathom_scan_workspace_bytes(_desc(H=H, d=d, n=n, residency=1), 64)
+        mirror = H * d * 4 * fp.fathom_n_words(n) * 4
+        assert host - dev == (mirror + 255) // 256 * 256
+
+
 @pytest.mark.parametrize("field,value", [("head_dim", 48), ("head_dim", 512), ("group", 9),
                                          ("group", 0), ("n_words", 6), ("n_keys", 0),
                                          ("residency", 7)])
