@@ -66,6 +66,7 @@ namespace {
 
 constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-word chunk
 constexpr int kMainStages = 3;
+constexpr int kMaskOrderValues = 16;   // reader sets of up to 4 query heads
 
 struct SessionDesc {
     const uint32_t *planes;      // device address of [H][d][4][n_words]
@@ -79,9 +80,10 @@ struct SessionDesc {
     uint32_t *qstate;            // [Q][4]: theta, count, fallback flag, spare
     uint32_t *sample;            // [Q][m_keys]
     unsigned long long *cand;    // [Q][cap]
+    unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int group_begin, sample_group_begin, q_begin;   // sample_group_begin: sampled-chunk index
+    int group_begin, sample_group_begin, q_begin, head_begin;   // sample_group_begin: sampled-chunk index
 };
 
 template <int NS>
@@ -102,12 +104,22 @@ struct alignas(16) ScanMeta {
                                               // bits 16-23: queries reading 0 < t < T planes
     uint8_t tq[kMaxHeadDim][GP];              // planes read per (union channel, query)
     uint8_t stage_partial[kMaxHeadDim / kStageChannels];   // a query reads 0 < t < T in the stage
+    unsigned stage_mask[kMaxHeadDim / kStageChannels];     // queries reading a stage's channel at
+                                                           // full union depth (OR over the stage)
     float bias[GP];
     int U, n_stages;
     int part[kScanThreads / 32];
+    int order[kScanThreads / 32][kMaskOrderValues];       // channel-order offsets per (warp, mask)
 };
 
 typedef uint32_t (*StageBuf)[kStageRows][kTileCols];
+
+// Query groups of up to 4 heads list a KV head's union channels by the set
+// of queries that read them at full union depth (then by channel), so that
+// a stage of 8 channels is mostly read by one set and its FMAs can be
+// specialised to that set.  Larger groups keep channel order.
+template <int GP>
+constexpr bool mask_ordered() { return GP <= 4; }
 
 // ------------------------------------------------------------ small helpers
 // Plain 16-byte copy (no source-size operand).
@@ -137,50 +149,39 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// (a & b) | c in one logic op.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // 8 nibbles of a word -> 8 exact floats, paired (m, m+4).  A nibble at bit
 // 4m is OR-ed under the mantissa of 2^(23-4m), whose unit in the last place
 // there is 1, so the float is 2^(23-4m) + v; subtracting the power leaves v.
-// Nibble m+4 sits at bit 4m of nib >> 16, so both halves of the 64-bit word
-// {nib, nib >> 16} use the same mask and power, and each pair is one
-// 64-bit and/or plus one paired add (add.rn.f32x2) with no repacking.
-// neg[m] holds -2^(23-4m) in both halves.
-__device__ __forceinline__ void nibbles_to_floats(uint32_t nib, const unsigned long long (&neg)[4],
+// Nibble m+4 sits at bit 4m of nib >> 16, so both halves of pair m use the
+// same mask and power: one fused and/or per key and one paired add
+// (add.rn.f32x2) per two keys.  neg[m] = -2^(23-4m).
+__device__ __forceinline__ void nibbles_to_floats(uint32_t nib, const float (&neg)[4],
                                                   float2 (&v)[4])
 {
-    unsigned long long r0, r1, r2, r3;
-    asm("{\n"
-        ".reg .b64 p, t;\n"
-        ".reg .b32 h;\n"
-        "shr.b32 h, %4, 16;\n"
-        "mov.b64 p, {%4, h};\n"
-        "and.b64 t, p, 0x0000000F0000000F;\n"
-        "or.b64 t, t, 0x4B0000004B000000;\n"
-        "add.rn.f32x2 %0, t, %5;\n"
-        "and.b64 t, p, 0x000000F0000000F0;\n"
-        "or.b64 t, t, 0x4900000049000000;\n"
-        "add.rn.f32x2 %1, t, %6;\n"
-        "and.b64 t, p, 0x00000F0000000F00;\n"
-        "or.b64 t, t, 0x4700000047000000;\n"
-        "add.rn.f32x2 %2, t, %7;\n"
-        "and.b64 t, p, 0x0000F0000000F000;\n"
-        "or.b64 t, t, 0x4500000045000000;\n"
-        "add.rn.f32x2 %3, t, %8;\n"
-        "}"
-        : "=l"(r0), "=l"(r1), "=l"(r2), "=l"(r3)
-        : "r"(nib), "l"(neg[0]), "l"(neg[1]), "l"(neg[2]), "l"(neg[3]));
-    v[0] = make_float2(__uint_as_float((uint32_t)r0), __uint_as_float((uint32_t)(r0 >> 32)));
-    v[1] = make_float2(__uint_as_float((uint32_t)r1), __uint_as_float((uint32_t)(r1 >> 32)));
-    v[2] = make_float2(__uint_as_float((uint32_t)r2), __uint_as_float((uint32_t)(r2 >> 32)));
-    v[3] = make_float2(__uint_as_float((uint32_t)r3), __uint_as_float((uint32_t)(r3 >> 32)));
+    const uint32_t hi = nib >> 16;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const uint32_t mask = 0xFu << (4 * m);
+        const uint32_t magic = (150u - 4u * (uint32_t)m) << 23;   // 2^(23-4m)
+        const float a = __uint_as_float(and_or(nib, mask, magic));
+        const float b = __uint_as_float(and_or(hi, mask, magic));
+        v[m] = __fadd2_rn(make_float2(a, b), make_float2(neg[m], neg[m]));
+    }
 }
 
-// -2^(23-4m) in both halves, m = 0..3.
-__constant__ unsigned long long c_neg_magic[4] = {0xCB000000CB000000ull, 0xC9000000C9000000ull,
-                                                  0xC7000000C7000000ull, 0xC5000000C5000000ull};
-__device__ __forceinline__ void magic_negatives(unsigned long long (&neg)[4])
+// -2^(23-4m), m = 0..3.
+__device__ __forceinline__ void magic_negatives(float (&neg)[4])
 {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) neg[m] = c_neg_magic[m];
+    for (int m = 0; m < 4; ++m) neg[m] = -__uint_as_float((150u - 4u * (uint32_t)m) << 23);
 }
 
 // Offset of the coarse-bin middle: (2^(4-t) - 1) / 2.
@@ -204,22 +205,75 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     const int c = tid;
     const int T = (c < d) ? min((int)tu_row[c], kBits) : 0;
     const bool has = T > 0;
+    // reader sets of this channel: full = queries reading all T planes,
+    // partial = queries reading 0 < t < T of them
+    unsigned full = 0, partial = 0;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        const int tg = (has && g < G) ? min((int)t_rows[g * d + c], T) : 0;
+        if (has && tg == T) full |= 1u << g;
+        else if (tg > 0) partial |= 1u << g;
+    }
     const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
     if (lane == 0) sm.part[warp] = __popc(bal);
-    if (tid < kMaxHeadDim / kStageChannels) sm.stage_partial[tid] = 0;
-    __syncthreads();
-    int base = 0, U = 0;
+    if (tid < kMaxHeadDim / kStageChannels) {
+        sm.stage_partial[tid] = 0;
+        sm.stage_mask[tid] = 0u;
+    }
+    // position among the lanes of this warp with the same ordering key
+    const unsigned key = mask_ordered<GP>() ? full : 0u;
+    int lane_rank = __popc(bal & ((1u << lane) - 1u));
+    if (mask_ordered<GP>()) {
 #pragma unroll
-    for (int w = 0; w < kScanThreads / 32; ++w) {
-        const int p = sm.part[w];
-        base += (w < warp) ? p : 0;
-        U += p;
+        for (unsigned v = 0; v < (1u << GP); ++v) {
+            const unsigned b = __ballot_sync(0xFFFFFFFFu, has && key == v);
+            if (lane == 0) sm.order[warp][v] = __popc(b);
+            if (key == v) lane_rank = __popc(b & ((1u << lane) - 1u));
+        }
+    }
+    __syncthreads();
+    int U = 0;
+#pragma unroll
+    for (int w = 0; w < kScanThreads / 32; ++w) U += sm.part[w];
+    if (mask_ordered<GP>()) {
+        // warp 0 turns the (warp, key) counts into exclusive offsets in
+        // (key, warp) order
+        if (warp == 0) {
+            const unsigned v = (unsigned)lane;
+            int tot = 0, cnt[kScanThreads / 32];
+#pragma unroll
+            for (int w = 0; w < kScanThreads / 32; ++w) {
+                cnt[w] = (v < (1u << GP)) ? sm.order[w][v] : 0;
+                tot += cnt[w];
+            }
+            int incl = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            int at = incl - tot;
+            if (v < (1u << GP)) {
+#pragma unroll
+                for (int w = 0; w < kScanThreads / 32; ++w) {
+                    sm.order[w][v] = at;
+                    at += cnt[w];
+                }
+            }
+        }
+        __syncthreads();
+    }
+    int base = 0;
+    if (mask_ordered<GP>()) {
+        base = has ? sm.order[warp][key] : 0;
+    } else {
+#pragma unroll
+        for (int w = 0; w < kScanThreads / 32; ++w) base += (w < warp) ? sm.part[w] : 0;
     }
     const int n_stages = (U + kStageChannels - 1) / kStageChannels;
     if (has) {
-        const int u = base + __popc(bal & ((1u << lane) - 1u));
+        const int u = base + lane_rank;
         const float sc = sc_h[c];
-        unsigned full = 0, partial = 0;
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
             int tg = 0;
@@ -228,8 +282,6 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
                 tg = min((int)t_rows[g * d + c], T);
                 w = __fmul_rn(bf16_to_float(q_rows[g * d + c]), sc);
             }
-            if (tg == T) full |= 1u << g;
-            else if (tg > 0) partial |= 1u << g;
             // full-depth readers use W2 in the unconditional fma; others add 0
             // there and, if partial, their own masked term
             sm.W2[u][g] = (tg == T) ? make_float2(w, w) : make_float2(0.0f, 0.0f);
@@ -238,6 +290,7 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
         }
         sm.meta[u] = full | (partial << 16);
         if (partial) sm.stage_partial[u / kStageChannels] = 1;
+        atomicOr(&sm.stage_mask[u / kStageChannels], full);
 #pragma unroll
         for (int s2 = 0; s2 < kBits; ++s2)
             sm.row_g[u * kBits + s2] = (s2 < T) ? (uint32_t)((h * d + c) * kBits + s2) : 0xFFFFFFFFu;
@@ -261,6 +314,22 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
         if (lane == 0) sm.bias[warp] = (float)acc;
     }
+    __syncthreads();
+}
+
+// Per-head tables are built once per (session, KV head) by prep_kernel and
+// copied by every CTA that scans the head: one round trip instead of the
+// dependent loads, barriers and fp64 bias sums of setup_head.  Ends with a
+// barrier; completes every cp.async group in flight.
+template <int GP>
+__device__ __forceinline__ void load_head(ScanMeta<GP> &sm, const unsigned char *tables, int h)
+{
+    constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
+    const uint4 *src = reinterpret_cast<const uint4 *>(tables + (size_t)h * sizeof(ScanMeta<GP>));
+    uint4 *dst = reinterpret_cast<uint4 *>(&sm);
+    for (int i = threadIdx.x; i < kUnits; i += blockDim.x) cp_async16_full(dst + i, src + i);
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
 }
 
@@ -304,7 +373,7 @@ __device__ __forceinline__ uint32_t gather_nibbles(const uint32_t (*rows)[COLS],
 template <int GP>
 __device__ __forceinline__ void fma_partial(unsigned pmask, uint32_t nib, int u,
                                             const ScanMeta<GP> &sm,
-                                            const unsigned long long (&neg)[4],
+                                            const float (&neg)[4],
                                             float2 (&acc)[GP][4])
 {
 #pragma unroll
@@ -328,7 +397,7 @@ __device__ __forceinline__ void fma_partial(unsigned pmask, uint32_t nib, int u,
 template <int GP, bool kPartial, int COLS = kTileCols>
 __device__ __forceinline__ void channel(const ScanMeta<GP> &sm, const uint32_t (*rows)[COLS],
                                         int u, int col, const uint32_t (&sh)[4],
-                                        const unsigned long long (&neg)[4], float2 (&acc)[GP][4])
+                                        const float (&neg)[4], float2 (&acc)[GP][4])
 {
     const uint32_t nib = gather_nibbles<COLS>(rows, col, sh);
     float2 v[4];
@@ -345,18 +414,86 @@ __device__ __forceinline__ void channel(const ScanMeta<GP> &sm, const uint32_t (
     }
 }
 
+// One union channel read at full union depth by exactly the queries in
+// MASK (and by no query at a partial depth): FMAs for those queries only.
+template <int GP, unsigned MASK, int COLS>
+__device__ __forceinline__ void channel_masked(const ScanMeta<GP> &sm, const uint32_t (*rows)[COLS],
+                                               int u, int col, const uint32_t (&sh)[4],
+                                               const float (&neg)[4],
+                                               float2 (&acc)[GP][4])
+{
+    const uint32_t nib = gather_nibbles<COLS>(rows, col, sh);
+    float2 v[4];
+    nibbles_to_floats(nib, neg, v);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        if ((MASK >> g) & 1u) {
+            const float2 w = sm.W2[u][g];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[g][i] = __ffma2_rn(v[i], w, acc[g][i]);
+        }
+    }
+}
+
+template <int GP, unsigned MASK, int COLS>
+__device__ __forceinline__ void stage_masked(const ScanMeta<GP> &sm, const uint32_t (*rows)[COLS],
+                                             int u0, int col, const uint32_t (&sh)[4],
+                                             const float (&neg)[4],
+                                             float2 (&acc)[GP][4])
+{
+    if constexpr (MASK < (1u << GP)) {
+        // unrolled by 2 only: 16 specialised bodies unrolled 8 times miss in
+        // the instruction cache
+#pragma unroll 2
+        for (int j = 0; j < kStageChannels; ++j)
+            channel_masked<GP, MASK, COLS>(sm, rows + kBits * j, u0 + j, col, sh, neg, acc);
+    }
+}
+
+// A full stage with no partial-depth reader, specialised to the set of
+// queries that read its channels (a query outside the set multiplies zeros).
+template <int GP, int COLS>
+__device__ __forceinline__ void stage_dispatch(unsigned mask, const ScanMeta<GP> &sm,
+                                               const uint32_t (*rows)[COLS], int u0, int col,
+                                               const uint32_t (&sh)[4],
+                                               const float (&neg)[4],
+                                               float2 (&acc)[GP][4])
+{
+    switch (mask) {
+    case 1: stage_masked<GP, 1, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 2: stage_masked<GP, 2, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 3: stage_masked<GP, 3, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 4: stage_masked<GP, 4, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 5: stage_masked<GP, 5, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 6: stage_masked<GP, 6, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 7: stage_masked<GP, 7, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 8: stage_masked<GP, 8, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 9: stage_masked<GP, 9, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 10: stage_masked<GP, 10, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 11: stage_masked<GP, 11, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 12: stage_masked<GP, 12, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 13: stage_masked<GP, 13, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    case 14: stage_masked<GP, 14, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    default: stage_masked<GP, 15, COLS>(sm, rows, u0, col, sh, neg, acc); break;
+    }
+}
+
 // Channels [u0, u1) of the stage held in `rows` (channel u0 in rows 0..3).
 template <int GP, int COLS = kTileCols>
 __device__ __forceinline__ void compute_stage(const ScanMeta<GP> &sm, int st,
                                               const uint32_t (*rows)[COLS], int u0, int u1,
                                               int col, const uint32_t (&sh)[4],
-                                              const unsigned long long (&neg)[4],
+                                              const float (&neg)[4],
                                               float2 (&acc)[GP][4])
 {
     if (u1 - u0 == kStageChannels && !sm.stage_partial[st]) {
+        if constexpr (mask_ordered<GP>()) {
+            stage_dispatch<GP, COLS>(sm.stage_mask[st], sm, rows, u0, col, sh, neg, acc);
+        } else {
 #pragma unroll
-        for (int j = 0; j < kStageChannels; ++j)
-            channel<GP, false, COLS>(sm, rows + kBits * j, u0 + j, col, sh, neg, acc);
+            for (int j = 0; j < kStageChannels; ++j)
+                channel<GP, false, COLS>(sm, rows + kBits * j, u0 + j, col, sh, neg, acc);
+        }
     } else {
         for (int u = u0; u < u1; ++u)
             channel<GP, true, COLS>(sm, rows + kBits * (u - u0), u, col, sh, neg, acc);
@@ -377,7 +514,7 @@ __device__ void scan_chunk(const ScanMeta<GP> &sm, StageBuf stage, const uint32_
     uint32_t sh[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
-    unsigned long long neg[4];
+    float neg[4];
     magic_negatives(neg);
 #pragma unroll
     for (int g = 0; g < GP; ++g)
@@ -444,6 +581,27 @@ constexpr int kMaxStages = kMaxHeadDim / kStageChannels;          // 32
 typedef uint32_t (*SampleBuf)[kStageRows][kSampleCols];
 constexpr size_t kSampleSmem = (size_t)kMaxStages * kStageRows * kSampleCols * sizeof(uint32_t);
 
+// One CTA per (session, KV head): build the head's scan tables and store
+// them for the sampling and scanning CTAs (load_head).
+template <int NS, int GP>
+__global__ void __launch_bounds__(kScanThreads) prep_kernel(const __grid_constant__ Batch<NS> b)
+{
+    __shared__ ScanMeta<GP> sm;
+    const int item = blockIdx.x;
+    int si = 0;
+    for (int s2 = 1; s2 < b.n_sessions; ++s2)
+        if (b.s[s2].head_begin <= item) si = s2;
+    const SessionDesc &S = b.s[si];
+    const int h = item - S.head_begin;
+    const int G = b.G, d = b.d, q0 = h * G;
+    setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
+                   S.mn + h * d, S.scale + h * d);
+    constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
+    const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
+    uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
+    for (int i = threadIdx.x; i < kUnits; i += blockDim.x) dst[i] = src[i];
+}
+
 template <int NS, int GP>
 __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_constant__ Batch<NS> b)
 {
@@ -462,9 +620,8 @@ __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_const
     const int tile_i = ci / kSampleChunks, chunk = ci - tile_i * kSampleChunks;
     const int col_lo = tile_i * S.sample_stride * kTileCols + chunk * kSampleCols;
     const int col_hi = min(S.n_cols, col_lo + kSampleCols);
-    const int G = b.G, d = b.d, q0 = h * G;
-    setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
-                   S.mn + h * d, S.scale + h * d);
+    const int G = b.G, q0 = h * G;
+    load_head<GP>(sm, S.tables, h);
     // every plane row of every stage, 4 x 16 bytes per row
     const int n_stages = sm.n_stages;
     const int n_chunks = n_stages * kStageRows * (kSampleCols / 4);
@@ -486,7 +643,7 @@ __global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_const
     uint32_t sh[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
-    unsigned long long neg[4];
+    float neg[4];
     magic_negatives(neg);
     float2 acc[GP][4];
 #pragma unroll
@@ -546,10 +703,14 @@ __global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
 scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
 {
     __shared__ ScanMeta<GP> sm;
+    __shared__ uint32_t s_theta[GP];
+    __shared__ unsigned s_wtot[kScanThreads / 32][GP];   // candidates per (warp, query)
+    __shared__ unsigned s_woff[kScanThreads / 32][GP];   // their first slot
     extern __shared__ __align__(16) uint32_t scan_dyn[];
     StageBuf stage = reinterpret_cast<StageBuf>(scan_dyn);
-    const int G = b.G, d = b.d;
+    const int G = b.G;
     const int col = threadIdx.x >> 2, r = threadIdx.x & 3, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     int g = blockIdx.x * per_cta;
     const int g_end = min(total_groups, g + per_cta);
     int cur_si = -1, cur_h = -1;
@@ -570,49 +731,75 @@ scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
         const int q0 = h * G;
         if (si != cur_si || h != cur_h) {
             __syncthreads();   // the previous chunk's epilogue may still read sm
-            setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
-                           S.mn + h * d, S.scale + h * d);
+            if (threadIdx.x < GP)
+                s_theta[threadIdx.x] = (threadIdx.x < G)
+                                           ? S.qstate[(q0 + threadIdx.x) * kQueryStateWords + 0]
+                                           : 0xFFFFFFFFu;
+            load_head<GP>(sm, S.tables, h);
             cur_si = si;
             cur_h = h;
         }
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
 
+        // keys scoring >= theta: counts per warp and query, one reservation
+        // per (CTA, query) in the query's candidate buffer, then the writes
         const bool mine = col < width && col_lo + col < col_hi;
         const int key0 = (col_lo + col) * 32 + r;
+        unsigned pass[GP];
+        int before[GP];
 #pragma unroll
         for (int gg = 0; gg < GP; ++gg) {
-            if (gg >= G) break;
-            const int qq = q0 + gg;
-            const float bias = sm.bias[gg];
-            const uint32_t theta = S.qstate[qq * kQueryStateWords + 0];
-            uint32_t ok[8];
-            unsigned pass = 0;
+            pass[gg] = 0u;
+            before[gg] = 0;
+            if (gg < G) {
+                const float bias = sm.bias[gg];
+                const uint32_t theta = s_theta[gg];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int j = key0 + 4 * m;
-                ok[m] = order_key(score_of(acc[gg], m, bias));
-                if (mine && j < S.n && ok[m] >= theta) pass |= 1u << m;
+                for (int m = 0; m < 8; ++m) {
+                    const int j = key0 + 4 * m;
+                    if (mine && j < S.n && order_key(score_of(acc[gg], m, bias)) >= theta)
+                        pass[gg] |= 1u << m;
+                }
+                const int cnt = __popc(pass[gg]);
+                int inc = cnt;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                    if (lane >= off) inc += y;
+                }
+                before[gg] = inc - cnt;
+                if (lane == 31) s_wtot[warp][gg] = (unsigned)inc;
             }
-            const int cnt = __popc(pass);
-            int inc = cnt;
+        }
+        __syncthreads();
+        if (threadIdx.x < G) {
+            const int gg = threadIdx.x;
+            unsigned tot = 0;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
-                if (lane >= off) inc += y;
+            for (int w = 0; w < kScanThreads / 32; ++w) tot += s_wtot[w][gg];
+            unsigned at = tot ? atomicAdd(&S.qstate[(q0 + gg) * kQueryStateWords + 1], tot) : 0u;
+#pragma unroll
+            for (int w = 0; w < kScanThreads / 32; ++w) {
+                s_woff[w][gg] = at;
+                at += s_wtot[w][gg];
             }
-            const int total = __shfl_sync(0xFFFFFFFFu, inc, 31);
-            if (total == 0) continue;
-            unsigned base = 0;
-            if (lane == 31) base = atomicAdd(&S.qstate[qq * kQueryStateWords + 1], (unsigned)total);
-            base = __shfl_sync(0xFFFFFFFFu, base, 31);
-            unsigned pos = base + (unsigned)(inc - cnt);
-            unsigned long long *cq = S.cand + (size_t)qq * b.cap;
+        }
+        __syncthreads();
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                if (pass & (1u << m)) {
-                    if (pos < (unsigned)b.cap) cq[pos] = composite(ok[m], (uint32_t)(key0 + 4 * m));
-                    ++pos;
+        for (int gg = 0; gg < GP; ++gg) {
+            if (gg < G && pass[gg]) {
+                const float bias = sm.bias[gg];
+                unsigned pos = s_woff[warp][gg] + (unsigned)before[gg];
+                unsigned long long *cq = S.cand + (size_t)(q0 + gg) * b.cap;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    if (pass[gg] & (1u << m)) {
+                        if (pos < (unsigned)b.cap)
+                            cq[pos] = composite(order_key(score_of(acc[gg], m, bias)),
+                                                (uint32_t)(key0 + 4 * m));
+                        ++pos;
+                    }
                 }
             }
         }
@@ -1132,8 +1319,20 @@ Sizing size_session(int n, int n_words, int k)
 }
 
 struct WsLayout {
-    size_t qstate, sample, cand, mirror, total;
+    size_t qstate, sample, cand, tables, mirror, total;
 };
+
+// Query heads per KV head rounded up to the kernels' template width.
+inline int gp_for(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
+inline size_t head_table_bytes(int G)
+{
+    switch (gp_for(G)) {
+    case 1: return sizeof(ScanMeta<1>);
+    case 2: return sizeof(ScanMeta<2>);
+    case 4: return sizeof(ScanMeta<4>);
+    default: return sizeof(ScanMeta<8>);
+    }
+}
 
 // A host-resident index is fetched into a device mirror of its planes
 // before the scoring passes (fetch.cu); the mirror is part of the workspace.
@@ -1155,6 +1354,8 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     at += align256((size_t)Q * z.m_keys * sizeof(uint32_t));
     L.cand = at;
     at += align256((size_t)Q * cap * sizeof(unsigned long long));
+    L.tables = at;
+    at += align256((size_t)ix.n_kv_heads * head_table_bytes(ix.group));
     L.mirror = at;
     if (host_resident(ix)) at += align256(plane_bytes(ix));
     L.total = at;
@@ -1219,8 +1420,8 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 
 template <int NS, int GP>
 cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_groups,
-                      int total_queries, int max_m_keys, const FetchJob *fetch, int n_fetch,
-                      uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
+                      int total_queries, int total_heads, int max_m_keys, const FetchJob *fetch,
+                      int n_fetch, uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
 {
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
@@ -1233,6 +1434,11 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
             record_timing_event(hook->end, stream);
             hook->recorded = true;
         }
+    }
+    if (!force && total_groups > 0) {
+        prep_kernel<NS, GP><<<total_heads, kScanThreads, 0, stream>>>(bt);
+        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "prep launch");
+        ++launches;
     }
     if (!force && total_sample_groups > 0) {
         static int sample_smem_set[64];
@@ -1252,13 +1458,14 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
     ++launches;
     if (!force && total_groups > 0) {
         const bool timed = hook && hook->enabled && n_fetch == 0;
-        const int ctas = (total_groups + kTileGroups - 1) / kTileGroups;   // one 64-word chunk each
+        const int per_cta = kTileGroups;   // one 64-word chunk per CTA
+        const int ctas = (total_groups + per_cta - 1) / per_cta;
         static int main_smem_set[64];
         auto kern = scan_kernel<NS, GP, kMainStages>;
         const size_t dyn = kMainStages * kStageBytes;
         if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
         if (timed) record_timing_event(hook->begin, stream);
-        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, kTileGroups);
+        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, per_cta);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
         if (timed) {
             record_timing_event(hook->end, stream);
@@ -1301,7 +1508,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, sgroups = 0, queries = 0, max_m = 0, n_fetch = 0;
+    int groups = 0, sgroups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
     FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
@@ -1328,6 +1535,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.qstate = reinterpret_cast<uint32_t *>(base + L.qstate);
         D.sample = reinterpret_cast<uint32_t *>(base + L.sample);
         D.cand = reinterpret_cast<unsigned long long *>(base + L.cand);
+        D.tables = reinterpret_cast<unsigned char *>(base + L.tables);
         D.H = ix.n_kv_heads;
         D.n = ix.n_keys;
         D.n_words = ix.n_words;
@@ -1341,19 +1549,21 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.group_begin = groups;
         D.sample_group_begin = sgroups;
         D.q_begin = queries;
+        D.head_begin = heads;
+        heads += ix.n_kv_heads;
         groups += D.H * D.col_groups;
         sgroups += D.H * D.m_tiles * kSampleChunks;   // sampled 16-word chunks
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    return run_batch<NS, 8>(bt, groups, sgroups, queries, max_m, fetch, n_fetch, flags,
+    return run_batch<NS, 8>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
 }
 
