@@ -2,21 +2,23 @@
 """Benchmark of the Fathom per-query read-depth top-k key scan on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
-                    [--workload qwen3_8b_layer_128k|host_1m]
+                    [--workload qwen3_8b_layer_128k|host_1m|fixed_vs_wf_1m|agent_16_sessions]
 
 A step is one decode-step scan of a whole layer through the hot path, once
-per bit budget of the workload: plan (reverse water-filling, GQA union) then
-scan + top-k, for every KV head and query head.  Default workload: a
-Qwen3-8B-shaped layer resident in HBM (8 KV heads x 4 query heads,
-head_dim 128, 131072 keys, B in {68, 92, 136}, k = 2048).  Inputs are
-synthetic (seeded, see synth/); each step gets fresh queries and the L2 is
-flushed (256 MiB write) between timed steps, outside the step's events.
+per plan of the workload: plan (reverse water-filling at B bits per key, or
+a fixed top-r plan; GQA union) then scan + top-k, for every KV head and
+query head.  agent_16_sessions instead plans 16 independent sessions and
+scans them in one batched call per step.  Default workload: a Qwen3-8B-shaped
+layer resident in HBM (8 KV heads x 4 query heads, head_dim 128, 131072
+keys, B in {68, 92, 136}, k = 2048).  Inputs are synthetic (seeded, see
+synth/); each step gets fresh queries and the L2 is flushed (256 MiB write)
+between timed steps, outside the step's events.
 
 Prints one JSON line (rank 0).  value = Gkeys/s over all ranks (keys per KV
-head x KV heads x budgets x steps / the slowest rank's summed step time).
-For N > 1 each rank scans its own independent layer (weak scaling; the path
-needs no collective).  --impl reference times the CPU oracle instead, on a
-bounded sample of the same workload.
+head x KV heads x scans per step x steps / the slowest rank's summed step
+time).  For N > 1 each rank scans its own independent layer (weak scaling;
+the path needs no collective).  --impl reference times the CPU oracle
+instead, on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -42,12 +44,30 @@ UNIT = "Gkeys/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
+# plans: ("wf", B) = reverse water-filling at B bits per key; ("fixed", r) =
+# the top-r channels by |q_c| at 4 bits.  "device_keys": keys drawn on the
+# GPU (synth.device_keys) instead of numpy, for sizes numpy would take
+# minutes on.  agent_16_sessions scans its sessions in one batched call.
 WORKLOADS = {
-    "qwen3_8b_layer_128k": dict(H=8, G=4, n=131072, d=128, budgets=(68, 92, 136), k=2048,
-                                residency="device"),
-    "host_1m": dict(H=8, G=4, n=1 << 20, d=128, budgets=(18, 68, 92, 136), k=2048,
-                    residency="host_mapped"),
+    "qwen3_8b_layer_128k": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
+                                plans=(("wf", 68), ("wf", 92), ("wf", 136))),
+    "host_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
+                    plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
+    "fixed_vs_wf_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
+                           plans=(("fixed", 34), ("fixed", 17), ("wf", 68), ("wf", 92)),
+                           device_keys=True),
+    "agent_16_sessions": dict(H=8, G=4, n=None, d=128, k=1024, residency="host_mapped",
+                              sessions=16, plans=None, device_keys=True, batched=True),
 }
+
+
+def plan_name(spec):
+    return f"{spec[0]}{spec[1]}"
+
+
+def plan_bits(spec):
+    """Bits per key a query of this plan reads."""
+    return spec[1] if spec[0] == "wf" else 4 * spec[1]
 
 
 def parse_args():
@@ -83,11 +103,20 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def config_of(wl_name, wl, flush_note):
-    return {"workload": wl_name, "kv_heads": wl["H"], "query_heads_per_kv": wl["G"],
-            "head_dim": wl["d"], "n_keys": wl["n"], "budgets_bits_per_key": list(wl["budgets"]),
-            "k": wl["k"], "residency": "hbm" if wl["residency"] == "device" else "host_pinned_mapped",
-            "l2": flush_note}
+def config_of(wl_name, wl, flush_note, sessions=None):
+    c = {"workload": wl_name, "kv_heads": wl["H"], "query_heads_per_kv": wl["G"],
+         "head_dim": wl["d"], "k": wl["k"],
+         "residency": "hbm" if wl["residency"] == "device" else "host_pinned_mapped",
+         "l2": flush_note}
+    if sessions is None:
+        c["n_keys"] = wl["n"]
+        c["plans"] = [plan_name(p) for p in wl["plans"]]
+    else:
+        c["sessions"] = len(sessions)
+        c["n_keys_per_session"] = [x["n"] for x in sessions]
+        c["budget_per_session"] = [x["budget"] for x in sessions]
+        c["batched"] = True
+    return c
 
 
 # ------------------------------------------------------------------ clocks
@@ -167,62 +196,74 @@ def measure_host_link(fp, torch, nbytes=1 << 30, reps=10):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_sample(ses, budgets, k, heads, ref=None):
-    """Time the oracle (plan + fp64 score + full-sort top-k per query) on the
-    given KV heads at every budget.  The index build (storage side, off the
-    decode path) is not timed.  Returns (seconds, head-scans, keys)."""
+def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None):
+    """Time the oracle (plan + fp64 score + full-sort top-k per query) over
+    the given KV heads' keys (float32 [h][n][d]) at every plan spec.  The
+    index build (storage side, off the decode path) is not timed.
+    Returns (seconds, head-scans, keys)."""
     import oracle
     if ref is None:
-        ref = oracle.build_index(ses.keys[list(heads)])
-    G = ses.group
+        ref = oracle.build_index(keys_heads)
+    n = keys_heads.shape[1]
     t0 = time.perf_counter()
     scans = 0
-    for hi, h in enumerate(heads):
-        for B in budgets:
+    for hi in range(keys_heads.shape[0]):
+        for spec in plans:
             for g in range(G):
-                qrow = ses.q_bf16[h * G + g]
-                tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), B)
+                qrow = q_bf16[hi * G + g]
+                if spec[0] == "wf":
+                    tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1])
+                else:
+                    tq = oracle.fixed_plan(qrow, spec[1])
                 s = oracle.score_planes(ref["planes"][hi], ref["mn"][hi], ref["scale"][hi],
-                                        qrow, tq, ses.n_keys)
+                                        qrow, tq, n)
                 oracle.topk(s, k)
             scans += 1
-    return time.perf_counter() - t0, scans, scans * ses.n_keys
+    return time.perf_counter() - t0, scans, scans * n
 
 
-def cpu_baseline(ses, wl):
-    # about 10-30 s of single-thread oracle work
-    heads = tuple(range(max(1, min(4, wl["H"], (4 * 131072) // wl["n"]))))
-    secs, scans, keys = oracle_sample(ses, wl["budgets"], wl["k"], heads)
+def cpu_baseline(keys_heads, q_bf16, G, plans, k):
+    """About 10-30 s of single-thread oracle work on a few KV heads."""
+    secs, scans, keys = oracle_sample(keys_heads, q_bf16, G, plans, k)
     return {"value": keys / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"KV heads {list(heads)} x budgets {list(wl['budgets'])}: {scans} head "
-                      f"scans of {ses.n_keys} keys (4 query heads each), single thread, "
+            "sample": f"{keys_heads.shape[0]} KV head(s) x plans "
+                      f"{[plan_name(p) for p in plans]}: {scans} head scans of "
+                      f"{keys_heads.shape[1]} keys ({G} query heads each), single thread, "
                       f"{secs:.1f} s"}
+
+
+def reference_plans(wl):
+    if wl.get("plans"):
+        return wl["plans"]
+    return tuple(("wf", B) for B in (68, 92, 136))
 
 
 def run_reference(args, wl_name, wl):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    n = wl["n"] if wl["residency"] == "device" else min(wl["n"], 1 << 18)
-    ses = synth.make_session(0, 1, wl["G"], n, wl["budgets"][0], head_dim=wl["d"])
-    budgets = wl["budgets"]
+    n = wl["n"] if (wl["n"] and wl["residency"] == "device") else min(wl["n"] or (1 << 18), 1 << 18)
+    plans = reference_plans(wl)
+    ses = synth.make_session(0, 1, wl["G"], n, plan_bits(plans[0]), head_dim=wl["d"])
     import oracle
     ref = oracle.build_index(ses.keys[:1])
     times = []
     for i in range(args.warmup + args.steps):
-        secs, _, _ = oracle_sample(ses, (budgets[i % len(budgets)],), wl["k"], (0,), ref)
+        secs, _, _ = oracle_sample(ses.keys[:1], ses.q_bf16, wl["G"], (plans[i % len(plans)],),
+                                   wl["k"], ref)
         if i >= args.warmup:
             times.append(secs)
-    keys_per_step = n                      # one KV head, one budget, per step
+    keys_per_step = n                      # one KV head, one plan, per step
     total = sum(times)
     value = keys_per_step * len(times) / total / 1e9
-    sample = (f"each step: 1 of {wl['H']} KV heads ({wl['G']} query heads), one budget "
-              f"(cycling {list(budgets)}), {n} keys, single thread")
+    sample = (f"each step: 1 of {wl['H']} KV heads ({wl['G']} query heads), one plan "
+              f"(cycling {[plan_name(p) for p in plans]}), {n} keys, single thread")
+    cfg = config_of(wl_name, dict(wl, n=n, plans=plans), "n/a (CPU)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(wl_name, wl, "n/a (CPU)"),
+            "config": cfg,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -230,7 +271,51 @@ def run_reference(args, wl_name, wl):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ ranks
+def max_over_ranks(dist, values, device):
+    """Each value's maximum over the ranks (the slowest rank's device-timed
+    totals); the values themselves when there is no process group."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(keys_per_step, steps, world, total_ms, e2e_seconds):
+    """Whole-job Gkeys/s: every rank scans keys_per_step keys per step (weak
+    scaling), timed by the slowest rank.  -> (device-timed, end to end)."""
+    keys = keys_per_step * steps * world
+    return keys / (total_ms / 1e3) / 1e9, keys / e2e_seconds / 1e9
+
+
 # ---------------------------------------------------------------- GPU path
+def build_sessions(wl, rank, torch, fp):
+    """-> list of dicts {n, budget, keys (device float32 [H][n][d]), index,
+    plans}: the workload's sessions packed into their indices."""
+    H, G, d = wl["H"], wl["G"], wl["d"]
+    if wl.get("sessions"):
+        params = synth.agent_session_params(wl["sessions"], base_seed=1000 + 100 * rank,
+                                            n_kv_heads=H, head_dim=d)
+    else:
+        sigma, _ = synth.channel_sigma(rank, H, d)
+        params = [dict(seed=rank, n=wl["n"], budget=None, sigma=sigma)]
+    out = []
+    for p in params:
+        if wl.get("device_keys"):
+            keys = synth.device_keys(torch, p["sigma"], p["n"], p["seed"])
+        else:
+            ses = synth.make_session(p["seed"], H, G, p["n"], 64, head_dim=d)
+            keys = torch.from_numpy(ses.keys).cuda()
+        index = fp.KeyIndex(H, G, p["n"], d, wl["residency"])
+        index.pack(keys)
+        plans = wl["plans"] if wl.get("plans") else (("wf", p["budget"]),)
+        out.append(dict(n=p["n"], budget=p["budget"], keys=keys, index=index, plans=plans))
+    torch.cuda.synchronize()
+    return out
+
+
 def run_fathom(args, wl_name, wl):
     import torch
     import decode_fathom_plan_b200 as fp
@@ -244,27 +329,54 @@ def run_fathom(args, wl_name, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     fp.load_library()
-    H, G, n, d, k = wl["H"], wl["G"], wl["n"], wl["d"], wl["k"]
-    budgets = wl["budgets"]
+    H, G, d, k = wl["H"], wl["G"], wl["d"], wl["k"]
     Q = H * G
-    ses = synth.make_session(rank, H, G, n, budgets[0], head_dim=d)
-    keys_dev = torch.from_numpy(ses.keys).cuda()
-    index = fp.KeyIndex(H, G, n, d, wl["residency"])
-    index.pack(keys_dev)
-    torch.cuda.synchronize()
+    batched = bool(wl.get("batched"))
+    sessions = build_sessions(wl, rank, torch, fp)
     assert fp.fathom_last_device_status() == fp.FATHOM_OK
 
     link = measure_host_link(fp, torch) if wl["residency"] != "device" else None
     W, K = max(3, args.warmup), args.steps
-    qsets = synth.draw_queries(10_000 + rank, Q, d, count=W + K)
-    q_dev = torch.from_numpy(qsets.view(np.int16)).cuda()
-    bvec = [torch.full((Q,), B, dtype=torch.int32, device="cuda") for B in budgets]
-    bufs = [fp.ScanBuffers(index, k) for _ in budgets]
+    # scans of one step: (session, plan spec, buffers, budget vector)
+    jobs = []
+    for si, S in enumerate(sessions):
+        S["q"] = torch.from_numpy(synth.draw_queries(10_000 + 100 * rank + si, Q, d,
+                                                     count=W + K).view(np.int16)).cuda()
+        for spec in S["plans"]:
+            B = plan_bits(spec)
+            jobs.append(dict(s=si, spec=spec, buf=fp.ScanBuffers(S["index"], k),
+                             bvec=torch.full((Q,), B, dtype=torch.int32, device="cuda")))
+    ws_batch = None
+    if batched:
+        descs = [S["index"].desc for S in sessions]
+        ws_batch = torch.empty(max(16, fp.fathom_scan_batched_workspace_bytes(descs, k)),
+                               dtype=torch.uint8, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    def step(i, flags=0):
-        for bi in range(len(budgets)):
-            fp.plan_and_scan(index, q_dev[i], bvec[bi], bufs[bi], flags=flags)
+    def plan(j, i):
+        S = sessions[j["s"]]
+        b = j["buf"]
+        if j["spec"][0] == "wf":
+            fp.fathom_plan(S["index"].desc, S["q"][i], j["bvec"], b.t, b.t_union, b.nbytes)
+        else:
+            fp.fathom_fixed_plan(S["index"].desc, S["q"][i], j["spec"][1], b.t, b.t_union,
+                                 b.nbytes)
+
+    def step(i, flags=0, qsrc=None):
+        if batched:
+            for j in jobs:
+                plan(j, i)
+            fp.fathom_scan_topk_batched(
+                [S["index"].desc for S in sessions], [S["q"][i] for S in sessions],
+                [j["buf"].t for j in jobs], [j["buf"].t_union for j in jobs], k,
+                [j["buf"].idx for j in jobs], [j["buf"].score for j in jobs], ws_batch, flags)
+        else:
+            for j in jobs:
+                S = sessions[j["s"]]
+                plan(j, i)
+                b = j["buf"]
+                fp.fathom_scan_topk(S["index"].desc, S["q"][i], b.t, b.t_union, k, b.idx,
+                                    b.score, b.workspace, flags)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -323,63 +435,65 @@ def run_fathom(args, wl_name, wl):
     status = fp.fathom_last_device_status()
     assert status == fp.FATHOM_OK, fp.status_str(status)
 
-    # plan byte counts of the last step (identical structure every step)
-    per_budget = []
-    union_bytes_total = 0
-    for bi, B in enumerate(budgets):
-        nb = bufs[bi].nbytes.cpu().numpy()
-        qb, ub = nb[:Q].astype(np.float64), nb[Q:].astype(np.float64)
-        union_bytes_total += ub.sum()
-        per_budget.append({"B": B, "bytes_per_query": float(qb.mean()),
-                           "union_bytes_per_kv_head": float(ub.mean()),
-                           "union_factor": float(ub.sum() / (qb.sum() / G))})
-
-    # quality: recall against the exact fp32 top-k (torch, outside the path)
+    # plan byte counts and quality of the last step (same structure every step)
+    per_plan = []
+    union_bytes_total = 0.0
     with torch.no_grad():
-        qf = q_dev[W + K - 1].view(torch.bfloat16).float().reshape(H, G, d)
-        for bi, pb in enumerate(per_budget):
-            got = bufs[bi].idx.reshape(H, G, k).long()
+        for j in jobs:
+            S = sessions[j["s"]]
+            nb = j["buf"].nbytes.cpu().numpy()
+            qb, ub = nb[:Q].astype(np.float64), nb[Q:].astype(np.float64)
+            union_bytes_total += ub.sum()
+            # recall against the exact fp32 top-k (torch, outside the path)
+            qf = S["q"][W + K - 1].view(torch.bfloat16).float().reshape(H, G, d)
+            got = j["buf"].idx.reshape(H, G, k).long()
             rec = []
             for h in range(H):
-                exact = (keys_dev[h] @ qf[h].T).topk(k, dim=0).indices.T     # [G][k]
+                exact = (S["keys"][h] @ qf[h].T).topk(k, dim=0).indices.T     # [G][k]
                 for g in range(G):
                     inter = np.intersect1d(exact[g].cpu().numpy(), got[h, g].cpu().numpy())
                     rec.append(len(inter) / k)
-            pb["recall_vs_exact_fp32"] = float(np.mean(rec))
+            per_plan.append({"plan": plan_name(j["spec"]), "session": j["s"], "n_keys": S["n"],
+                             "bits_per_key": plan_bits(j["spec"]),
+                             "bytes_per_query": float(qb.mean()),
+                             "union_bytes_per_kv_head": float(ub.mean()),
+                             "union_factor": float(ub.sum() / (qb.sum() / G)),
+                             "recall_vs_exact_fp32": float(np.mean(rec))})
 
     # end to end through the public API with host buffers
-    q_host = torch.from_numpy(qsets[W:W + K].view(np.int16)).pin_memory()
-    b_host = [torch.full((Q,), B, dtype=torch.int32).pin_memory() for B in budgets]
-    q_stage = torch.empty((Q, d), dtype=torch.int16, device="cuda")
-    idx_host = [torch.empty((Q, k), dtype=torch.int32).pin_memory() for _ in budgets]
-    sc_host = [torch.empty((Q, k), dtype=torch.float32).pin_memory() for _ in budgets]
+    q_host = [torch.from_numpy(S["q"][W:W + K].cpu().numpy()).pin_memory() for S in sessions]
+    b_host = [j["bvec"].cpu().pin_memory() for j in jobs]
+    q_stage = [torch.empty((Q, d), dtype=torch.int16, device="cuda") for _ in sessions]
+    idx_host = [torch.empty((Q, k), dtype=torch.int32).pin_memory() for _ in jobs]
+    sc_host = [torch.empty((Q, k), dtype=torch.float32).pin_memory() for _ in jobs]
+    saved_q = [S["q"] for S in sessions]
     e2e_s = []
     for s in range(K):
         flush.fill_(s & 0xFF)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        for bi in range(len(budgets)):
-            q_stage.copy_(q_host[s], non_blocking=True)
-            bvec[bi].copy_(b_host[bi], non_blocking=True)
-            fp.plan_and_scan(index, q_stage, bvec[bi], bufs[bi])
-            idx_host[bi].copy_(bufs[bi].idx, non_blocking=True)
-            sc_host[bi].copy_(bufs[bi].score, non_blocking=True)
+        for si, S in enumerate(sessions):
+            q_stage[si].copy_(q_host[si][s], non_blocking=True)
+            S["q"] = q_stage[si].unsqueeze(0)
+        for ji, j in enumerate(jobs):
+            j["bvec"].copy_(b_host[ji], non_blocking=True)
+        step(0)
+        for ji, j in enumerate(jobs):
+            idx_host[ji].copy_(j["buf"].idx, non_blocking=True)
+            sc_host[ji].copy_(j["buf"].score, non_blocking=True)
         torch.cuda.synchronize()
         e2e_s.append(time.perf_counter() - t0)
-    h2d = len(budgets) * (Q * d * 2 + Q * 4)
-    d2h = len(budgets) * (Q * k * 8)
+    for S, q in zip(sessions, saved_q):
+        S["q"] = q
+    h2d = len(sessions) * Q * d * 2 + len(jobs) * Q * 4
+    d2h = len(jobs) * Q * k * 8
 
-    keys_per_step = H * n * len(budgets)
-    if dist:
-        t = torch.tensor([total_ms, sum(e2e_s)], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_total = float(t[0]), float(t[1])
-    else:
-        e2e_total = sum(e2e_s)
-    value = keys_per_step * K * world / (total_ms / 1e3) / 1e9
-    e2e_value = keys_per_step * K * world / e2e_total / 1e9
+    keys_per_step = sum(H * sessions[j["s"]]["n"] for j in jobs)
+    total_ms, e2e_total = max_over_ranks(dist, [total_ms, sum(e2e_s)], "cuda")
+    value, e2e_value = job_throughput(keys_per_step, K, world, total_ms, e2e_total)
 
-    bytes_per_launch = union_bytes_total / len(budgets)
+    launches_per_step = 1 if batched else len(jobs)
+    bytes_per_launch = union_bytes_total / launches_per_step
     avg_launch_ms = scan_ms / max(1, scan_launches)
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
     if wl["residency"] == "device":
@@ -395,20 +509,26 @@ def run_fathom(args, wl_name, wl):
                 "peak_source": peak_note, "avg_launch_us": avg_launch_ms * 1e3,
                 "algorithmic_bytes_per_launch": bytes_per_launch}
 
+    cfg = config_of(wl_name, wl, "flushed between steps (256 MiB write)",
+                    sessions=sessions if wl.get("sessions") else None)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": config_of(wl_name, wl, "flushed between steps (256 MiB write)"),
+            "config": cfg,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches), "launch_mode": "cuda_graph" if args.graph else "eager",
             "roofline": roofline, "clocks": clk,
-            "per_budget": per_budget,
+            "per_plan": per_plan,
             "step_ms_median": statistics.median(step_ms)}
     if link is not None:
         line["host_link"] = link
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(ses, wl)
+        S0 = sessions[0]
+        nh = max(1, min(4, H, (4 * 131072) // S0["n"]))
+        line["cpu_baseline"] = cpu_baseline(S0["keys"][:nh].cpu().numpy(),
+                                            S0["q"][0].cpu().numpy().view(np.uint16), G,
+                                            S0["plans"], k)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

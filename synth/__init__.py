@@ -89,6 +89,52 @@ def _draw_keys(rng: np.random.Generator, sigma: np.ndarray, n: int) -> np.ndarra
     return keys
 
 
+def channel_sigma(seed: int, n_kv_heads: int, head_dim: int = HEAD_DIM,
+                  rng: Optional[np.random.Generator] = None):
+    """Steps 1-2 of the recipe alone (the first draws of make_session):
+    -> (sigma float64 [H][d] with outliers applied, outliers int64 [H][4])."""
+    if rng is None:
+        rng = np.random.Generator(np.random.PCG64(seed))
+    sigma = rng.lognormal(0.0, SIGMA_LOGNORMAL, size=(n_kv_heads, head_dim))
+    outliers = np.empty((n_kv_heads, N_OUTLIERS), dtype=np.int64)
+    for h in range(n_kv_heads):
+        outliers[h] = rng.choice(head_dim, N_OUTLIERS, replace=False)
+        sigma[h, outliers[h]] *= OUTLIER_MULT
+    return sigma, outliers
+
+
+def device_keys(torch, sigma: np.ndarray, n: int, seed: int, device="cuda"):
+    """Keys of step 3 drawn on a device: N(0, 1) from torch's generator on
+    `device` seeded with `seed`, times sigma, as float32 [H][n][d].  This is
+    a different random stream from step 3's numpy draw (same distribution);
+    the benchmark uses it for workloads whose keys would take minutes and
+    tens of GB to draw on the host."""
+    H, d = sigma.shape
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    sig = torch.as_tensor(sigma, dtype=torch.float32, device=device)
+    keys = torch.empty((H, n, d), dtype=torch.float32, device=device)
+    for h in range(H):
+        keys[h] = torch.randn((n, d), generator=gen, device=device, dtype=torch.float32) * sig[h]
+    return keys
+
+
+def agent_session_params(n_sessions: int = 16, base_seed: int = 1000, n_kv_heads: int = 8,
+                         n_min: int = 65536, n_max: int = 524288,
+                         budget_choices=(68, 92, 136), head_dim: int = HEAD_DIM):
+    """The draws of make_agent_sessions that precede the keys: per session s
+    (seed base_seed + s) its key count n, budget B, sigma and outliers.
+    -> list of dicts {seed, n, budget, sigma, outliers}."""
+    out = []
+    for s in range(n_sessions):
+        rng = np.random.Generator(np.random.PCG64(base_seed + s))
+        n = int(rng.integers(n_min, n_max, endpoint=True))
+        B = int(rng.choice(np.asarray(budget_choices)))
+        sigma, outliers = channel_sigma(base_seed + s, n_kv_heads, head_dim, rng=rng)
+        out.append(dict(seed=base_seed + s, n=n, budget=B, sigma=sigma, outliers=outliers))
+    return out
+
+
 def make_session(seed: int, n_kv_heads: int, group: int, n_keys: int,
                  budget, head_dim: int = HEAD_DIM, n_planted: int = 0,
                  rng: Optional[np.random.Generator] = None) -> Session:
@@ -97,11 +143,7 @@ def make_session(seed: int, n_kv_heads: int, group: int, n_keys: int,
     if rng is None:
         rng = np.random.Generator(np.random.PCG64(seed))
     H, G, n, d = n_kv_heads, group, n_keys, head_dim
-    sigma = rng.lognormal(0.0, SIGMA_LOGNORMAL, size=(H, d))
-    outliers = np.empty((H, N_OUTLIERS), dtype=np.int64)
-    for h in range(H):
-        outliers[h] = rng.choice(d, N_OUTLIERS, replace=False)
-        sigma[h, outliers[h]] *= OUTLIER_MULT
+    sigma, outliers = channel_sigma(seed, H, d, rng=rng)
     keys = _draw_keys(rng, sigma, n)
     q32 = rng.standard_normal((H * G, d)).astype(np.float32)
     q_bf16 = f32_to_bf16_bits(q32)
