@@ -17,40 +17,39 @@
 // per query head", with no per-bit work.
 //
 // Data path.  A KV head reads the union plan T_c = max_g t_gc of its G query
-// heads once.  Union channels are ordered by the set of query heads reading
-// them (stable counting sort), so the fma pattern is chosen once per run of
-// equal sets instead of once per channel.  A stage is 8 union channels x 4
-// plane rows x a chunk of up to 64 plane words (2048 keys); rows past a
-// channel's depth are zero-filled by cp.async without a global read, so every
-// channel is processed the same way.  Stages are copied into shared memory
-// with 16-byte cp.async, STAGES buffers deep.  Thread (column, row r) owns
-// keys 32*column + 4m + r, m = 0..7: a funnel-shift rotate and a mask move
-// bit 4m+r of each plane word to bit 4m+p, so one register holds the
-// thread's 8 nibbles; each nibble becomes a float by OR-ing it under the
-// mantissa of a power of two and subtracting that power (exact), two at a
-// time with __fadd2_rn; each query head reading the channel adds W*v with
-// __ffma2_rn (two keys per instruction).
-//
-// Work distribution: persistent CTAs (as many as are resident) each take an
-// equal contiguous range of 4-word column groups of the (session, KV head)
-// sequence, so there is no partial last wave; a CTA rebuilds its per-head
-// tables only when its range crosses into the next head.
+// heads once.  prep_kernel builds each KV head's tables once (union channel
+// list, plane rows, weights, biases); every later CTA copies them.  Union
+// channels are listed by the set of query heads reading them at full depth,
+// and an 8-channel stage runs a body specialised to its set, so a query head
+// that does not read a channel issues no fma for it.  A stage is 8 union
+// channels x 4 plane rows x a chunk of up to 64 plane words (2048 keys);
+// rows past a channel's depth are zero-filled in shared memory with no
+// global read.  Stages are copied with 16-byte cp.async, 3 buffers deep.
+// Thread (column, row r) owns keys 32*column + 4m + r, m = 0..7: a
+// funnel-shift rotate and a mask move bit 4m+r of each plane word to bit
+// 4m+p, so one register holds the thread's 8 nibbles; each nibble becomes a
+// float by OR-ing it under the mantissa of a power of two and subtracting
+// that power (exact), two at a time with __fadd2_rn; each reading query head
+// adds W*v with __ffma2_rn (two keys per instruction).  One CTA per 64-word
+// chunk of a KV head; host-resident planes are first fetched into a device
+// mirror (fetch.cu) and read from there.
 //
 // No tensor cores: this is a sparse binary-weighted reduction.
 //
 // Selection without materialising n scores per query:
-//   1. sample:   score evenly strided whole tiles (about 3% of the keys) and
-//                write their order keys to the workspace;
-//   2. theta:    per query, theta = the r-th largest sampled key, with r
-//                about 2*k*m/n, so ~2k keys are expected to pass;
-//   3. filter:   the full scan appends (key, index) of every key scoring
-//                >= theta to a per-query candidate buffer;
-//   4. final:    if k <= candidates <= capacity, an exact radix select over
-//                the unique composite (order key, ~index) and a bitonic sort
-//                give the top-k; otherwise the query is flagged;
-//   5. fallback: a flagged query is redone exactly by one CTA that
-//                recomputes its scores once per radix digit (no score
-//                buffer), so results never depend on the sample.
+//   1. threshold: per query, score evenly strided whole tiles (about 3% of
+//                 the keys) from the query's own plan, and take theta = the
+//                 r-th largest sampled key, r about 2*k*m/n, so ~2k keys are
+//                 expected to pass;
+//   2. filter:    the full scan appends (key, index) of every key scoring
+//                 >= theta to a per-query candidate buffer;
+//   3. final:     if k <= candidates <= capacity, an exact radix select over
+//                 the unique composite (order key, ~index) gives the top-k,
+//                 listed in ascending key index; otherwise the query is
+//                 flagged;
+//   4. fallback:  a flagged query is redone exactly by one CTA that
+//                 recomputes its scores once per radix digit (no score
+//                 buffer), so results never depend on the sample.
 // Correctness needs only that every key scoring at least the k-th largest
 // score is a candidate, which "count >= k" guarantees for any theta.
 #include <math.h>
@@ -78,12 +77,11 @@ struct SessionDesc {
     int32_t *out_idx;            // [Q][k]
     float *out_score;            // [Q][k]
     uint32_t *qstate;            // [Q][4]: theta, count, fallback flag, spare
-    uint32_t *sample;            // [Q][m_keys]
     unsigned long long *cand;    // [Q][cap]
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int group_begin, sample_group_begin, q_begin, head_begin;   // sample_group_begin: sampled-chunk index
+    int group_begin, q_begin, head_begin;
 };
 
 template <int NS>
@@ -201,18 +199,40 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
                            const uint8_t *t_rows, const uint16_t *q_rows, const float *mn_h,
                            const float *sc_h)
 {
+    __shared__ double bias_part[kScanThreads / 32][GP];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c = tid;
-    const int T = (c < d) ? min((int)tu_row[c], kBits) : 0;
+    const bool in = c < d;
+    // every input of channel c, loaded at once
+    int T = 0;
+    float sc = 0.0f, mn = 0.0f;
+    int tg[GP];
+    float qf[GP];
+    if (in) {
+        T = min((int)tu_row[c], kBits);
+        sc = sc_h[c];
+        mn = mn_h[c];
+    }
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        const bool live = in && g < G;
+        tg[g] = live ? (int)t_rows[g * d + c] : 0;
+        qf[g] = live ? bf16_to_float(q_rows[g * d + c]) : 0.0f;
+    }
     const bool has = T > 0;
     // reader sets of this channel: full = queries reading all T planes,
-    // partial = queries reading 0 < t < T of them
+    // partial = queries reading 0 < t < T of them; each query's bias term
+    // q_gc * (mn_c + scale_c * (2^(4-t) - 1) / 2) at its own clamped depth
     unsigned full = 0, partial = 0;
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-        const int tg = (has && g < G) ? min((int)t_rows[g * d + c], T) : 0;
-        if (has && tg == T) full |= 1u << g;
-        else if (tg > 0) partial |= 1u << g;
+        tg[g] = min(tg[g], T);
+        if (has && tg[g] == T) full |= 1u << g;
+        else if (tg[g] > 0) partial |= 1u << g;
+        double term = in ? (double)qf[g] * ((double)mn + (double)sc * bin_offset(tg[g])) : 0.0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
+        if (lane == 0) bias_part[warp][g] = term;
     }
     const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
     if (lane == 0) sm.part[warp] = __popc(bal);
@@ -235,6 +255,12 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     int U = 0;
 #pragma unroll
     for (int w = 0; w < kScanThreads / 32; ++w) U += sm.part[w];
+    if (tid < GP) {
+        double acc = 0.0;
+#pragma unroll
+        for (int w = 0; w < kScanThreads / 32; ++w) acc += bias_part[w][tid];
+        sm.bias[tid] = (float)acc;
+    }
     if (mask_ordered<GP>()) {
         // warp 0 turns the (warp, key) counts into exclusive offsets in
         // (key, warp) order
@@ -273,20 +299,14 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     const int n_stages = (U + kStageChannels - 1) / kStageChannels;
     if (has) {
         const int u = base + lane_rank;
-        const float sc = sc_h[c];
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
-            int tg = 0;
-            float w = 0.0f;
-            if (g < G) {
-                tg = min((int)t_rows[g * d + c], T);
-                w = __fmul_rn(bf16_to_float(q_rows[g * d + c]), sc);
-            }
+            const float w = __fmul_rn(qf[g], sc);
             // full-depth readers use W2 in the unconditional fma; others add 0
             // there and, if partial, their own masked term
-            sm.W2[u][g] = (tg == T) ? make_float2(w, w) : make_float2(0.0f, 0.0f);
+            sm.W2[u][g] = (tg[g] == T) ? make_float2(w, w) : make_float2(0.0f, 0.0f);
             sm.Wp[u][g] = w;
-            sm.tq[u][g] = (uint8_t)tg;
+            sm.tq[u][g] = (uint8_t)tg[g];
         }
         sm.meta[u] = full | (partial << 16);
         if (partial) sm.stage_partial[u / kStageChannels] = 1;
@@ -299,20 +319,6 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     if (tid == 0) {
         sm.U = U;
         sm.n_stages = n_stages;
-    }
-    // bias_g over every channel, each at its own (clamped) depth
-    if (warp < GP) {
-        double acc = 0.0;
-        if (warp < G) {
-            for (int cc = lane; cc < d; cc += 32) {
-                const int tg = min((int)t_rows[warp * d + cc], min((int)tu_row[cc], kBits));
-                const double qf = (double)bf16_to_float(q_rows[warp * d + cc]);
-                acc += qf * ((double)mn_h[cc] + (double)sc_h[cc] * bin_offset(tg));
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-        if (lane == 0) sm.bias[warp] = (float)acc;
     }
     __syncthreads();
 }
@@ -567,20 +573,6 @@ __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
     return si;
 }
 
-// ----------------------------------------------------------- sampled pass
-// Scores of the sampled keys, latency-first: a CTA takes 16 plane words
-// (512 keys) of one sampled tile, copies every selected plane row of them
-// into shared memory at once, and splits the union channels over four
-// groups of 64 threads (stage st goes to group st % 4); the groups' partial
-// sums are added in group order.  The order keys of all 512 keys (0 past the
-// last key) go to the sample buffer.
-constexpr int kSampleCols = 16;
-constexpr int kSampleGroups = kScanThreads / (kSampleCols * 4);   // 4
-constexpr int kSampleChunks = kTileCols / kSampleCols;            // per sampled tile
-constexpr int kMaxStages = kMaxHeadDim / kStageChannels;          // 32
-typedef uint32_t (*SampleBuf)[kStageRows][kSampleCols];
-constexpr size_t kSampleSmem = (size_t)kMaxStages * kStageRows * kSampleCols * sizeof(uint32_t);
-
 // One CTA per (session, KV head): build the head's scan tables and store
 // them for the sampling and scanning CTAs (load_head).
 template <int NS, int GP>
@@ -600,97 +592,6 @@ __global__ void __launch_bounds__(kScanThreads) prep_kernel(const __grid_constan
     const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
     uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
     for (int i = threadIdx.x; i < kUnits; i += blockDim.x) dst[i] = src[i];
-}
-
-template <int NS, int GP>
-__global__ void __launch_bounds__(kScanThreads) sample_kernel(const __grid_constant__ Batch<NS> b)
-{
-    __shared__ ScanMeta<GP> sm;
-    extern __shared__ __align__(16) uint32_t sample_dyn[];
-    SampleBuf buf = reinterpret_cast<SampleBuf>(sample_dyn);
-    const int item = blockIdx.x;
-    int si = 0;
-    for (int s2 = 1; s2 < b.n_sessions; ++s2)
-        if (b.s[s2].sample_group_begin <= item) si = s2;
-    const SessionDesc &S = b.s[si];
-    const int per_head = S.m_tiles * kSampleChunks;
-    const int local = item - S.sample_group_begin;
-    const int h = local / per_head;
-    const int ci = local - h * per_head;
-    const int tile_i = ci / kSampleChunks, chunk = ci - tile_i * kSampleChunks;
-    const int col_lo = tile_i * S.sample_stride * kTileCols + chunk * kSampleCols;
-    const int col_hi = min(S.n_cols, col_lo + kSampleCols);
-    const int G = b.G, q0 = h * G;
-    load_head<GP>(sm, S.tables, h);
-    // every plane row of every stage, 4 x 16 bytes per row
-    const int n_stages = sm.n_stages;
-    const int n_chunks = n_stages * kStageRows * (kSampleCols / 4);
-    for (int e = threadIdx.x; e < n_chunks; e += kScanThreads) {
-        const int row = e >> 2, part = e & 3;          // row over all stages
-        const int col = col_lo + part * 4;
-        const uint32_t g = sm.row_g[row];
-        const bool live = col < col_hi && g != 0xFFFFFFFFu;
-        copy_or_zero16(&buf[row / kStageRows][row % kStageRows][part * 4],
-                       S.planes + (size_t)g * (size_t)S.n_words + col, live);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-
-    const int grp = threadIdx.x / (kSampleCols * 4);
-    const int lt = threadIdx.x - grp * kSampleCols * 4;
-    const int col = lt >> 2, r = lt & 3;
-    uint32_t sh[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
-    float neg[4];
-    magic_negatives(neg);
-    float2 acc[GP][4];
-#pragma unroll
-    for (int g = 0; g < GP; ++g)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[g][i] = make_float2(0.0f, 0.0f);
-    for (int st = grp; st < n_stages; st += kSampleGroups) {
-        const int u0 = st * kStageChannels;
-        compute_stage<GP, kSampleCols>(sm, st, buf[st], u0, min(u0 + kStageChannels, sm.U), col,
-                                       sh, neg, acc);
-    }
-    __syncthreads();   // the stage buffer becomes the reduction buffer
-    float2 *red = reinterpret_cast<float2 *>(sample_dyn);    // [groups-1][64][GP*4]
-    if (grp > 0) {
-#pragma unroll
-        for (int g = 0; g < GP; ++g)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                red[((grp - 1) * kSampleCols * 4 + lt) * GP * 4 + g * 4 + i] = acc[g][i];
-    }
-    __syncthreads();
-    if (grp == 0) {
-#pragma unroll
-        for (int o = 1; o < kSampleGroups; ++o)
-#pragma unroll
-            for (int g = 0; g < GP; ++g)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 pv = red[((o - 1) * kSampleCols * 4 + lt) * GP * 4 + g * 4 + i];
-                    acc[g][i].x += pv.x;
-                    acc[g][i].y += pv.y;
-                }
-        const int key0 = (col_lo + col) * 32 + r;
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-            if (g >= G) break;
-            const float bias = sm.bias[g];
-            uint32_t *dst = S.sample + (size_t)(q0 + g) * S.m_keys + (size_t)tile_i * kTileKeys +
-                            (chunk * kSampleCols + col) * 32 + r;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int j = key0 + 4 * m;
-                dst[4 * m] = (j < S.n && col_lo + col < col_hi)
-                                 ? order_key(score_of(acc[g], m, bias)) : 0u;
-            }
-        }
-    }
 }
 
 // ------------------------------------------------------- filtered scan
@@ -1087,15 +988,29 @@ __device__ void emit_in_index_order(const unsigned long long *sel, int k, int n,
     }
 }
 
-// ---------------------------------------------------------------- theta
-// One CTA per query: theta = the sample_rank-th largest sampled order key,
-// and reset the candidate count and fallback flag.
-template <int NS>
-__global__ void __launch_bounds__(kSelThreads) theta_kernel(const __grid_constant__ Batch<NS> b,
-                                                            uint32_t force_exact)
+// ------------------------------------------------------- sampled threshold
+// One CTA per query: score the query's sampled keys (m_tiles whole 64-word
+// tiles, evenly strided) from its own plan, then theta = the sample_rank-th
+// largest sampled order key.  Only the query's own channels are read (t > 0,
+// from the KV head's tables), 8 channels x 2 tiles per stage, two stages in
+// flight.  Every query of a KV head reads its sampled rows itself; they are
+// a few tens of KB and mostly L2 hits.
+constexpr int kThetaTilesPerPass = kSelThreads / kScanThreads;            // 2
+constexpr int kThetaCols = kThetaTilesPerPass * kTileCols;                // 128 words
+typedef uint32_t (*ThetaBuf)[kStageRows][kThetaCols];
+constexpr size_t kThetaStageBytes = (size_t)kStageRows * kThetaCols * sizeof(uint32_t);
+
+template <int NS, int GP>
+__global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_constant__ Batch<NS> b,
+                                                                uint32_t force_exact)
 {
-    extern __shared__ uint32_t vals[];
+    extern __shared__ __align__(16) uint32_t th_dyn[];
+    __shared__ ScanMeta<GP> sm;
     __shared__ SelShared ss;
+    __shared__ uint16_t own[kMaxHeadDim];   // union positions of the query's channels
+    __shared__ int n_own_s;
+    ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
+    uint32_t *vals = th_dyn + 2 * kStageRows * kThetaCols;
     const int gq = blockIdx.x;
     const int si = find_session_by_query(b, gq);
     const SessionDesc &S = b.s[si];
@@ -1109,14 +1024,100 @@ __global__ void __launch_bounds__(kSelThreads) theta_kernel(const __grid_constan
         if (threadIdx.x == 0) { st[0] = 0; st[1] = 0; st[2] = 0; }
         return;
     }
+    const int G = b.G;
+    const int h = qq / G, g = qq - h * G;
+    load_head<GP>(sm, S.tables, h);
+    if (threadIdx.x < 32) {   // the query's channels, in union order
+        const int lane = threadIdx.x;
+        int n = 0;
+        for (int u0 = 0; u0 < sm.U; u0 += 32) {
+            const int u = u0 + lane;
+            const bool mine = u < sm.U && sm.tq[u][g] > 0;
+            const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
+            if (mine) own[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)u;
+            n += __popc(bal);
+        }
+        if (lane == 0) n_own_s = n;
+    }
+    __syncthreads();
+    const int n_own = n_own_s;
+    const int n_stages = (n_own + kStageChannels - 1) / kStageChannels;
+    const int sub = threadIdx.x / kScanThreads;             // tile of the pass
+    const int lt = threadIdx.x - sub * kScanThreads;
+    const int col = lt >> 2, r = lt & 3;
+    uint32_t sh[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
+    float neg[4];
+    magic_negatives(neg);
+    const float bias = sm.bias[g];
+    // copy stage s of tile pass t0 into buffer bufi: rows of own channels
+    // 8s..8s+7 (4 slots each), 2 tiles x 16 column groups per row
+    auto load = [&](int t0, int s, int bufi) {
+        for (int e = threadIdx.x; e < kStageRows * (kThetaCols / 4); e += kSelThreads) {
+            const int row = e / (kThetaCols / 4), part = e - row * (kThetaCols / 4);
+            const int tsub = part / (kTileCols / 4), c16 = part - tsub * (kTileCols / 4);
+            const int tile = t0 + tsub;
+            const int j = s * kStageChannels + row / kBits;
+            const int wcol = tile * S.sample_stride * kTileCols + c16 * 4;
+            uint32_t grow = 0xFFFFFFFFu;
+            if (j < n_own && tile < S.m_tiles && wcol < S.n_cols)
+                grow = sm.row_g[(int)own[j] * kBits + (row % kBits)];
+            copy_or_zero16(&stage[bufi][row][part * 4],
+                           S.planes + (size_t)grow * (size_t)S.n_words + wcol,
+                           grow != 0xFFFFFFFFu);
+        }
+        cp_async_commit();
+    };
+    for (int t0 = 0; t0 < S.m_tiles; t0 += kThetaTilesPerPass) {
+        float2 acc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        __syncthreads();   // the buffers are free
+        if (n_stages > 0) load(t0, 0, 0);
+        for (int s2 = 0; s2 < n_stages; ++s2) {
+            if (s2 + 1 < n_stages) {
+                load(t0, s2 + 1, (s2 + 1) & 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();
+            const uint32_t(*rows)[kThetaCols] = stage[s2 & 1];
+            const int j1 = min(n_own, (s2 + 1) * kStageChannels);
+            for (int j = s2 * kStageChannels; j < j1; ++j) {
+                const int u = own[j];
+                const int tg = sm.tq[u][g];
+                const uint32_t keep = ((0xFu << (kBits - tg)) & 0xFu) * 0x11111111u;
+                const uint32_t nib =
+                    gather_nibbles<kThetaCols>(rows + kBits * (j - s2 * kStageChannels),
+                                               sub * kTileCols + col, sh) & keep;
+                float2 v[4];
+                nibbles_to_floats(nib, neg, v);
+                const float w = sm.Wp[u][g];
+                const float2 w2 = make_float2(w, w);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = __ffma2_rn(v[i], w2, acc[i]);
+            }
+            __syncthreads();   // buffer s2 & 1 is reloaded two stages on
+        }
+        const int tile = t0 + sub;
+        if (tile < S.m_tiles) {
+            const int wcol = tile * S.sample_stride * kTileCols + col;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int j = wcol * 32 + r + 4 * m;
+                vals[tile * kTileKeys + col * 32 + r + 4 * m] =
+                    (wcol < S.n_cols && j < S.n) ? order_key(score_of(acc, m, bias)) : 0u;
+            }
+        }
+    }
+    __syncthreads();
     const int m = S.m_keys;
-    const uint4 *src = reinterpret_cast<const uint4 *>(S.sample + (size_t)qq * m);
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (int i = threadIdx.x; i < m / 4; i += kSelThreads) {
-        const uint4 v = src[i];
-        reinterpret_cast<uint4 *>(vals)[i] = v;
-        lo = min(min(lo, min(v.x, v.y)), min(v.z, v.w));
-        hi = max(max(hi, max(v.x, v.y)), max(v.z, v.w));
+    for (int i = threadIdx.x; i < m; i += kSelThreads) {
+        lo = min(lo, vals[i]);
+        hi = max(hi, vals[i]);
     }
     sel_range(ss, lo, hi);
     const uint32_t base = ss.lo;
@@ -1319,7 +1320,7 @@ Sizing size_session(int n, int n_words, int k)
 }
 
 struct WsLayout {
-    size_t qstate, sample, cand, tables, mirror, total;
+    size_t qstate, cand, tables, mirror, total;
 };
 
 // Query heads per KV head rounded up to the kernels' template width.
@@ -1345,13 +1346,10 @@ inline size_t plane_bytes(const fathom_index &ix)
 WsLayout layout_session(const fathom_index &ix, int k, size_t at)
 {
     const int Q = ix.n_kv_heads * ix.group;
-    const Sizing z = size_session(ix.n_keys, ix.n_words, k);
     const int cap = capacity_for(std::min(k, kMaxFastK));
     WsLayout L{};
     L.qstate = at;
     at += align256((size_t)Q * kQueryStateWords * sizeof(uint32_t));
-    L.sample = at;
-    at += align256((size_t)Q * z.m_keys * sizeof(uint32_t));
     L.cand = at;
     at += align256((size_t)Q * cap * sizeof(unsigned long long));
     L.tables = at;
@@ -1383,9 +1381,8 @@ cudaError_t ensure_smem(int (&done)[64], Kernel kernel, size_t max_bytes)
 // One set of "limit raised" flags per kernel instantiation.
 template <int NS>
 struct SmemFlags {
-    static int theta[64], final_[64], fallback[64];
+    static int final_[64], fallback[64];
 };
-template <int NS> int SmemFlags<NS>::theta[64];
 template <int NS> int SmemFlags<NS>::final_[64];
 template <int NS> int SmemFlags<NS>::fallback[64];
 
@@ -1419,8 +1416,7 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 }
 
 template <int NS, int GP>
-cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_groups,
-                      int total_queries, int total_heads, int max_m_keys, const FetchJob *fetch,
+cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int total_heads, int max_m_keys, const FetchJob *fetch,
                       int n_fetch, uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
 {
     cudaError_t e;
@@ -1440,22 +1436,19 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_sample_gr
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "prep launch");
         ++launches;
     }
-    if (!force && total_sample_groups > 0) {
-        static int sample_smem_set[64];
-        if ((e = ensure_smem(sample_smem_set, sample_kernel<NS, GP>, kSampleSmem)) != cudaSuccess)
-            return note_error(e, "sample set-up");
-        const int ctas = total_sample_groups;   // one CTA per sampled 16-word chunk
-        sample_kernel<NS, GP><<<ctas, kScanThreads, kSampleSmem, stream>>>(bt);
-        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "sample launch");
+    {
+        // sampled scores and theta per query (or the exact-path flags)
+        static int threshold_smem_set[64];
+        auto kern = threshold_kernel<NS, GP>;
+        const size_t dyn = 2 * kThetaStageBytes + (size_t)max_m_keys * sizeof(uint32_t);
+        if ((e = ensure_smem(threshold_smem_set, kern,
+                             2 * kThetaStageBytes + (size_t)kSampleMaxKeys * sizeof(uint32_t))) !=
+            cudaSuccess)
+            return note_error(e, "threshold set-up");
+        kern<<<total_queries, kSelThreads, dyn, stream>>>(bt, force ? 1u : 0u);
+        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "threshold launch");
         ++launches;
     }
-    const size_t theta_smem = (size_t)max_m_keys * sizeof(uint32_t);
-    if ((e = ensure_smem(SmemFlags<NS>::theta, theta_kernel<NS>,
-                         (size_t)kSampleMaxKeys * sizeof(uint32_t))) != cudaSuccess)
-        return note_error(e, "theta set-up");
-    theta_kernel<NS><<<total_queries, kSelThreads, theta_smem, stream>>>(bt, force ? 1u : 0u);
-    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "theta launch");
-    ++launches;
     if (!force && total_groups > 0) {
         const bool timed = hook && hook->enabled && n_fetch == 0;
         const int per_cta = kTileGroups;   // one 64-word chunk per CTA
@@ -1508,7 +1501,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, sgroups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
+    int groups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
     FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
@@ -1533,7 +1526,6 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.out_idx = ss[s].out_idx;
         D.out_score = ss[s].out_score;
         D.qstate = reinterpret_cast<uint32_t *>(base + L.qstate);
-        D.sample = reinterpret_cast<uint32_t *>(base + L.sample);
         D.cand = reinterpret_cast<unsigned long long *>(base + L.cand);
         D.tables = reinterpret_cast<unsigned char *>(base + L.tables);
         D.H = ix.n_kv_heads;
@@ -1547,23 +1539,21 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
         D.group_begin = groups;
-        D.sample_group_begin = sgroups;
         D.q_begin = queries;
         D.head_begin = heads;
         heads += ix.n_kv_heads;
         groups += D.H * D.col_groups;
-        sgroups += D.H * D.m_tiles * kSampleChunks;   // sampled 16-word chunks
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    return run_batch<NS, 8>(bt, groups, sgroups, queries, heads, max_m, fetch, n_fetch, flags,
+    return run_batch<NS, 8>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
 }
 

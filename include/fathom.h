@@ -191,10 +191,11 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
  * array that the library reserves as a static __device__ variable on every
  * GPU that loads it, held until the process exits.
  *   - Same arguments and results as fathom_scan_topk, minus the workspace.
- *   - A problem needing more than 8 MiB of scratch (about one Qwen3-8B-shaped
- *     layer, 32 query heads, at up to 1,048,576 keys with k <= 2048) is
- *     rejected with FATHOM_ERR_WORKSPACE before anything is enqueued; use
- *     fathom_scan_topk for it.
+ *   - A problem needing more than 8 MiB of scratch is rejected with
+ *     FATHOM_ERR_WORKSPACE before anything is enqueued; use fathom_scan_topk
+ *     for it.  For a device index, a layer of 64 query heads at 1,048,576
+ *     keys with k <= 2048 needs 6.3 MiB; a host-resident index also needs
+ *     room for its plane mirror, so only small ones fit.
  *   - The first call on each device looks up the scratch array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
  *     first call before any stream capture.

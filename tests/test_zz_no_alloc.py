@@ -72,7 +72,7 @@ def test_static_scratch_rejects_problems_beyond_its_size():
     fp.load_library()
     n = 1 << 20
     fake = 0x10000    # never dereferenced: the size check comes first
-    big = fp.fathom_index(8, 8, 128, n, fp.fathom_n_words(n), 0, fake, fake, fake, fake,
+    big = fp.fathom_index(16, 8, 128, n, fp.fathom_n_words(n), 0, fake, fake, fake, fake,
                           fake, fake)
     assert fp.fathom_scan_workspace_bytes(big, 2048) > 8 << 20
     rc = fp.load_library().fathom_scan_topk_static(ctypes.byref(big), fake, fake, fake, 2048,
