@@ -17,8 +17,8 @@
 // per query head", with no per-bit work.
 //
 // Data path.  A KV head reads the union plan T_c = max_g t_gc of its G query
-// heads once.  prep_kernel builds each KV head's tables once (union channel
-// list, plane rows, weights, biases); every later CTA copies them.  Union
+// heads once.  The threshold kernel builds each KV head's tables once (union
+// channel list, plane rows, weights, biases); every scanning CTA copies them.  Union
 // channels are listed by the set of query heads reading them at full depth,
 // and an 8-channel stage runs a body specialised to its set, so a query head
 // that does not read a channel issues no fma for it.  A stage is 8 union
@@ -81,7 +81,7 @@ struct SessionDesc {
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int group_begin, q_begin, head_begin;
+    int group_begin, q_begin;
 };
 
 template <int NS>
@@ -189,11 +189,13 @@ __device__ __forceinline__ double bin_offset(int t)
 }
 
 // ------------------------------------------------------- per-head set-up
-// Builds the union channel list (channel order), plane-row table, weights
+// Builds the union channel list (by reader set, then channel, for groups of
+// up to 4 query heads; channel order otherwise), plane-row table, weights
 // (zero for a query that does not read the channel at full union depth) and
 // biases for query heads q_rows[0..G) of KV head h.
 // tu_row: the union plan to read; t_rows: each query's own plan.
-// 256 threads, d <= 256.  Ends with a barrier.
+// Thread c handles channel c: at least 256 threads, d <= 256.  Ends with a
+// barrier.
 template <int GP>
 __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t *tu_row,
                            const uint8_t *t_rows, const uint16_t *q_rows, const float *mn_h,
@@ -232,10 +234,10 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
         double term = in ? (double)qf[g] * ((double)mn + (double)sc * bin_offset(tg[g])) : 0.0;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
-        if (lane == 0) bias_part[warp][g] = term;
+        if (lane == 0 && warp < kScanThreads / 32) bias_part[warp][g] = term;
     }
     const unsigned bal = __ballot_sync(0xFFFFFFFFu, has);
-    if (lane == 0) sm.part[warp] = __popc(bal);
+    if (lane == 0 && warp < kScanThreads / 32) sm.part[warp] = __popc(bal);
     if (tid < kMaxHeadDim / kStageChannels) {
         sm.stage_partial[tid] = 0;
         sm.stage_mask[tid] = 0u;
@@ -247,7 +249,7 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
 #pragma unroll
         for (unsigned v = 0; v < (1u << GP); ++v) {
             const unsigned b = __ballot_sync(0xFFFFFFFFu, has && key == v);
-            if (lane == 0) sm.order[warp][v] = __popc(b);
+            if (lane == 0 && warp < kScanThreads / 32) sm.order[warp][v] = __popc(b);
             if (key == v) lane_rank = __popc(b & ((1u << lane) - 1u));
         }
     }
@@ -323,8 +325,8 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     __syncthreads();
 }
 
-// Per-head tables are built once per (session, KV head) by prep_kernel and
-// copied by every CTA that scans the head: one round trip instead of the
+// Per-head tables are built once per (session, KV head) by threshold_kernel
+// and copied by every CTA that scans the head: one round trip instead of the
 // dependent loads, barriers and fp64 bias sums of setup_head.  Ends with a
 // barrier; completes every cp.async group in flight.
 template <int GP>
@@ -571,27 +573,6 @@ __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
     for (int s = 1; s < b.n_sessions; ++s)
         if (b.s[s].q_begin <= gq) si = s;
     return si;
-}
-
-// One CTA per (session, KV head): build the head's scan tables and store
-// them for the sampling and scanning CTAs (load_head).
-template <int NS, int GP>
-__global__ void __launch_bounds__(kScanThreads) prep_kernel(const __grid_constant__ Batch<NS> b)
-{
-    __shared__ ScanMeta<GP> sm;
-    const int item = blockIdx.x;
-    int si = 0;
-    for (int s2 = 1; s2 < b.n_sessions; ++s2)
-        if (b.s[s2].head_begin <= item) si = s2;
-    const SessionDesc &S = b.s[si];
-    const int h = item - S.head_begin;
-    const int G = b.G, d = b.d, q0 = h * G;
-    setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)q0 * d, S.q + (size_t)q0 * d,
-                   S.mn + h * d, S.scale + h * d);
-    constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
-    const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
-    uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
-    for (int i = threadIdx.x; i < kUnits; i += blockDim.x) dst[i] = src[i];
 }
 
 // ------------------------------------------------------- filtered scan
@@ -990,15 +971,19 @@ __device__ void emit_in_index_order(const unsigned long long *sel, int k, int n,
 
 // ------------------------------------------------------- sampled threshold
 // One CTA per query: score the query's sampled keys (m_tiles whole 64-word
-// tiles, evenly strided) from its own plan, then theta = the sample_rank-th
-// largest sampled order key.  Only the query's own channels are read (t > 0,
-// from the KV head's tables), 8 channels x 2 tiles per stage, two stages in
-// flight.  Every query of a KV head reads its sampled rows itself; they are
-// a few tens of KB and mostly L2 hits.
+// tiles, evenly strided) from its own plan, then theta = the lower edge of a
+// 2^-22-of-the-range bin holding the sample_rank-th largest sampled order key
+// (two 11-bit radix passes; any theta is correct, it only sizes the candidate
+// set).  The query's channels, weights and bias come straight from its plan
+// and the index statistics; the CTA of each KV head's first query also
+// builds that head's scan tables for the filtering pass.  Stages of 8 own
+// channels x 2 tiles are copied with cp.async, two in flight; every query of
+// a KV head reads its sampled rows itself (a few tens of KB, mostly L2 hits).
 constexpr int kThetaTilesPerPass = kSelThreads / kScanThreads;            // 2
 constexpr int kThetaCols = kThetaTilesPerPass * kTileCols;                // 128 words
 typedef uint32_t (*ThetaBuf)[kStageRows][kThetaCols];
 constexpr size_t kThetaStageBytes = (size_t)kStageRows * kThetaCols * sizeof(uint32_t);
+constexpr int kThetaResolutionBits = 2 * kSelBits;
 
 template <int NS, int GP>
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_constant__ Batch<NS> b,
@@ -1007,15 +992,28 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     extern __shared__ __align__(16) uint32_t th_dyn[];
     __shared__ ScanMeta<GP> sm;
     __shared__ SelShared ss;
-    __shared__ uint16_t own[kMaxHeadDim];   // union positions of the query's channels
-    __shared__ int n_own_s;
+    __shared__ uint16_t own_c[kMaxHeadDim];   // the query's channels (t > 0) ...
+    __shared__ uint8_t own_t[kMaxHeadDim];    // ... their depths ...
+    __shared__ float own_w[kMaxHeadDim];      // ... and weights q*scale
+    __shared__ double bias_part[kSelThreads / 32];
+    __shared__ float bias_s;
     ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
     uint32_t *vals = th_dyn + 2 * kStageRows * kThetaCols;
     const int gq = blockIdx.x;
     const int si = find_session_by_query(b, gq);
     const SessionDesc &S = b.s[si];
     const int qq = gq - S.q_begin;
+    const int G = b.G, d = b.d;
+    const int h = qq / G, g = qq - h * G;
     uint32_t *st = S.qstate + qq * kQueryStateWords;
+    if (!force_exact && g == 0) {   // this KV head's tables for the filtering pass
+        setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)h * G * d, S.q + (size_t)h * G * d,
+                       S.mn + h * d, S.scale + h * d);
+        constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
+        const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
+        uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
+        for (int i = threadIdx.x; i < kUnits; i += blockDim.x) dst[i] = src[i];
+    }
     if (force_exact || S.exact_only) {
         if (threadIdx.x == 0) { st[0] = 0xFFFFFFFFu; st[1] = 0; st[2] = 1; }
         return;
@@ -1024,23 +1022,39 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
         if (threadIdx.x == 0) { st[0] = 0; st[1] = 0; st[2] = 0; }
         return;
     }
-    const int G = b.G;
-    const int h = qq / G, g = qq - h * G;
-    load_head<GP>(sm, S.tables, h);
-    if (threadIdx.x < 32) {   // the query's channels, in union order
-        const int lane = threadIdx.x;
-        int n = 0;
-        for (int u0 = 0; u0 < sm.U; u0 += 32) {
-            const int u = u0 + lane;
-            const bool mine = u < sm.U && sm.tq[u][g] > 0;
-            const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
-            if (mine) own[n + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)u;
-            n += __popc(bal);
+    // the query's own plan: channel c on thread c, depth clamped to the union
+    {
+        const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+        int tq = 0;
+        float w = 0.0f;
+        double term = 0.0;
+        if (c < d) {
+            const int T = min((int)S.tu[h * d + c], kBits);
+            tq = min((int)S.t[(size_t)qq * d + c], T);
+            const float qf = bf16_to_float(S.q[(size_t)qq * d + c]);
+            const float sc = S.scale[h * d + c];
+            w = __fmul_rn(qf, sc);
+            term = (double)qf * ((double)S.mn[h * d + c] + (double)sc * bin_offset(tq));
         }
-        if (lane == 0) n_own_s = n;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
+        if (lane == 0) bias_part[warp] = term;
+        unsigned n_own;
+        const unsigned pos = block_exclusive_scan(tq > 0 ? 1u : 0u, ss.wsum, &n_own);
+        if (tq > 0) {
+            own_c[pos] = (uint16_t)c;
+            own_t[pos] = (uint8_t)tq;
+            own_w[pos] = w;
+        }
+        if (threadIdx.x == 0) {
+            double acc = 0.0;
+            for (int w2 = 0; w2 < kSelThreads / 32; ++w2) acc += bias_part[w2];
+            bias_s = (float)acc;
+            ss.krem = n_own;   // parked until the barrier below
+        }
+        __syncthreads();
     }
-    __syncthreads();
-    const int n_own = n_own_s;
+    const int n_own = (int)ss.krem;
     const int n_stages = (n_own + kStageChannels - 1) / kStageChannels;
     const int sub = threadIdx.x / kScanThreads;             // tile of the pass
     const int lt = threadIdx.x - sub * kScanThreads;
@@ -1050,22 +1064,23 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     for (int p = 0; p < 4; ++p) sh[p] = (uint32_t)(r - p) & 31u;
     float neg[4];
     magic_negatives(neg);
-    const float bias = sm.bias[g];
-    // copy stage s of tile pass t0 into buffer bufi: rows of own channels
-    // 8s..8s+7 (4 slots each), 2 tiles x 16 column groups per row
+    const float bias = bias_s;
+    const size_t head_row0 = (size_t)h * d * kBits;
+    // copy stage s of tile pass t0 into buffer bufi: plane rows of own
+    // channels 8s..8s+7 (4 slots each, zeros past the channel's depth),
+    // 2 tiles x 16 column groups per row
     auto load = [&](int t0, int s, int bufi) {
         for (int e = threadIdx.x; e < kStageRows * (kThetaCols / 4); e += kSelThreads) {
             const int row = e / (kThetaCols / 4), part = e - row * (kThetaCols / 4);
             const int tsub = part / (kTileCols / 4), c16 = part - tsub * (kTileCols / 4);
             const int tile = t0 + tsub;
-            const int j = s * kStageChannels + row / kBits;
+            const int j = s * kStageChannels + row / kBits, slot = row % kBits;
             const int wcol = tile * S.sample_stride * kTileCols + c16 * 4;
-            uint32_t grow = 0xFFFFFFFFu;
-            if (j < n_own && tile < S.m_tiles && wcol < S.n_cols)
-                grow = sm.row_g[(int)own[j] * kBits + (row % kBits)];
-            copy_or_zero16(&stage[bufi][row][part * 4],
-                           S.planes + (size_t)grow * (size_t)S.n_words + wcol,
-                           grow != 0xFFFFFFFFu);
+            const bool live = j < n_own && slot < own_t[min(j, kMaxHeadDim - 1)] &&
+                              tile < S.m_tiles && wcol < S.n_cols;
+            const size_t grow = live ? head_row0 + (size_t)own_c[j] * kBits + slot : 0;
+            copy_or_zero16(&stage[bufi][row][part * 4], S.planes + grow * (size_t)S.n_words + wcol,
+                           live);
         }
         cp_async_commit();
     };
@@ -1086,16 +1101,12 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
             const uint32_t(*rows)[kThetaCols] = stage[s2 & 1];
             const int j1 = min(n_own, (s2 + 1) * kStageChannels);
             for (int j = s2 * kStageChannels; j < j1; ++j) {
-                const int u = own[j];
-                const int tg = sm.tq[u][g];
-                const uint32_t keep = ((0xFu << (kBits - tg)) & 0xFu) * 0x11111111u;
                 const uint32_t nib =
                     gather_nibbles<kThetaCols>(rows + kBits * (j - s2 * kStageChannels),
-                                               sub * kTileCols + col, sh) & keep;
+                                               sub * kTileCols + col, sh);
                 float2 v[4];
-                nibbles_to_floats(nib, neg, v);
-                const float w = sm.Wp[u][g];
-                const float2 w2 = make_float2(w, w);
+                nibbles_to_floats(nib, neg, v);   // rows past the depth are zero
+                const float2 w2 = make_float2(own_w[j], own_w[j]);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = __ffma2_rn(v[i], w2, acc[i]);
             }
@@ -1122,7 +1133,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     sel_range(ss, lo, hi);
     const uint32_t base = ss.lo;
     const int top = 32 + bit_length(ss.hi - base);
-    sel_run(ss, (unsigned)m, (unsigned)S.sample_rank, top, 32,
+    sel_run(ss, (unsigned)m, (unsigned)S.sample_rank, top, max(32, top - kThetaResolutionBits),
             [&](unsigned i) { return (unsigned long long)(vals[i] - base) << 32; });
     if (threadIdx.x == 0) {
         st[0] = base + (uint32_t)(ss.prefix >> 32);
@@ -1416,8 +1427,9 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 }
 
 template <int NS, int GP>
-cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int total_heads, int max_m_keys, const FetchJob *fetch,
-                      int n_fetch, uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
+cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int max_m_keys,
+                      const FetchJob *fetch, int n_fetch, uint32_t flags, cudaStream_t stream,
+                      ScanProfileHook *hook)
 {
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
@@ -1431,13 +1443,9 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, 
             hook->recorded = true;
         }
     }
-    if (!force && total_groups > 0) {
-        prep_kernel<NS, GP><<<total_heads, kScanThreads, 0, stream>>>(bt);
-        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "prep launch");
-        ++launches;
-    }
     {
-        // sampled scores and theta per query (or the exact-path flags)
+        // per-head tables, sampled scores and theta per query (or the
+        // exact-path flags)
         static int threshold_smem_set[64];
         auto kern = threshold_kernel<NS, GP>;
         const size_t dyn = 2 * kThetaStageBytes + (size_t)max_m_keys * sizeof(uint32_t);
@@ -1501,7 +1509,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
+    int groups = 0, queries = 0, max_m = 0, n_fetch = 0;
     FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
@@ -1540,20 +1548,18 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.exact_only = z.exact_only;
         D.group_begin = groups;
         D.q_begin = queries;
-        D.head_begin = heads;
-        heads += ix.n_kv_heads;
         groups += D.H * D.col_groups;
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    return run_batch<NS, 8>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
+    return run_batch<NS, 8>(bt, groups, queries, max_m, fetch, n_fetch, flags,
                                            stream, hook);
 }
 
