@@ -2,7 +2,8 @@
 """Benchmark of the Fathom per-query read-depth top-k key scan on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
-                    [--workload qwen3_8b_layer_128k|host_1m|fixed_vs_wf_1m|agent_16_sessions]
+                    [--workload qwen3_8b_layer_128k|host_1m|host_256k|fixed_vs_wf_1m|
+                               agent_16_sessions]
 
 A step is one decode-step scan of a whole layer through the hot path, once
 per plan of the workload: plan (reverse water-filling at B bits per key, or
@@ -53,6 +54,10 @@ WORKLOADS = {
                                 plans=(("wf", 68), ("wf", 92), ("wf", 136))),
     "host_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                     plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
+    # the host path at a quarter of the keys: the profiling case of the fetch
+    # kernel (its traffic scales with n)
+    "host_256k": dict(H=8, G=4, n=1 << 18, d=128, k=2048, residency="host_mapped",
+                      plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
     "fixed_vs_wf_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                            plans=(("fixed", 34), ("fixed", 17), ("wf", 68), ("wf", 92)),
                            device_keys=True),
@@ -271,6 +276,39 @@ def run_reference(args, wl_name, wl):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ traffic
+def recorded_traffic(wl_name, wl, kernel):
+    """Measured traffic per launch of the dominant kernel, from the ncu
+    capture recorded in profiles/traffic.json: DRAM read+write bytes for the
+    HBM scan, host-memory read bytes (sysmem sectors x 32 B) for the fetch.
+    None unless the kernel's source is unchanged since the capture (sha256)
+    and the capture covers this workload's plans; host workloads of other
+    sizes scale the capture by their key count (the union planes are
+    proportional to it)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None, "kernel changed since the recorded capture"
+    except (OSError, KeyError, ValueError):
+        return None, "no recorded capture"
+    plans = [plan_name(p) for p in (wl.get("plans") or ())]
+    if plans != rec["plans"]:
+        return None, "no capture of these plans"
+    if kernel == "scan_kernel":
+        if wl_name != rec["workload"]:
+            return None, "no capture of this workload"
+        vals = rec["dram_bytes_per_launch"]
+        note = f"ncu dram__bytes_read+write, {rec['workload']}, mean over plans"
+    else:
+        vals = [v * wl["n"] / rec["n_keys"] for v in rec["host_link_read_bytes_per_launch"]]
+        note = (f"ncu host-memory read sectors x 32 B, {rec['workload']} scaled to "
+                f"{wl['n']} keys, mean over plans")
+    return sum(vals) / len(vals), note
+
+
 # ------------------------------------------------------------ ranks
 def max_over_ranks(dist, values, device):
     """Each value's maximum over the ranks (the slowest rank's device-timed
@@ -391,8 +429,9 @@ def run_fathom(args, wl_name, wl):
     status = fp.fathom_last_device_status()
     assert status == fp.FATHOM_OK, fp.status_str(status)
 
-    ev = [(torch.cuda.Event(enable_timing=True, external=True),
-           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K)]
+    # external records keep the events timing points inside a captured graph
+    ev = [(torch.cuda.Event(enable_timing=True, external=bool(args.graph)),
+           torch.cuda.Event(enable_timing=True, external=bool(args.graph))) for _ in range(K)]
 
     def timed_steps():
         for s in range(K):
@@ -504,8 +543,10 @@ def run_fathom(args, wl_name, wl):
         peak = max(link["h2d_memcpy_gbs"], link["zero_copy_read_gbs"])
         bound, peak_note = "host_link", "measured in this run: max(pinned copy, zero-copy read)"
         kernel = "fetch_kernel (union planes, host -> device mirror)"
+    traffic, traffic_note = recorded_traffic(wl_name, wl, "fetch_kernel" if link else "scan_kernel")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "kernel": kernel,
+                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_note,
+                "kernel": kernel,
                 "peak_source": peak_note, "avg_launch_us": avg_launch_ms * 1e3,
                 "algorithmic_bytes_per_launch": bytes_per_launch}
 
