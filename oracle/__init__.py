@@ -47,6 +47,7 @@ def _load():
             "fo_quantize": ([P, I, I, I, P, P, P], ctypes.c_int),
             "fo_pack_planes": ([P, I, I, I, I, P], ctypes.c_int),
             "fo_unpack_planes": ([P, I, I, I, I, P], ctypes.c_int),
+            "fo_append": ([P, I, I, I, I, I, P, P, P, P, P, P, P], ctypes.c_int),
             "fo_channel_stats": ([P, I, I, I, P, P, P, P], ctypes.c_int),
             "fo_importance": ([P, P, I, P], ctypes.c_int),
             "fo_plan_greedy": ([P, I, I, P], ctypes.c_int),
@@ -110,6 +111,27 @@ def unpack_planes(planes: np.ndarray, n: int) -> np.ndarray:
     codes = np.empty((H, d, n), np.uint8)
     _check(_load().fo_unpack_planes(_p(planes), H, n, d, n_words, _p(codes)), "unpack_planes")
     return codes
+
+
+def append(index: Dict[str, np.ndarray], keys: np.ndarray, clamped=None):
+    """Append keys float32 [H][m][d] to an index dict (build_index's layout)
+    in place: planes, s1, s2, sigma2, codes and n are updated; clamped
+    (uint32 [H][d], optional) is incremented.  Returns the new key count."""
+    keys = np.ascontiguousarray(keys, dtype=np.float32)
+    H, m, d = keys.shape
+    n = index["n"]
+    n_words = index["planes"].shape[-1]
+    for name in ("planes", "s1", "s2", "sigma2"):
+        assert index[name].flags["C_CONTIGUOUS"]
+    if clamped is not None:
+        assert clamped.dtype == np.uint32 and clamped.flags["C_CONTIGUOUS"]
+    _check(_load().fo_append(_p(keys), H, n, m, d, n_words, _p(index["mn"]), _p(index["scale"]),
+                             _p(index["planes"]), _p(index["s1"]), _p(index["s2"]),
+                             _p(index["sigma2"]), None if clamped is None else _p(clamped)),
+           "append")
+    index["n"] = n + m
+    index["codes"] = unpack_planes(index["planes"], n + m)
+    return n + m
 
 
 def channel_stats(codes: np.ndarray, scale: np.ndarray):
@@ -224,11 +246,12 @@ def recall(selected, reference) -> float:
 
 
 # --------------------------------------------------------------- whole pipeline
-def build_index(keys: np.ndarray) -> Dict[str, np.ndarray]:
-    """Storage side for one session: quantise, pack, channel statistics."""
+def build_index(keys: np.ndarray, capacity: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Storage side for one session: quantise, pack, channel statistics.
+    capacity: keys the planes can hold (for appends); default n."""
     mn, scale, codes = quantize(keys)
     n = keys.shape[1]
-    planes = pack_planes(codes)
+    planes = pack_planes(codes, n_words_for(max(n, capacity or n)))
     s1, s2, sigma2 = channel_stats(codes, scale)
     return dict(mn=mn, scale=scale, codes=codes, planes=planes, s1=s1, s2=s2,
                 sigma2=sigma2, n=n, n_words=planes.shape[-1])

@@ -112,6 +112,61 @@ int fo_pack_planes(const uint8_t *codes, int64_t H, int64_t n, int64_t d,
     return FO_OK;
 }
 
+/* Append m keys per KV head to an index holding n keys: the decode step's
+ * new keys enter the 4-bit K cache the explainer's read side scans
+ * (核心方法 / 存储侧; the cache comes from the serving stack, 适用边界).
+ * Reading: the new keys are quantised with the index's existing mn and
+ * scale, in the quantiser's own float32 steps, and the level is clamped to
+ * 0..15 (a key outside the stored range takes the nearest level); their
+ * bits go to key positions n..n+m-1 of the planes; S1 and S2 grow by the
+ * new codes and sigma^2 is recomputed from them with n+m keys.
+ * clamped[h][c] (may be NULL) is incremented once per new key whose level
+ * fell outside 0..15 (for a constant channel: any key other than mn), the
+ * measure of range drift a caller re-quantises on.
+ * keys float32 [H][m][d]; planes [H][d][4][n_words], 32*n_words >= n+m,
+ * words past key n zero. */
+int fo_append(const float *keys, int64_t H, int64_t n, int64_t m, int64_t d, int64_t n_words,
+              const float *mn, const float *scale, uint32_t *planes, int64_t *s1, int64_t *s2,
+              float *sigma2, uint32_t *clamped)
+{
+    if (H <= 0 || n < 0 || m <= 0 || d <= 0 || n_words * 32 < n + m) return FO_ERR_ARG;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t c = 0; c < d; ++c) {
+            const int64_t hc = h * d + c;
+            const float lo = mn[hc], sc = scale[hc];
+            uint32_t *pc = planes + hc * FO_BITS * n_words;
+            for (int64_t i = 0; i < m; ++i) {
+                const float x = keys[(h * m + i) * d + c];
+                if (!isfinite(x)) return FO_ERR_NONFINITE;
+                int v;
+                int out_of_range;
+                if (sc == 0.0f) {
+                    v = 0;
+                    out_of_range = x != lo;
+                } else {
+                    float diff = x - lo;
+                    float ratio = diff / sc;
+                    float shifted = ratio + 0.5f;
+                    float level = floorf(shifted);
+                    out_of_range = level < 0.0f || level > (float)FO_LEVELS;
+                    v = level < 0.0f ? 0 : (level > (float)FO_LEVELS ? FO_LEVELS : (int)level);
+                }
+                const int64_t j = n + i;
+                for (int p = 0; p < FO_BITS; ++p)
+                    if ((v >> p) & 1)
+                        pc[(FO_BITS - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
+                s1[hc] += v;
+                s2[hc] += (int64_t)v * v;
+                if (clamped && out_of_range) clamped[hc] += 1;
+            }
+            const int64_t nn = n + m;
+            const int64_t num = nn * s2[hc] - s1[hc] * s1[hc];
+            const double sd = (double)sc;
+            sigma2[hc] = (float)((sd * sd) * ((double)num / ((double)nn * (double)nn)));
+        }
+    return FO_OK;
+}
+
 /* Inverse of fo_pack_planes (reads all four slots). */
 int fo_unpack_planes(const uint32_t *planes, int64_t H, int64_t n, int64_t d,
                      int64_t n_words, uint8_t *codes)

@@ -26,6 +26,12 @@ MUTATIONS = {
     "topk_ties_to_higher_index": ("return (a->j < b->j) ? -1 : (a->j > b->j);",
                                   "return (a->j > b->j) ? -1 : (a->j < b->j);"),
     "union_takes_min": ("if (t[g * d + c] > m) m = t[g * d + c];", "if (g == 0) m = t[g * d + c];"),
+    "append_lsb_first": ("if ((v >> p) & 1)\n                        pc[(FO_BITS - 1 - p) * n_words",
+                         "if ((v >> p) & 1)\n                        pc[p * n_words"),
+    "append_ignores_min": ("float diff = x - lo;", "float diff = x;"),
+    "append_variance_old_count": ("const int64_t nn = n + m;", "const int64_t nn = n;"),
+    "append_no_high_clamp_count": ("out_of_range = level < 0.0f || level > (float)FO_LEVELS;",
+                                   "out_of_range = level < 0.0f;"),
 }
 
 PIN_TESTS = [
@@ -40,6 +46,9 @@ PIN_TESTS = [
     lambda: pins.test_coarse_bin_midpoint_hand_worked(read_golden),
     pins.test_reading_t_planes_equals_requantising_to_t_bits,
     lambda: pins.test_topk_hand_worked(read_golden),
+    lambda: pins.test_append_in_range_equals_repacking_everything(127, 129),
+    pins.test_append_clamps_out_of_range_keys_to_the_end_levels,
+    pins.test_append_keeps_sigma2_the_variance_of_the_stored_keys,
 ]
 
 

@@ -337,3 +337,75 @@ def test_tiny_workload_planted_keys_rank_high():
     t, T, nb = oracle.plan_session(ix, ses.q_bf16, ses.budgets, 1)
     idx, _, _ = oracle.scan_query(ix, ses.q_bf16[0], t[0], 0, 64)
     assert len(set(ses.planted[0].tolist()) & set(idx.tolist())) >= 12
+
+
+# ------------------------------------------------------------------ append
+def _split_in_range(seed, H, n, m, d):
+    """n keys to pack, then m new keys clipped into the packed keys' range."""
+    ses = synth.make_session(seed, H, 1, n + m, 64, head_dim=d)
+    first = ses.keys[:, :n]
+    lo = first.min(axis=1, keepdims=True)
+    hi = first.max(axis=1, keepdims=True)
+    return first, np.clip(ses.keys[:, n:], lo, hi).astype(np.float32)
+
+
+@pytest.mark.parametrize("n,m", [(900, 100), (31, 2), (32, 1), (127, 129), (4096, 1)])
+def test_append_in_range_equals_repacking_everything(n, m):
+    """Keys inside the stored range leave min and max, so scale and every
+    code are unchanged: appending must give exactly the index of all n+m."""
+    first, new = _split_in_range(n + m, 2, n, m, 32)
+    ix = oracle.build_index(first, capacity=n + m)
+    clamped = np.zeros((2, 32), np.uint32)
+    assert oracle.append(ix, new, clamped) == n + m
+    full = oracle.build_index(np.concatenate([first, new], axis=1))
+    for name in ("planes", "s1", "s2", "sigma2", "mn", "scale"):
+        assert np.array_equal(ix[name], full[name]), name
+    assert clamped.sum() == 0
+
+
+def test_append_one_by_one_equals_one_batch():
+    first, new = _split_in_range(7, 1, 500, 70, 16)
+    a = oracle.build_index(first, capacity=570)
+    b = oracle.build_index(first, capacity=570)
+    oracle.append(a, new)
+    for i in range(70):
+        oracle.append(b, new[:, i:i + 1])
+    for name in ("planes", "s1", "s2", "sigma2"):
+        assert np.array_equal(a[name], b[name]), name
+
+
+def test_append_clamps_out_of_range_keys_to_the_end_levels():
+    keys = np.zeros((1, 16, 2), np.float32)
+    keys[0, :, 0] = np.arange(16)          # channel 0: 0..15, scale 1
+    keys[0, :, 1] = 3.0                    # channel 1: constant, scale 0
+    ix = oracle.build_index(keys, capacity=128)
+    assert ix["scale"][0, 0] == 1.0 and ix["scale"][0, 1] == 0.0
+    new = np.array([[[-10.0, 3.0], [0.0, 4.0], [15.0, 3.0], [40.0, -1.0], [7.4, 3.0]]],
+                   np.float32)
+    clamped = np.zeros((1, 2), np.uint32)
+    oracle.append(ix, new, clamped)
+    codes = ix["codes"][0]
+    assert list(codes[0, 16:]) == [0, 0, 15, 15, 7]
+    assert list(codes[1, 16:]) == [0, 0, 0, 0, 0]
+    assert list(clamped[0]) == [2, 2]      # -10 and 40; the two values != 3
+
+
+def test_append_keeps_sigma2_the_variance_of_the_stored_keys():
+    ses = synth.make_session(9, 2, 1, 3000, 64, head_dim=16)
+    ix = oracle.build_index(ses.keys[:, :2000], capacity=3000)
+    oracle.append(ix, ses.keys[:, 2000:] * 1.3)        # partly out of range
+    deq = ix["mn"][:, :, None].astype(np.float64) + \
+        ix["scale"][:, :, None].astype(np.float64) * ix["codes"].astype(np.float64)
+    np.testing.assert_allclose(ix["sigma2"], deq.var(axis=2), rtol=1e-5)
+    assert np.array_equal(ix["s1"], ix["codes"].astype(np.int64).sum(axis=2))
+
+
+def test_append_rejects_overflow_and_nonfinite():
+    ses = synth.make_session(3, 1, 1, 200, 64, head_dim=8)
+    ix = oracle.build_index(ses.keys[:, :100])              # capacity 128
+    with pytest.raises(ValueError):
+        oracle.append(ix, ses.keys[:, 100:130])
+    bad = ses.keys[:, 100:101].copy()
+    bad[0, 0, 3] = np.inf
+    with pytest.raises(ValueError):
+        oracle.append(ix, bad)
