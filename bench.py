@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
                     [--workload qwen3_8b_layer_128k|host_1m|host_256k|fixed_vs_wf_1m|
-                               agent_16_sessions]
+                               agent_16_sessions|append_layer_128k]
 
 A step is one decode-step scan of a whole layer through the hot path, once
 per plan of the workload: plan (reverse water-filling at B bits per key, or
@@ -61,6 +61,10 @@ WORKLOADS = {
     "fixed_vs_wf_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                            plans=(("fixed", 34), ("fixed", 17), ("wf", 68), ("wf", 92)),
                            device_keys=True),
+    # the append path: decode-step keys (m = 1 per KV head) and a bulk chunk
+    # into a packed Qwen3-8B-shaped layer
+    "append_layer_128k": dict(H=8, G=4, n=131072, d=128, k=0, residency="device",
+                              append=(1, 8192), plans=None),
     "agent_16_sessions": dict(H=8, G=4, n=None, d=128, k=1024, residency="host_mapped",
                               sessions=16, plans=None, device_keys=True, batched=True),
 }
@@ -582,9 +586,88 @@ def run_fathom(args, wl_name, wl):
         dist.destroy_process_group()
 
 
+def run_append(args, wl_name, wl):
+    """Append path: K timed appends of m keys per KV head for each m of the
+    workload (after W warm-up appends), each timed with CUDA events; the
+    index is packed with room for all of them.  Roofline: the append reads
+    its keys (H*m*d*4 bytes) and read-modify-writes the touched plane words
+    (2 * H*d*4 slots * words * 4 bytes), against measured HBM."""
+    import torch
+    import decode_fathom_plan_b200 as fp
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    fp.load_library()
+    H, G, n, d = wl["H"], wl["G"], wl["n"], wl["d"]
+    W, K = max(3, args.warmup), args.steps
+    results = []
+    for m in wl["append"]:
+        total = n + (W + K) * m
+        sigma, _ = synth.channel_sigma(rank, H, d)
+        keys = synth.device_keys(torch, sigma, total, rank)
+        index = fp.KeyIndex(H, G, n, d, wl["residency"], capacity=total)
+        index.pack(keys[:, :n].contiguous())
+        chunks = [keys[:, n + i * m:n + (i + 1) * m].contiguous() for i in range(W + K)]
+        clamped = torch.zeros((H, d), dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        for i in range(W):
+            index.append(chunks[i], clamped)
+        # the K timed appends as one CUDA graph (each append's key count is
+        # fixed at capture; replaying once performs each exactly once), so the
+        # events time the device, not the host's launch path
+        ev = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+                for i in range(K):
+                    ev[i][0].record()
+                    index.append(chunks[W + i], clamped)
+                    ev[i][1].record()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        del graph
+        assert fp.fathom_last_device_status() == fp.FATHOM_OK
+        ms = [a.elapsed_time(b) for a, b in ev]
+        med = statistics.median(ms)
+        words = m // 32 + 2
+        nbytes = H * m * d * 4 + 2 * H * d * 4 * words * 4
+        results.append({"m": m, "us_per_append_median": med * 1e3,
+                        "keys_per_s": H * m / (med / 1e3),
+                        "bytes_per_append": nbytes,
+                        "achieved_gbs": nbytes / (med / 1e3) / 1e9,
+                        "clamped_keys_total": int(clamped.sum().item())})
+        del keys, index, chunks
+    peak, peak_src = load_peaks()
+    bulk = results[-1]
+    line = {"metric": "KV-head keys appended per second (append path)",
+            "value": bulk["keys_per_s"] / 1e9, "unit": "Gkeys/s", "n_gpus": 1, "steps": K,
+            "warmup": W, "ms_per_step": bulk["us_per_append_median"] / 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": wl_name, "kv_heads": H, "head_dim": d,
+                                            "n_keys_packed": n, "appends": list(wl["append"])},
+            "roofline": {"bound": "hbm", "achieved": bulk["achieved_gbs"], "peak": peak,
+                         "unit": "GB/s", "frac": bulk["achieved_gbs"] / peak, "traffic": None,
+                         "kernel": f"append_kernel (m = {bulk['m']})",
+                         "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},
+            "per_m": results, "launch_mode": "cuda_graph"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     wl = WORKLOADS[args.workload]
+    if wl.get("append"):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the append workload has no CPU reference leg"}))
+        else:
+            run_append(args, args.workload, wl)
+        return
     if args.impl == "reference":
         run_reference(args, args.workload, wl)
     else:

@@ -37,7 +37,7 @@ EXPORTED = (
     "fathom_plan", "fathom_fixed_plan", "fathom_scan_workspace_bytes", "fathom_scan_topk",
     "fathom_scan_batched_workspace_bytes", "fathom_scan_topk_batched",
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
-    "fathom_scan_topk_static", "fathom_link_probe",
+    "fathom_scan_topk_static", "fathom_link_probe", "fathom_append_keys",
 )
 
 
@@ -78,6 +78,7 @@ def load_library(path: str = LIB_PATH):
         "fathom_status_str": ([ctypes.c_int], ctypes.c_char_p),
         "fathom_pack_workspace_bytes": ([IX], SZ),
         "fathom_pack_keys": ([P, IX, P, SZ, P], ctypes.c_int),
+        "fathom_append_keys": ([IX, P, I32, P, P], ctypes.c_int),
         "fathom_plan": ([IX, P, P, P, P, P, P], ctypes.c_int),
         "fathom_fixed_plan": ([IX, P, I32, P, P, P, P], ctypes.c_int),
         "fathom_scan_workspace_bytes": ([IX, I32], SZ),
@@ -143,6 +144,14 @@ def fathom_pack_keys(keys, index: fathom_index, workspace, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(load_library().fathom_pack_keys(_ptr(keys), ctypes.byref(index), _ptr(workspace),
                                            ws_bytes, _stream(stream)), "fathom_pack_keys")
+
+
+def fathom_append_keys(keys, index: fathom_index, m: int, clamped=None, stream=None):
+    """Append m keys (device float32 [H][m][d]) to the index; index.n_keys
+    grows by m.  clamped: optional device uint32 [H][d] drift counters."""
+    _check(load_library().fathom_append_keys(ctypes.byref(index), _ptr(keys), int(m),
+                                             None if clamped is None else _ptr(clamped),
+                                             _stream(stream)), "fathom_append_keys")
 
 
 def fathom_plan(index: fathom_index, q_bf16, budget, t, t_union, nbytes, stream=None):
@@ -238,10 +247,11 @@ class KeyIndex:
     device either way."""
 
     def __init__(self, n_kv_heads: int, group: int, n_keys: int, head_dim: int = 128,
-                 residency: str = "device", device: Optional[int] = None):
+                 residency: str = "device", device: Optional[int] = None,
+                 capacity: Optional[int] = None):
         import torch
         dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
-        self.n_words = fathom_n_words(n_keys)
+        self.n_words = fathom_n_words(max(n_keys, capacity or n_keys))
         H, d = n_kv_heads, head_dim
         shape = (H, d, 4, self.n_words)
         if residency == "device":
@@ -279,6 +289,16 @@ class KeyIndex:
     @property
     def n_keys(self):
         return self.desc.n_keys
+
+    @property
+    def capacity(self):
+        return 32 * self.n_words
+
+    def append(self, keys, clamped=None, stream=None):
+        """Append device float32 keys [H][m][d] (decode-step keys) to this
+        index; clamped: optional device uint32 [H][d] drift counters."""
+        fathom_append_keys(keys, self.desc, keys.shape[1], clamped, stream)
+        return self
 
     def pack(self, keys, stream=None):
         """Quantise and pack device float32 keys [H][n][d] into this index."""

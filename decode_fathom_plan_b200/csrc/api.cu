@@ -204,6 +204,19 @@ fathom_status fathom_pack_keys(const float *keys, const fathom_index *index, voi
     return cuda_status(launch_pack(keys, ix, static_cast<uint32_t *>(workspace), stream));
 }
 
+fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t m,
+                                 uint32_t *clamped, cudaStream_t stream)
+{
+    if (!keys || !index_shape_ok(index) || !stats_ok(index) || m < 1) return FATHOM_ERR_INVALID_ARG;
+    if ((long long)index->n_keys + m > (long long)index->n_words * 32) return FATHOM_ERR_INVALID_ARG;
+    fathom_index ix = *index;
+    fathom_status st = resolve_planes(index, &ix.planes);
+    if (st != FATHOM_OK) return st;
+    st = cuda_status(launch_append(keys, ix, m, clamped, stream));
+    if (st == FATHOM_OK) index->n_keys += m;
+    return st;
+}
+
 fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
                           const int32_t *budget, uint8_t *t, uint8_t *t_union, uint64_t *bytes,
                           cudaStream_t stream)

@@ -1,0 +1,110 @@
+// Append path: the decode step's new keys into an existing 4-bit K index.
+//
+// Source: Fathom explainer (papers.ananclaw.com, arXiv 2609.17652),
+// section 核心方法 / 存储侧 (per-channel 4-bit quantisation stored as
+// MSB-first bit planes) and 适用边界 (the 4-bit K cache comes from the
+// serving stack, which grows it by one key per decode step).  A new key is
+// quantised with the index's stored min and scale in the quantiser's own
+// float32 steps, its level clamped to 0..15 (a key outside the stored
+// range takes the nearest level, and the clamp is counted per channel as
+// the measure of range drift), its bits are ORed into the zero padding
+// words past the last key, the exact sums S1, S2 grow, and sigma^2 is
+// recomputed for the new key count (by the appending thread itself when
+// all new keys fall in one plane word, the decode step's case).
+//
+// One thread per (KV head, plane word, channel), channel fastest: it owns
+// the up-to-32 new keys of that word for that channel, so every plane word
+// has a single writer and the key loads of a warp are contiguous channels.
+#include "common.cuh"
+#include "internal.h"
+
+namespace fathom {
+namespace {
+
+__global__ void __launch_bounds__(256)
+append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_words,
+              const float *__restrict__ mn, const float *__restrict__ scale, uint32_t *planes,
+              int64_t *s1, int64_t *s2, float *sigma2, uint32_t *clamped, int *status)
+{
+    const int w_first = n >> 5;
+    const int words = ((n + m - 1) >> 5) - w_first + 1;
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (tid >= (long long)H * words * d) return;
+    const int c = (int)(tid % d);
+    const long long rest = tid / d;
+    const int wi = (int)(rest % words), h = (int)(rest / words);
+    const int w = w_first + wi;
+    const int j_lo = max(n, w * 32), j_hi = min(n + m, w * 32 + 32);
+    const int hc = h * d + c;
+    const float lo = mn[hc], sc = scale[hc];
+    uint32_t slot[kBits] = {0u, 0u, 0u, 0u};
+    unsigned long long a1 = 0, a2 = 0;
+    unsigned n_clamped = 0;
+    bool bad = false;
+    auto take = [&](int j, float x) {
+        int v = 0;
+        if (!isfinite(x)) {
+            bad = true;
+        } else if (sc == 0.0f) {
+            n_clamped += (x != lo);
+        } else {
+            const float level = floorf(__fadd_rn(__fdiv_rn(__fsub_rn(x, lo), sc), 0.5f));
+            const bool out = level < 0.0f || level > 15.0f;
+            n_clamped += out;
+            v = level < 0.0f ? 0 : (level > 15.0f ? 15 : static_cast<int>(level));
+        }
+#pragma unroll
+        for (int s = 0; s < kBits; ++s)   // slot s holds bit 3-s
+            slot[s] |= (uint32_t)((v >> (kBits - 1 - s)) & 1) << (j & 31);
+        a1 += (unsigned long long)v;
+        a2 += (unsigned long long)(v * v);
+    };
+    const float *kc = keys + (size_t)h * m * d + c;   // key j at kc[(j - n) * d]
+    if (j_hi - j_lo == 32) {
+        // a whole word: 8 independent loads in flight per round
+#pragma unroll
+        for (int j0 = 0; j0 < 32; j0 += 8) {
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = kc[(size_t)(j_lo + j0 + i - n) * d];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) take(j_lo + j0 + i, x[i]);
+        }
+    } else {
+        for (int j = j_lo; j < j_hi; ++j) take(j, kc[(size_t)(j - n) * d]);
+    }
+    uint32_t *pw = planes + (size_t)hc * kBits * n_words + w;
+#pragma unroll
+    for (int s = 0; s < kBits; ++s)
+        if (slot[s]) pw[(size_t)s * n_words] |= slot[s];
+    const unsigned long long o1 = atomicAdd(reinterpret_cast<unsigned long long *>(&s1[hc]), a1);
+    const unsigned long long o2 = atomicAdd(reinterpret_cast<unsigned long long *>(&s2[hc]), a2);
+    // all new keys in one word: this thread is the channel's only writer and
+    // holds its final sums (several words: a second pass recomputes sigma^2)
+    if (words == 1)
+        sigma2[hc] = channel_sigma2((long long)(o1 + a1), (long long)(o2 + a2), sc, n + m);
+    if (clamped && n_clamped) atomicAdd(&clamped[hc], n_clamped);
+    if (bad) set_status(status, FATHOM_ERR_NONFINITE);
+}
+
+}  // namespace
+
+cudaError_t launch_append(const float *keys, const fathom_index &ix, int m, uint32_t *clamped,
+                          cudaStream_t stream)
+{
+    const int H = ix.n_kv_heads, d = ix.head_dim, n = ix.n_keys;
+    const int words = ((n + m - 1) >> 5) - (n >> 5) + 1;
+    const long long threads = (long long)H * words * d;
+    const int block = 256;
+    const long long grid = (threads + block - 1) / block;
+    append_kernel<<<(unsigned)grid, block, 0, stream>>>(keys, H, n, m, d, ix.n_words, ix.mn,
+                                                        ix.scale, ix.planes, ix.sum_code,
+                                                        ix.sum_code2, ix.sigma2, clamped,
+                                                        device_status_ptr());
+    note_launch(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || words == 1) return e;
+    return launch_channel_stats(ix, n + m, stream);
+}
+
+}  // namespace fathom

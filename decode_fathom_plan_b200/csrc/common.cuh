@@ -68,4 +68,16 @@ __device__ __forceinline__ unsigned long long composite(uint32_t okey, uint32_t 
     return (static_cast<unsigned long long>(okey) << 32) | static_cast<unsigned long long>(~j);
 }
 
+// Variance of the stored 4-bit keys of a channel from its exact sums:
+// scale^2 * (n*S2 - S1^2) / n^2 in fp64, rounded once to float32 (the
+// importance weight of the read side).
+__device__ __forceinline__ float channel_sigma2(long long s1, long long s2, float scale, long long n)
+{
+    const long long num = n * s2 - s1 * s1;
+    const double sc = (double)scale;
+    const double sc2 = __dmul_rn(sc, sc);
+    const double frac = __ddiv_rn((double)num, __dmul_rn((double)n, (double)n));
+    return __double2float_rn(__dmul_rn(sc2, frac));
+}
+
 }  // namespace fathom

@@ -20,6 +20,14 @@ cudaError_t note_error(cudaError_t e, const char *site);
 // ---- pack.cu
 cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_minmax,
                         cudaStream_t stream);
+// sigma^2 of every (head, channel) from its exact sums and the key count n.
+cudaError_t launch_channel_stats(const fathom_index &ix, int n, cudaStream_t stream);
+
+// ---- append.cu
+// Appends m keys (device float32 [H][m][d]) at positions ix.n_keys.. and
+// recomputes sigma^2 for ix.n_keys + m keys; clamped may be null.
+cudaError_t launch_append(const float *keys, const fathom_index &ix, int m, uint32_t *clamped,
+                          cudaStream_t stream);
 
 // ---- plan.cu
 cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t *budget,

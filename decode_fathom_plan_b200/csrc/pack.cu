@@ -152,12 +152,7 @@ __global__ void pack_stats_kernel(const int64_t *s1, const int64_t *s2, const fl
 {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= count) return;
-    const long long nn = n;
-    const long long num = nn * s2[i] - s1[i] * s1[i];
-    const double sc = (double)scale[i];
-    const double sc2 = __dmul_rn(sc, sc);
-    const double frac = __ddiv_rn((double)num, __dmul_rn((double)nn, (double)nn));
-    sigma2[i] = __double2float_rn(__dmul_rn(sc2, frac));
+    sigma2[i] = channel_sigma2(s1[i], s2[i], scale[i], n);
 }
 
 }  // namespace
@@ -182,9 +177,18 @@ cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_
     dim3 g2((n_words + kQuantWordsPerBlock - 1) / kQuantWordsPerBlock, H);
     pack_quant_kernel<<<g2, kQuantThreads, smem, stream>>>(keys, n, d, n_words, ix.mn, ix.scale,
                                                           ix.planes, ix.sum_code, ix.sum_code2);
+    note_launch(4);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_channel_stats(ix, n, stream);
+}
+
+cudaError_t launch_channel_stats(const fathom_index &ix, int n, cudaStream_t stream)
+{
+    const int count = ix.n_kv_heads * ix.head_dim;
+    const int eb = 256, eg = (count + eb - 1) / eb;
     pack_stats_kernel<<<eg, eb, 0, stream>>>(ix.sum_code, ix.sum_code2, ix.scale, ix.sigma2, n,
                                              count);
-    note_launch(5);
+    note_launch(1);
     return cudaGetLastError();
 }
 

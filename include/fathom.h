@@ -133,6 +133,28 @@ fathom_status fathom_pack_keys(const float *keys, const fathom_index *index,
                                void *workspace, size_t workspace_bytes,
                                cudaStream_t stream);
 
+/* Append m new keys per KV head at positions n..n+m-1 of an index holding
+ * n = index->n_keys keys: the decode step's keys entering the 4-bit K
+ * cache the read side scans (explainer, 核心方法 / 存储侧; the cache comes
+ * from the serving stack, 适用边界).  Each new key is quantised with the
+ * index's stored mn and scale exactly as fathom_pack_keys quantises, its
+ * level clamped to 0..15 (a key outside the stored range takes the nearest
+ * level; a constant channel stores code 0); its bits go to key positions
+ * n..n+m-1 of the planes; sum_code, sum_code2 grow by the new codes and
+ * sigma2 is recomputed for n+m keys.  Keys inside the stored range give
+ * exactly the index that packing all n+m keys would.
+ * keys: device float32 [H][m][d].  clamped: optional (may be NULL) device
+ * uint32 [H][d], incremented by the number of new keys whose level was
+ * clamped (for a constant channel: keys other than mn) -- the range-drift
+ * measure; re-pack with fathom_pack_keys when a channel's count passes the
+ * caller's tolerance.  Requires n + m <= 32*n_words, with the plane words
+ * past key n zero (as fathom_pack_keys and earlier appends leave them);
+ * planes may be a mapped host pointer.  On success index->n_keys grows by
+ * m (host field).  A non-finite key stores code 0 and sets
+ * FATHOM_ERR_NONFINITE in the device status. */
+fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t m,
+                                 uint32_t *clamped, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Read side: plans.                                                      */
 /* ---------------------------------------------------------------------- */

@@ -110,3 +110,16 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(fp, "_lib", None)
     with pytest.raises(ImportError):
         fp.load_library(str(tmp_path / "missing.so"))
+
+
+def test_append_rejects_bad_arguments_before_launching(lib):
+    ix = _desc(n=100)                       # capacity: 128 keys
+    fake = 0x1000
+    F = fp.FATHOM_ERR_INVALID_ARG
+    append = lib.fathom_append_keys
+    assert append(ctypes.byref(ix), None, 1, None, None) == F           # no keys
+    assert append(ctypes.byref(ix), fake, 0, None, None) == F           # m < 1
+    assert append(ctypes.byref(ix), fake, 29, None, None) == F          # past the capacity
+    bad = _desc(d=48)
+    assert append(ctypes.byref(bad), fake, 1, None, None) == F
+    assert ix.n_keys == 100                  # untouched on error
