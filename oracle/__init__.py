@@ -59,6 +59,7 @@ def _load():
             "fo_score_abs_planes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
             "fo_exact_scores": ([P, P, I, I, P], None),
             "fo_topk": ([P, I, I, P, P], ctypes.c_int),
+            "fo_attention": ([P, P, I, I, P, P, I, ctypes.c_double, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -282,3 +283,32 @@ def scan_query(index, q_bf16_row, t_row, h: int, k: int):
     s = score_planes(index["planes"][h], index["mn"][h], index["scale"][h], q_bf16_row, t_row, n)
     idx, top = topk(s, k)
     return idx, top, s
+
+
+# ------------------------------------------------------------------ after the scan
+def attention(keys_h: np.ndarray, values_h: np.ndarray, q_bf16_row: np.ndarray, idx=None,
+              scale: Optional[float] = None) -> np.ndarray:
+    """fp64 softmax attention of one query over keys idx (all keys if None).
+    keys_h, values_h float32 [n][d]; scale defaults to 1/sqrt(d)."""
+    keys_h = np.ascontiguousarray(keys_h, np.float32)
+    values_h = np.ascontiguousarray(values_h, np.float32)
+    n, d = keys_h.shape
+    q = np.ascontiguousarray(q_bf16_row, np.uint16)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.empty(d, np.float64)
+    if idx is None:
+        rc = _load().fo_attention(_p(keys_h), _p(values_h), n, d, _p(q), None, 0, scale, _p(out))
+    else:
+        ii = np.ascontiguousarray(idx, np.int32)
+        rc = _load().fo_attention(_p(keys_h), _p(values_h), n, d, _p(q), _p(ii), ii.shape[0],
+                                  scale, _p(out))
+    _check(rc, "attention")
+    return out
+
+
+def attention_error(o: np.ndarray, o_exact: np.ndarray) -> float:
+    """Relative L2 error ||o - o_exact|| / ||o_exact|| (the pages name an
+    attention error but give no formula; this is the reading used)."""
+    o = np.asarray(o, np.float64)
+    o_exact = np.asarray(o_exact, np.float64)
+    return float(np.linalg.norm(o - o_exact) / np.linalg.norm(o_exact))

@@ -439,3 +439,45 @@ int fo_topk(const double *s, int64_t n, int64_t k, int32_t *idx, double *top_s)
     free(items);
     return FO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* After the scan: attention over the selected keys.                    */
+/* ------------------------------------------------------------------ */
+
+/* Softmax attention of one query over the keys listed in idx (the top-k the
+ * scan selected; the explainer scores keys to decide which K/V to fetch for
+ * sparse decoding, 解决什么真问题): logits l_i = scale * (q . K[idx_i]) with
+ * q the bf16 query widened exactly, p = softmax(l) (max subtracted), out =
+ * sum_i p_i V[idx_i]; all in fp64.  idx = NULL attends to all n keys (the
+ * dense reference of the attention-error metric).
+ * keys_h, values_h float32 [n][d]; out [d]. */
+int fo_attention(const float *keys_h, const float *values_h, int64_t n, int64_t d,
+                 const uint16_t *q_bf16, const int32_t *idx, int64_t k, double scale,
+                 double *out)
+{
+    const int64_t cnt = idx ? k : n;
+    if (cnt < 1 || d < 1) return FO_ERR_ARG;
+    double *logit = (double *)malloc((size_t)cnt * sizeof *logit);
+    if (!logit) return FO_ERR_ARG;
+    double mx = -INFINITY;
+    for (int64_t i = 0; i < cnt; ++i) {
+        const int64_t j = idx ? idx[i] : i;
+        if (j < 0 || j >= n) { free(logit); return FO_ERR_ARG; }
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            acc += (double)bf16_value(q_bf16[c]) * (double)keys_h[j * d + c];
+        logit[i] = scale * acc;
+        if (logit[i] > mx) mx = logit[i];
+    }
+    for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+    double denom = 0.0;
+    for (int64_t i = 0; i < cnt; ++i) {
+        const int64_t j = idx ? idx[i] : i;
+        const double p = exp(logit[i] - mx);
+        denom += p;
+        for (int64_t c = 0; c < d; ++c) out[c] += p * (double)values_h[j * d + c];
+    }
+    for (int64_t c = 0; c < d; ++c) out[c] /= denom;
+    free(logit);
+    return FO_OK;
+}

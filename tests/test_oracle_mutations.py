@@ -32,6 +32,10 @@ MUTATIONS = {
     "append_variance_old_count": ("const int64_t nn = n + m;", "const int64_t nn = n;"),
     "append_no_high_clamp_count": ("out_of_range = level < 0.0f || level > (float)FO_LEVELS;",
                                    "out_of_range = level < 0.0f;"),
+    "attention_no_max_shift": ("const double p = exp(logit[i] - mx);", "const double p = exp(logit[i]);"),
+    "attention_unscaled_logits": ("logit[i] = scale * acc;", "logit[i] = acc;"),
+    "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
+                               "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
 }
 
 PIN_TESTS = [
@@ -49,6 +53,8 @@ PIN_TESTS = [
     lambda: pins.test_append_in_range_equals_repacking_everything(127, 129),
     pins.test_append_clamps_out_of_range_keys_to_the_end_levels,
     pins.test_append_keeps_sigma2_the_variance_of_the_stored_keys,
+    pins.test_attention_over_every_key_is_dense_attention,
+    pins.test_attention_special_cases,
 ]
 
 

@@ -409,3 +409,50 @@ def test_append_rejects_overflow_and_nonfinite():
     bad[0, 0, 3] = np.inf
     with pytest.raises(ValueError):
         oracle.append(ix, bad)
+
+
+# ------------------------------------------------------------- attention
+def _kv(seed, n, d):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((n, d)).astype(np.float32),
+            rng.standard_normal((n, d)).astype(np.float32),
+            synth.f32_to_bf16_bits(rng.standard_normal(d).astype(np.float32)))
+
+
+def test_attention_over_every_key_is_dense_attention():
+    K, V, q = _kv(1, 300, 16)
+    dense = oracle.attention(K, V, q)
+    listed = oracle.attention(K, V, q, np.arange(300)[::-1].copy())   # order is irrelevant
+    np.testing.assert_allclose(listed, dense, rtol=1e-12, atol=1e-14)
+    # against the softmax written with numpy's exp and matmul
+    qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+    logit = (K.astype(np.float64) @ qf) / 4.0
+    p = np.exp(logit - logit.max())
+    np.testing.assert_allclose(dense, (p / p.sum()) @ V.astype(np.float64), rtol=1e-10)
+
+
+def test_attention_special_cases():
+    K, V, q = _kv(2, 50, 8)
+    # one key: its value row exactly
+    assert np.array_equal(oracle.attention(K, V, q, np.array([17])), V[17].astype(np.float64))
+    # a zero query: the plain mean of the listed value rows
+    zero = np.zeros(8, np.uint16)
+    sel = np.array([3, 9, 20, 41])
+    np.testing.assert_allclose(oracle.attention(K, V, zero, sel), V[sel].astype(np.float64).mean(0),
+                               rtol=1e-12)
+    # a key far above the others takes all the weight, even with logits in
+    # the thousands (softmax must stay finite)
+    K2 = K.copy()
+    K2[5] = 1000.0 * synth.bf16_bits_to_f32(q)
+    out = oracle.attention(K2, V, q, np.array([1, 5, 7]))
+    assert np.all(np.isfinite(out))
+    np.testing.assert_allclose(out, V[5], atol=1e-9)
+
+
+def test_attention_error_metric():
+    o = np.array([1.0, 0.0, 0.0])
+    assert oracle.attention_error(o, o) == 0.0
+    assert abs(oracle.attention_error(np.array([1.0, 0.5, 0.0]), o) - 0.5) < 1e-15
+    with pytest.raises(ValueError):
+        oracle.attention(np.zeros((4, 2), np.float32), np.zeros((4, 2), np.float32),
+                         np.zeros(2, np.uint16), np.array([4]))
