@@ -3,7 +3,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
                     [--workload qwen3_8b_layer_128k|host_1m|host_256k|fixed_vs_wf_1m|
-                               agent_16_sessions|append_layer_128k]
+                               agent_16_sessions|append_layer_128k|
+                               attention_layer_128k]
 
 A step is one decode-step scan of a whole layer through the hot path, once
 per plan of the workload: plan (reverse water-filling at B bits per key, or
@@ -65,6 +66,11 @@ WORKLOADS = {
     # into a packed Qwen3-8B-shaped layer
     "append_layer_128k": dict(H=8, G=4, n=131072, d=128, k=0, residency="device",
                               append=(1, 8192), plans=None),
+    # after the scan: attention over each plan's top-k, with its error
+    # against dense attention (and against attention over the exact top-k)
+    "attention_layer_128k": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
+                                 plans=(("wf", 68), ("wf", 92), ("wf", 136), ("fixed", 34),
+                                        ("fixed", 17)), attention=True),
     "agent_16_sessions": dict(H=8, G=4, n=None, d=128, k=1024, residency="host_mapped",
                               sessions=16, plans=None, device_keys=True, batched=True),
 }
@@ -658,9 +664,112 @@ def run_append(args, wl_name, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_attention_bench(args, wl_name, wl):
+    """Attention over the selected keys: for each plan, plan + scan once, then
+    K timed attention calls over that top-k (one CUDA graph, CUDA events per
+    call).  Roofline: the attention reads k K rows and k V rows per query
+    (Q*k*2*d*4 bytes).  Quality: relative L2 error of the output against
+    dense attention over all n keys (torch, outside the path), beside the
+    error of attention over the exact fp32 top-k (the best k keys)."""
+    import torch
+    import decode_fathom_plan_b200 as fp
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    fp.load_library()
+    H, G, n, d, k = wl["H"], wl["G"], wl["n"], wl["d"], wl["k"]
+    Q = H * G
+    W, K = max(3, args.warmup), args.steps
+    ses = synth.make_session(rank, H, G, n, 64, head_dim=d)
+    keys = torch.from_numpy(ses.keys).cuda()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(10_000 + rank)
+    values = torch.randn((H, n, d), generator=gen, device="cuda", dtype=torch.float32)
+    index = fp.KeyIndex(H, G, n, d, "device")
+    index.pack(keys)
+    q = torch.from_numpy(synth.draw_queries(20_000 + rank, Q, d, count=1)[0].view(np.int16)).cuda()
+    scale = 1.0 / float(np.sqrt(d))
+    out = torch.empty((Q, d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(fp.fathom_sparse_attention_workspace_bytes(Q, d, k), dtype=torch.uint8,
+                     device="cuda")
+    qf = q.view(torch.bfloat16).float().reshape(H, G, d)
+
+    def attend(idx):
+        fp.fathom_sparse_attention(keys, values, H, G, d, n, q, idx, k, scale, out, ws)
+
+    with torch.no_grad():
+        logits = torch.einsum("hnd,hgd->hgn", keys, qf) * scale          # [H][G][n]
+        dense = torch.einsum("hgn,hnd->hgd", torch.softmax(logits, dim=-1), values)
+        exact_idx = logits.topk(k, dim=-1).indices.reshape(Q, k).int().contiguous()
+    attend(exact_idx)
+    torch.cuda.synchronize()
+    o_exactk = out.clone().reshape(H, G, d)
+
+    def rel_err(o):
+        return float(((o - dense).norm(dim=-1) / dense.norm(dim=-1)).mean())
+
+    per_plan, times = [], []
+    for spec in wl["plans"]:
+        buf = fp.ScanBuffers(index, k)
+        bvec = torch.full((Q,), plan_bits(spec), dtype=torch.int32, device="cuda")
+        fp.plan_and_scan(index, q, bvec, buf, fixed_r=spec[1] if spec[0] == "fixed" else None)
+        for _ in range(W):
+            attend(buf.idx)
+        ev = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+                for i in range(K):
+                    ev[i][0].record()
+                    attend(buf.idx)
+                    ev[i][1].record()
+        torch.cuda.current_stream().wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
+        del graph
+        assert fp.fathom_last_device_status() == fp.FATHOM_OK
+        ms = statistics.median([a.elapsed_time(b) for a, b in ev])
+        times.append(ms)
+        per_plan.append({"plan": plan_name(spec), "bits_per_key": plan_bits(spec),
+                         "attention_us": ms * 1e3,
+                         "attention_error_vs_dense": rel_err(out.reshape(H, G, d)),
+                         "recall_vs_exact_fp32": float(np.mean([
+                             len(np.intersect1d(buf.idx[i].cpu().numpy(),
+                                                exact_idx[i].cpu().numpy())) / k
+                             for i in range(Q)]))})
+    nbytes = Q * k * 2 * d * 4
+    ms = statistics.median(times)
+    peak, peak_src = load_peaks()
+    line = {"metric": "sparse attention over the selected keys: KV-head keys attended per second",
+            "value": Q * k / (ms / 1e3) / 1e9, "unit": "Gkeys/s", "n_gpus": 1, "steps": K,
+            "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl_name, "kv_heads": H, "query_heads_per_kv": G,
+                       "head_dim": d, "n_keys": n, "k": k,
+                       "plans": [plan_name(p) for p in wl["plans"]]},
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / peak,
+                         "traffic": None, "kernel": "attention_split_kernel + combine",
+                         "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)",
+                         "algorithmic_bytes_per_launch": nbytes},
+            "attention_error_exact_topk_vs_dense": rel_err(o_exactk),
+            "per_plan": per_plan, "launch_mode": "cuda_graph"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     wl = WORKLOADS[args.workload]
+    if wl.get("attention"):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the attention workload has no CPU reference leg"}))
+        else:
+            run_attention_bench(args, args.workload, wl)
+        return
     if wl.get("append"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable":

@@ -38,6 +38,7 @@ EXPORTED = (
     "fathom_scan_batched_workspace_bytes", "fathom_scan_topk_batched",
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
     "fathom_scan_topk_static", "fathom_link_probe", "fathom_append_keys",
+    "fathom_sparse_attention_workspace_bytes", "fathom_sparse_attention",
 )
 
 
@@ -79,6 +80,9 @@ def load_library(path: str = LIB_PATH):
         "fathom_pack_workspace_bytes": ([IX], SZ),
         "fathom_pack_keys": ([P, IX, P, SZ, P], ctypes.c_int),
         "fathom_append_keys": ([IX, P, I32, P, P], ctypes.c_int),
+        "fathom_sparse_attention_workspace_bytes": ([I32, I32, I32], SZ),
+        "fathom_sparse_attention": ([P, P, I32, I32, I32, I32, P, P, I32, ctypes.c_float, P, P,
+                                     SZ, P], ctypes.c_int),
         "fathom_plan": ([IX, P, P, P, P, P, P], ctypes.c_int),
         "fathom_fixed_plan": ([IX, P, I32, P, P, P, P], ctypes.c_int),
         "fathom_scan_workspace_bytes": ([IX, I32], SZ),
@@ -213,6 +217,22 @@ def fathom_scan_topk_batched(sessions: Sequence[fathom_index], q_bf16, t, t_unio
         vp(*[_ptr(x) for x in t_union]), int(k), vp(*[_ptr(x) for x in out_idx]),
         vp(*[_ptr(x) for x in out_score]), _ptr(workspace), ws_bytes, int(flags),
         _stream(stream)), "fathom_scan_topk_batched")
+
+
+def fathom_sparse_attention_workspace_bytes(n_queries: int, head_dim: int, k: int) -> int:
+    return int(load_library().fathom_sparse_attention_workspace_bytes(int(n_queries),
+                                                                       int(head_dim), int(k)))
+
+
+def fathom_sparse_attention(keys, values, n_kv_heads: int, group: int, head_dim: int,
+                            n_keys: int, q_bf16, idx, k: int, softmax_scale: float, out,
+                            workspace, stream=None):
+    """Softmax attention of each query over its k selected keys (fp32)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().fathom_sparse_attention(
+        _ptr(keys), _ptr(values), int(n_kv_heads), int(group), int(head_dim), int(n_keys),
+        _ptr(q_bf16), _ptr(idx), int(k), float(softmax_scale), _ptr(out), _ptr(workspace),
+        ws_bytes, _stream(stream)), "fathom_sparse_attention")
 
 
 def fathom_last_device_status(stream=None) -> int:

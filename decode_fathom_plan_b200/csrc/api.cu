@@ -162,6 +162,39 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
     return cuda_status(e);
 }
 
+// A device-usable address for a K or V array: device or managed memory as
+// is, pinned host memory through its device mapping; 16-byte aligned.
+fathom_status resolve_kv(const float *p, const float **out)
+{
+    if (!p || !aligned16(p)) return FATHOM_ERR_INVALID_ARG;
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return FATHOM_ERR_INVALID_ARG;
+    }
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return FATHOM_OK;
+    }
+    if (attr.type == cudaMemoryTypeHost) {
+        void *dptr = nullptr;
+        if (cudaHostGetDevicePointer(&dptr, const_cast<float *>(p), 0) != cudaSuccess || !dptr) {
+            cudaGetLastError();
+            return FATHOM_ERR_INVALID_ARG;
+        }
+        *out = static_cast<const float *>(dptr);
+        return FATHOM_OK;
+    }
+    return FATHOM_ERR_INVALID_ARG;
+}
+
+size_t attention_bytes(int32_t n_queries, int32_t head_dim, int32_t k)
+{
+    if (n_queries < 1 || head_dim < 32 || head_dim > kMaxHeadDim || head_dim % 32 || k < 1)
+        return 0;
+    return (size_t)n_queries * fathom::attention_splits(k) * (size_t)(head_dim + 2) * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
@@ -314,6 +347,32 @@ fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_
     if (scan_kernel_ms) *scan_kernel_ms = total;
     if (scan_kernel_launches) *scan_kernel_launches = recs.size();
     return st;
+}
+
+size_t fathom_sparse_attention_workspace_bytes(int32_t n_queries, int32_t head_dim, int32_t k)
+{
+    return attention_bytes(n_queries, head_dim, k);
+}
+
+fathom_status fathom_sparse_attention(const float *keys, const float *values, int32_t n_kv_heads,
+                                      int32_t group, int32_t head_dim, int32_t n_keys,
+                                      const uint16_t *q_bf16, const int32_t *idx, int32_t k,
+                                      float softmax_scale, float *out, void *workspace,
+                                      size_t workspace_bytes, cudaStream_t stream)
+{
+    if (n_kv_heads < 1 || group < 1 || group > kMaxGroup || n_keys < 1) return FATHOM_ERR_INVALID_ARG;
+    if (head_dim < 32 || head_dim > kMaxHeadDim || head_dim % 32) return FATHOM_ERR_INVALID_ARG;
+    if (k < 1 || k > n_keys || !q_bf16 || !idx || !out || !isfinite(softmax_scale))
+        return FATHOM_ERR_INVALID_ARG;
+    const float *kd = nullptr, *vd = nullptr;
+    fathom_status st = resolve_kv(keys, &kd);
+    if (st != FATHOM_OK) return st;
+    if ((st = resolve_kv(values, &vd)) != FATHOM_OK) return st;
+    const size_t need = attention_bytes(n_kv_heads * group, head_dim, k);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FATHOM_ERR_WORKSPACE;
+    return cuda_status(fathom::launch_attention(kd, vd, n_kv_heads, group, head_dim, n_keys, q_bf16,
+                                                idx, k, softmax_scale, out,
+                                                static_cast<float *>(workspace), stream));
 }
 
 }  // extern "C"

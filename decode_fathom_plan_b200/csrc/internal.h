@@ -46,6 +46,15 @@ struct FetchJob {
 };
 cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream);
 
+// ---- attention.cu
+// Split-K runs per query for k selected keys.
+int attention_splits(int k);
+// Attention of Q = H*G queries over their k selected keys; part: workspace
+// of Q * attention_splits(k) * (d + 2) floats.
+cudaError_t launch_attention(const float *keys, const float *values, int H, int G, int d, int n,
+                             const uint16_t *q_bf16, const int32_t *idx, int k, float scale,
+                             float *out, float *part, cudaStream_t stream);
+
 // ---- scan.cu
 struct ScanSessionArgs {
     const fathom_index *ix;

@@ -247,6 +247,31 @@ fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_s
                                        uint32_t flags, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
+/* After the scan: attention over the selected keys.                      */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes fathom_sparse_attention needs (0 for invalid sizes). */
+size_t fathom_sparse_attention_workspace_bytes(int32_t n_queries, int32_t head_dim, int32_t k);
+
+/* Softmax attention of each query over the k keys its top-k selected (the
+ * step after the scan: the explainer's decode step fetches and attends over
+ * the selected K/V rows, 解决什么真问题): for query q of KV head q / G,
+ *   l_i = softmax_scale * (q . K[h][idx[q][i]]),  p = softmax(l),
+ *   out[q] = sum_i p_i * V[h][idx[q][i]],
+ * in float32 (q the bf16 query widened exactly).
+ * keys, values: float32 [H][n][d], device memory or pinned host memory
+ * (read through its device mapping), 16-byte aligned; q_bf16 [Q][d],
+ * idx int32 [Q][k] (e.g. fathom_scan_topk's out_idx), out float32 [Q][d]:
+ * device pointers.  1 <= k <= n; head_dim a multiple of 32, at most 256;
+ * G 1..8.  An index outside [0, n) is skipped and sets
+ * FATHOM_ERR_INVALID_ARG in the device status. */
+fathom_status fathom_sparse_attention(const float *keys, const float *values, int32_t n_kv_heads,
+                                      int32_t group, int32_t head_dim, int32_t n_keys,
+                                      const uint16_t *q_bf16, const int32_t *idx, int32_t k,
+                                      float softmax_scale, float *out, void *workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* Status and instrumentation.                                            */
 /* ---------------------------------------------------------------------- */
 

@@ -123,3 +123,24 @@ def test_append_rejects_bad_arguments_before_launching(lib):
     bad = _desc(d=48)
     assert append(ctypes.byref(bad), fake, 1, None, None) == F
     assert ix.n_keys == 100                  # untouched on error
+
+
+def test_sparse_attention_sizes_and_argument_checks(lib):
+    ws = fp.fathom_sparse_attention_workspace_bytes
+    assert ws(32, 128, 2048) == 32 * 16 * 130 * 4       # 16 runs of 128 keys per query
+    assert ws(1, 32, 1) == 1 * 1 * 34 * 4
+    assert ws(1, 48, 10) == 0 and ws(0, 128, 10) == 0 and ws(1, 128, 0) == 0
+    fake = 0x1000
+    att = lib.fathom_sparse_attention
+    F = fp.FATHOM_ERR_INVALID_ARG
+    args = lambda **kw: dict(dict(keys=fake, values=fake, H=1, G=1, d=128, n=10, q=fake,
+                                  idx=fake, k=4, scale=0.1, out=fake, ws=fake, wsb=1 << 20), **kw)
+    def call(a):
+        return att(a["keys"], a["values"], a["H"], a["G"], a["d"], a["n"], a["q"], a["idx"],
+                   a["k"], ctypes.c_float(a["scale"]), a["out"], a["ws"], a["wsb"], None)
+    assert call(args(k=11)) == F            # k > n
+    assert call(args(k=0)) == F
+    assert call(args(d=40)) == F
+    assert call(args(G=9)) == F
+    assert call(args(idx=None)) == F
+    assert call(args(scale=float("nan"))) == F
