@@ -51,6 +51,7 @@ def _load():
             "fo_channel_stats": ([P, I, I, I, P, P, P, P], ctypes.c_int),
             "fo_importance": ([P, P, I, P], ctypes.c_int),
             "fo_plan_greedy": ([P, I, I, P], ctypes.c_int),
+            "fo_plan_marginal": ([P, I, I, P], ctypes.c_int),
             "fo_fixed_plan": ([P, I, I, P], ctypes.c_int),
             "fo_union": ([P, I, I, P], None),
             "fo_plan_bytes": ([P, I, I], ctypes.c_uint64),
@@ -165,6 +166,14 @@ def plan_greedy(w: np.ndarray, B: int) -> np.ndarray:
     return t
 
 
+def plan_marginal(w: np.ndarray, B: int) -> np.ndarray:
+    """Marginal-gain plan: bits one at a time to the largest w_c * 4^-t_c."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    t = np.empty(w.shape[0], np.uint8)
+    _check(_load().fo_plan_marginal(_p(w), w.shape[0], int(B), _p(t)), "plan_marginal")
+    return t
+
+
 def fixed_plan(q_bf16: np.ndarray, r: int) -> np.ndarray:
     q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
     t = np.empty(q.shape[0], np.uint8)
@@ -259,17 +268,19 @@ def build_index(keys: np.ndarray, capacity: Optional[int] = None) -> Dict[str, n
 
 
 def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
-                 fixed_r: Optional[int] = None):
+                 fixed_r: Optional[int] = None, marginal: bool = False):
     """-> (t uint8 [Q][d], T uint8 [H][d], bytes uint64 [Q+H])."""
     H, d = index["mn"].shape
     Q = H * group
     t = np.empty((Q, d), np.uint8)
     for q in range(Q):
         h = q // group
-        if fixed_r is None:
-            t[q] = plan_greedy(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
-        else:
+        if fixed_r is not None:
             t[q] = fixed_plan(q_bf16[q], fixed_r)
+        elif marginal:
+            t[q] = plan_marginal(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
+        else:
+            t[q] = plan_greedy(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
     T = np.stack([union(t[h * group:(h + 1) * group]) for h in range(H)])
     nb = np.array([plan_bytes(t[q], index["n_words"]) for q in range(Q)]
                   + [plan_bytes(T[h], index["n_words"]) for h in range(H)], np.uint64)

@@ -278,6 +278,36 @@ int fo_plan_greedy(const float *w, int64_t d, int64_t B, uint8_t *t)
     return FO_OK;
 }
 
+/* Marginal-gain plan (a finer reverse water-filling for continuous
+ * importance; the explainer's simplified walk hands out whole 4-bit
+ * channels, 核心方法 / 读侧, and notes that finer handling is possible).
+ * Reading: the distortion of a channel read at t bits falls as 4^-t, so
+ * bit t+1 of channel c is worth w_c * 4^-t; the B bits go one at a time to
+ * the channel of largest w_c * 4^-t_c (t_c < 4), ties to the lower channel.
+ * 4^-t is a power of two, so the float gains are exact.  B in [0, 4d]. */
+int fo_plan_marginal(const float *w, int64_t d, int64_t B, uint8_t *t)
+{
+    if (B < 0 || B > FO_BITS * d) return FO_ERR_ARG;
+    for (int64_t c = 0; c < d; ++c) {
+        if (!isfinite(w[c])) return FO_ERR_NONFINITE;
+        t[c] = 0;
+    }
+    for (int64_t b = 0; b < B; ++b) {
+        int64_t best = -1;
+        float best_gain = 0.0f;
+        for (int64_t c = 0; c < d; ++c) {
+            if (t[c] >= FO_BITS) continue;
+            const float gain = w[c] * (1.0f / (float)(1 << (2 * t[c])));
+            if (best < 0 || gain > best_gain) {
+                best = c;
+                best_gain = gain;
+            }
+        }
+        t[best] += 1;
+    }
+    return FO_OK;
+}
+
 /* Fixed-width baseline plan: the r channels of largest |q_c| (ties to the
  * lower channel) are read at all 4 bits, the rest not at all. */
 int fo_fixed_plan(const uint16_t *q_bf16, int64_t d, int64_t r, uint8_t *t)

@@ -34,6 +34,9 @@ MUTATIONS = {
                                    "out_of_range = level < 0.0f;"),
     "attention_no_max_shift": ("const double p = exp(logit[i] - mx);", "const double p = exp(logit[i]);"),
     "attention_unscaled_logits": ("logit[i] = scale * acc;", "logit[i] = acc;"),
+    "marginal_gain_ignores_depth": ("const float gain = w[c] * (1.0f / (float)(1 << (2 * t[c])));",
+                                    "const float gain = w[c];"),
+    "marginal_gain_halves": ("(float)(1 << (2 * t[c]))", "(float)(1 << t[c])"),
     "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
                                "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
 }
@@ -55,6 +58,8 @@ PIN_TESTS = [
     pins.test_append_keeps_sigma2_the_variance_of_the_stored_keys,
     pins.test_attention_over_every_key_is_dense_attention,
     pins.test_attention_special_cases,
+    pins.test_marginal_plan_spreads_uniform_importance_round_robin,
+    pins.test_marginal_plan_hand_worked,
 ]
 
 

@@ -456,3 +456,41 @@ def test_attention_error_metric():
     with pytest.raises(ValueError):
         oracle.attention(np.zeros((4, 2), np.float32), np.zeros((4, 2), np.float32),
                          np.zeros(2, np.uint16), np.array([4]))
+
+
+# ------------------------------------------------------- marginal-gain plan
+def _distortion_drop(w, t):
+    """Sum_c w_c (1 - 4^-t_c): the distortion a plan removes when a channel
+    read at t bits keeps 4^-t of its variance."""
+    return float(np.sum(np.asarray(w, np.float64) * (1.0 - 4.0 ** (-np.asarray(t, np.float64)))))
+
+
+@pytest.mark.parametrize("d", [3, 5])
+def test_marginal_plan_is_optimal_by_brute_force(d):
+    rng = np.random.default_rng(d)
+    for trial in range(6):
+        w = rng.lognormal(0.0, 1.5, d).astype(np.float32)
+        for B in range(0, 4 * d + 1):
+            t = oracle.plan_marginal(w, B)
+            assert int(t.sum()) == B and t.max() <= 4
+            best = max(_distortion_drop(w, c) for c in itertools.product(range(5), repeat=d)
+                       if sum(c) == B)
+            assert abs(_distortion_drop(w, t) - best) <= 1e-9 * max(1.0, best)
+
+
+def test_marginal_plan_spreads_uniform_importance_round_robin():
+    d = 10
+    w = np.full(d, 2.5, np.float32)
+    for B in range(0, 4 * d + 1):
+        t = oracle.plan_marginal(w, B)
+        expect = np.array([B // d + (c < B % d) for c in range(d)])
+        assert np.array_equal(t, expect), B
+
+
+def test_marginal_plan_hand_worked():
+    # gains of channel 0: 16, 4, 1, 1/4; channel 1: 1, 1/4, ...; ties -> channel 0
+    w = np.array([16.0, 1.0], np.float32)
+    assert [list(oracle.plan_marginal(w, B)) for B in range(1, 6)] == \
+        [[1, 0], [2, 0], [3, 0], [3, 1], [4, 1]]
+    # water-filling instead fills channel 0 to 4 bits before channel 1 gets any
+    assert list(oracle.plan_greedy(w, 4)) == [4, 0]
