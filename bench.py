@@ -2,7 +2,7 @@
 """Benchmark of the Fathom per-query read-depth top-k key scan on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
-                    [--workload qwen3_8b_layer_128k|host_1m|host_256k|fixed_vs_wf_1m|
+                    [--workload qwen3_8b_layer_128k|plan_variants_128k|host_1m|host_256k|fixed_vs_wf_1m|
                                agent_16_sessions|append_layer_128k|
                                attention_layer_128k]
 
@@ -46,8 +46,8 @@ UNIT = "Gkeys/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
-# plans: ("wf", B) = reverse water-filling at B bits per key; ("fixed", r) =
-# the top-r channels by |q_c| at 4 bits.  "device_keys": keys drawn on the
+# plans: ("wf", B) = reverse water-filling at B bits per key; ("mg", B) = the
+# marginal-gain variant; ("fixed", r) = the top-r channels by |q_c| at 4 bits.  "device_keys": keys drawn on the
 # GPU (synth.device_keys) instead of numpy, for sizes numpy would take
 # minutes on.  agent_16_sessions scans its sessions in one batched call.
 WORKLOADS = {
@@ -59,6 +59,10 @@ WORKLOADS = {
     # kernel (its traffic scales with n)
     "host_256k": dict(H=8, G=4, n=1 << 18, d=128, k=2048, residency="host_mapped",
                       plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
+    # reverse water-filling against its marginal-gain variant, same budgets
+    "plan_variants_128k": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
+                               plans=(("wf", 68), ("mg", 68), ("wf", 92), ("mg", 92),
+                                      ("wf", 136), ("mg", 136))),
     "fixed_vs_wf_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                            plans=(("fixed", 34), ("fixed", 17), ("wf", 68), ("wf", 92)),
                            device_keys=True),
@@ -82,7 +86,7 @@ def plan_name(spec):
 
 def plan_bits(spec):
     """Bits per key a query of this plan reads."""
-    return spec[1] if spec[0] == "wf" else 4 * spec[1]
+    return 4 * spec[1] if spec[0] == "fixed" else spec[1]
 
 
 def parse_args():
@@ -230,6 +234,8 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0):
             qrow = q_bf16[hi * G + g]
             if spec[0] == "wf":
                 tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1])
+            elif spec[0] == "mg":
+                tq = oracle.plan_marginal(oracle.importance(qrow, ref["sigma2"][hi]), spec[1])
             else:
                 tq = oracle.fixed_plan(qrow, spec[1])
             s = oracle.score_planes(ref["planes"][hi], ref["mn"][hi], ref["scale"][hi],
@@ -411,6 +417,9 @@ def run_fathom(args, wl_name, wl):
         b = j["buf"]
         if j["spec"][0] == "wf":
             fp.fathom_plan(S["index"].desc, S["q"][i], j["bvec"], b.t, b.t_union, b.nbytes)
+        elif j["spec"][0] == "mg":
+            fp.fathom_plan_marginal(S["index"].desc, S["q"][i], j["bvec"], b.t, b.t_union,
+                                    b.nbytes)
         else:
             fp.fathom_fixed_plan(S["index"].desc, S["q"][i], j["spec"][1], b.t, b.t_union,
                                  b.nbytes)

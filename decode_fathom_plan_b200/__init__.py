@@ -38,7 +38,7 @@ EXPORTED = (
     "fathom_scan_batched_workspace_bytes", "fathom_scan_topk_batched",
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
     "fathom_scan_topk_static", "fathom_link_probe", "fathom_append_keys",
-    "fathom_sparse_attention_workspace_bytes", "fathom_sparse_attention",
+    "fathom_sparse_attention_workspace_bytes", "fathom_sparse_attention", "fathom_plan_marginal",
 )
 
 
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH):
                                      SZ, P], ctypes.c_int),
         "fathom_plan": ([IX, P, P, P, P, P, P], ctypes.c_int),
         "fathom_fixed_plan": ([IX, P, I32, P, P, P, P], ctypes.c_int),
+        "fathom_plan_marginal": ([IX, P, P, P, P, P, P], ctypes.c_int),
         "fathom_scan_workspace_bytes": ([IX, I32], SZ),
         "fathom_scan_topk": ([IX, P, P, P, I32, P, P, P, SZ, U32, P], ctypes.c_int),
         "fathom_scan_topk_static": ([IX, P, P, P, I32, P, P, U32, P], ctypes.c_int),
@@ -162,6 +163,12 @@ def fathom_plan(index: fathom_index, q_bf16, budget, t, t_union, nbytes, stream=
     _check(load_library().fathom_plan(ctypes.byref(index), _ptr(q_bf16), _ptr(budget), _ptr(t),
                                       _ptr(t_union), _ptr(nbytes), _stream(stream)),
            "fathom_plan")
+
+
+def fathom_plan_marginal(index: fathom_index, q_bf16, budget, t, t_union, nbytes, stream=None):
+    _check(load_library().fathom_plan_marginal(ctypes.byref(index), _ptr(q_bf16), _ptr(budget),
+                                               _ptr(t), _ptr(t_union), _ptr(nbytes),
+                                               _stream(stream)), "fathom_plan_marginal")
 
 
 def fathom_fixed_plan(index: fathom_index, q_bf16, r: int, t, t_union, nbytes, stream=None):

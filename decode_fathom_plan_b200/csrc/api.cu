@@ -259,6 +259,15 @@ fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
     return cuda_status(launch_plan(*index, q_bf16, budget, 0, false, t, t_union, bytes, stream));
 }
 
+fathom_status fathom_plan_marginal(const fathom_index *index, const uint16_t *q_bf16,
+                                   const int32_t *budget, uint8_t *t, uint8_t *t_union,
+                                   uint64_t *bytes, cudaStream_t stream)
+{
+    if (!index_shape_ok(index) || !index->sigma2) return FATHOM_ERR_INVALID_ARG;
+    if (!q_bf16 || !budget || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
+    return cuda_status(launch_plan_marginal(*index, q_bf16, budget, t, t_union, bytes, stream));
+}
+
 fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf16, int32_t r,
                                 uint8_t *t, uint8_t *t_union, uint64_t *bytes,
                                 cudaStream_t stream)

@@ -33,6 +33,9 @@ cudaError_t launch_append(const float *keys, const fathom_index &ix, int m, uint
 cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
                         int32_t fixed_r, bool fixed, uint8_t *t, uint8_t *t_union,
                         uint64_t *bytes, cudaStream_t stream);
+cudaError_t launch_plan_marginal(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
+                                 uint8_t *t, uint8_t *t_union, uint64_t *bytes,
+                                 cudaStream_t stream);
 
 // ---- fetch.cu
 // One host-resident index to fetch: for each of its n_channels = H*d

@@ -136,6 +136,94 @@ plan_kernel(const uint16_t *__restrict__ q, const int32_t *__restrict__ budget, 
     }
 }
 
+// Marginal-gain plan (a finer reverse water-filling; the explainer's walk
+// hands out whole 4-bit channels, 核心方法 / 读侧): bit s+1 of channel c is
+// worth w_c * 4^-s, the B most valuable (channel, bit) pairs are read, ties
+// to the lower channel then the lower bit.  A warp sorts the 4*d pairs of
+// its query (value as an order key, then ~(4c + s)); since a channel's
+// values fall with s, the selected bits of a channel are a prefix and t_c is
+// one past its deepest selected bit.  4^-s is a power of two, so the values
+// are exact.  E = padded head_dim / 32.
+template <int E>
+__global__ void __launch_bounds__(kMaxGroup * 32)
+plan_marginal_kernel(const uint16_t *__restrict__ q, const int32_t *__restrict__ budget,
+                     const float *__restrict__ sigma2, int G, int d, int n_words, uint8_t *t,
+                     uint8_t *t_union, uint64_t *bytes, int Q, int *status)
+{
+    constexpr int E4 = kBits * E;
+    __shared__ int tt[kMaxGroup][kMaxHeadDim];
+    const int h = blockIdx.x;
+    const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned long long plane_bytes = 4ull * (unsigned long long)n_words;
+    const int qi = h * G + g;
+    unsigned long long key[E4];
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = lane * E + i;
+        float w = 0.0f;
+        if (c < d) {
+            const float qf = bf16_to_float(q[(size_t)qi * d + c]);
+            w = __fmul_rn(__fmul_rn(qf, qf), sigma2[h * d + c]);
+            bad |= !isfinite(w);
+            tt[g][c] = 0;
+        }
+#pragma unroll
+        for (int s = 0; s < kBits; ++s) {
+            const float gain = __fmul_rn(w, 1.0f / (float)(1 << (2 * s)));   // exact
+            key[i * kBits + s] = (c < d) ? (((unsigned long long)order_key(gain) << 32) |
+                                            (0xFFFFFFFFu - (uint32_t)(c * kBits + s)))
+                                         : 0ull;
+        }
+    }
+    bad = __any_sync(0xFFFFFFFFu, bad);
+    int B = budget[qi];
+    if (B < 0 || B > kBits * d) {
+        if (lane == 0) set_status(status, FATHOM_ERR_INVALID_ARG);
+        B = 0;
+    }
+    if (bad) {
+        if (lane == 0) set_status(status, FATHOM_ERR_NONFINITE);
+        B = 0;
+    }
+    __syncwarp();
+    warp_sort_desc<E4>(key);
+#pragma unroll
+    for (int i = 0; i < E4; ++i) {
+        const int rank = lane * E4 + i;
+        if (rank < B && key[i] != 0ull) {
+            const uint32_t cs = 0xFFFFFFFFu - (uint32_t)(key[i] & 0xFFFFFFFFull);
+            atomicMax(&tt[g][cs / kBits], (int)(cs % kBits) + 1);
+        }
+    }
+    __syncwarp();
+    unsigned long long my_bytes = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int c = lane * E + i;
+        if (c < d) {
+            t[(size_t)qi * d + c] = (uint8_t)tt[g][c];
+            my_bytes += (unsigned long long)tt[g][c] * plane_bytes;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) my_bytes += __shfl_xor_sync(0xFFFFFFFFu, my_bytes, off);
+    if (lane == 0) bytes[qi] = my_bytes;
+    __syncthreads();
+    if (g == 0) {   // GQA union, one warp
+        unsigned long long ub = 0;
+        for (int c = lane; c < d; c += 32) {
+            int m = 0;
+            for (int gg = 0; gg < G; ++gg) m = max(m, tt[gg][c]);
+            t_union[h * d + c] = (uint8_t)m;
+            ub += (unsigned long long)m * plane_bytes;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ub += __shfl_xor_sync(0xFFFFFFFFu, ub, off);
+        if (lane == 0) bytes[Q + h] = ub;
+    }
+}
+
 template <bool kFixed>
 void launch_plan_kernel(int E, dim3 grid, int threads, cudaStream_t stream, const uint16_t *q,
                         const int32_t *budget, int32_t fixed_r, const float *sigma2, int G, int d,
@@ -151,6 +239,26 @@ void launch_plan_kernel(int E, dim3 grid, int threads, cudaStream_t stream, cons
 }
 
 }  // namespace
+
+cudaError_t launch_plan_marginal(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
+                                 uint8_t *t, uint8_t *t_union, uint64_t *bytes, cudaStream_t stream)
+{
+    const int H = ix.n_kv_heads, G = ix.group, d = ix.head_dim;
+    const int Q = H * G;
+    int *status = device_status_ptr();
+    int E = 1;
+    while (32 * E < d) E <<= 1;
+    const dim3 grid(H);
+    const int threads = G * 32;
+    switch (E) {
+    case 1: plan_marginal_kernel<1><<<grid, threads, 0, stream>>>(q, budget, ix.sigma2, G, d, ix.n_words, t, t_union, bytes, Q, status); break;
+    case 2: plan_marginal_kernel<2><<<grid, threads, 0, stream>>>(q, budget, ix.sigma2, G, d, ix.n_words, t, t_union, bytes, Q, status); break;
+    case 4: plan_marginal_kernel<4><<<grid, threads, 0, stream>>>(q, budget, ix.sigma2, G, d, ix.n_words, t, t_union, bytes, Q, status); break;
+    default: plan_marginal_kernel<8><<<grid, threads, 0, stream>>>(q, budget, ix.sigma2, G, d, ix.n_words, t, t_union, bytes, Q, status); break;
+    }
+    note_launch(1);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
                         int32_t fixed_r, bool fixed, uint8_t *t, uint8_t *t_union,

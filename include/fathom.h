@@ -172,6 +172,18 @@ fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
                           const int32_t *budget, uint8_t *t, uint8_t *t_union,
                           uint64_t *bytes, cudaStream_t stream);
 
+/* Marginal-gain plan, a finer reverse water-filling (the explainer's walk
+ * hands out whole 4-bit channels; 核心方法 / 读侧 notes finer handling for
+ * continuous importance): bit s+1 of channel c is worth w_c * 4^-s (the
+ * distortion a channel read at t bits keeps falls as 4^-t), and each query
+ * reads its B most valuable (channel, bit) pairs, ties to the lower channel
+ * then the lower bit -- the same as handing the bits out one at a time to
+ * the channel of largest w_c * 4^-t_c.  Same arguments, outputs and errors
+ * as fathom_plan; sum_c t_c = B and t_c <= 4. */
+fathom_status fathom_plan_marginal(const fathom_index *index, const uint16_t *q_bf16,
+                                   const int32_t *budget, uint8_t *t, uint8_t *t_union,
+                                   uint64_t *bytes, cudaStream_t stream);
+
 /* Fixed-width baseline plan (the 136-bit / 68-bit key scans the explainer
  * compares against): the r channels of largest |q_c| (ties to the lower
  * channel) are read at 4 bits, the rest at 0.  Same outputs as
