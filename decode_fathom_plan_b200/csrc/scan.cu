@@ -81,7 +81,7 @@ struct SessionDesc {
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int group_begin, q_begin;
+    int group_begin, q_begin, head_begin;
 };
 
 template <int NS>
@@ -567,6 +567,15 @@ __device__ __forceinline__ int find_session_by_group(const Batch<NS> &b, int g)
 }
 
 template <int NS>
+__device__ __forceinline__ int find_session_by_head(const Batch<NS> &b, int gh)
+{
+    int si = 0;
+    for (int s = 1; s < b.n_sessions; ++s)
+        if (b.s[s].head_begin <= gh) si = s;
+    return si;
+}
+
+template <int NS>
 __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
 {
     int si = 0;
@@ -975,19 +984,21 @@ __device__ void emit_in_index_order(const unsigned long long *sel, int k, int n,
 // 2^-22-of-the-range bin holding the sample_rank-th largest sampled order key
 // (two 11-bit radix passes; any theta is correct, it only sizes the candidate
 // set).  The query's channels, weights and bias come straight from its plan
-// and the index statistics; the CTA of each KV head's first query also
-// builds that head's scan tables for the filtering pass.  Stages of 8 own
-// channels x 2 tiles are copied with cp.async, two in flight; every query of
+// and the index statistics; H further CTAs of the same launch build each KV
+// head's scan tables for the filtering pass.  Stages of 8 own
+// channels x 2 tiles are copied with cp.async, three in flight; every query of
 // a KV head reads its sampled rows itself (a few tens of KB, mostly L2 hits).
 constexpr int kThetaTilesPerPass = kSelThreads / kScanThreads;            // 2
 constexpr int kThetaCols = kThetaTilesPerPass * kTileCols;                // 128 words
 typedef uint32_t (*ThetaBuf)[kStageRows][kThetaCols];
 constexpr size_t kThetaStageBytes = (size_t)kStageRows * kThetaCols * sizeof(uint32_t);
 constexpr int kThetaResolutionBits = 2 * kSelBits;
+constexpr int kThetaBufs = 3;   // stages in flight
 
 template <int NS, int GP>
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_constant__ Batch<NS> b,
-                                                                uint32_t force_exact)
+                                                                uint32_t force_exact,
+                                                                int total_queries)
 {
     extern __shared__ __align__(16) uint32_t th_dyn[];
     __shared__ ScanMeta<GP> sm;
@@ -998,22 +1009,26 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     __shared__ double bias_part[kSelThreads / 32];
     __shared__ float bias_s;
     ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
-    uint32_t *vals = th_dyn + 2 * kStageRows * kThetaCols;
-    const int gq = blockIdx.x;
-    const int si = find_session_by_query(b, gq);
-    const SessionDesc &S = b.s[si];
-    const int qq = gq - S.q_begin;
+    uint32_t *vals = th_dyn + kThetaBufs * kStageRows * kThetaCols;
     const int G = b.G, d = b.d;
-    const int h = qq / G, g = qq - h * G;
-    uint32_t *st = S.qstate + qq * kQueryStateWords;
-    if (!force_exact && g == 0) {   // this KV head's tables for the filtering pass
+    if (blockIdx.x >= total_queries) {   // a KV head's tables for the filtering pass
+        const int gh = blockIdx.x - total_queries;
+        const SessionDesc &S = b.s[find_session_by_head(b, gh)];
+        const int h = gh - S.head_begin;
         setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)h * G * d, S.q + (size_t)h * G * d,
                        S.mn + h * d, S.scale + h * d);
         constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
         const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
         uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
         for (int i = threadIdx.x; i < kUnits; i += blockDim.x) dst[i] = src[i];
+        return;
     }
+    const int gq = blockIdx.x;
+    const int si = find_session_by_query(b, gq);
+    const SessionDesc &S = b.s[si];
+    const int qq = gq - S.q_begin;
+    const int h = qq / G;
+    uint32_t *st = S.qstate + qq * kQueryStateWords;
     if (force_exact || S.exact_only) {
         if (threadIdx.x == 0) { st[0] = 0xFFFFFFFFu; st[1] = 0; st[2] = 1; }
         return;
@@ -1089,16 +1104,19 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
         __syncthreads();   // the buffers are free
-        if (n_stages > 0) load(t0, 0, 0);
+        for (int s2 = 0; s2 < kThetaBufs - 1 && s2 < n_stages; ++s2) load(t0, s2, s2);
         for (int s2 = 0; s2 < n_stages; ++s2) {
-            if (s2 + 1 < n_stages) {
-                load(t0, s2 + 1, (s2 + 1) & 1);
+            // stage s2 has landed once at most (stages issued after it) groups are pending
+            if (s2 + kThetaBufs - 1 < n_stages) {
+                load(t0, s2 + kThetaBufs - 1, (s2 + kThetaBufs - 1) % kThetaBufs);
+                cp_async_wait<kThetaBufs - 1>();
+            } else if (s2 + 1 < n_stages) {
                 cp_async_wait<1>();
             } else {
                 cp_async_wait<0>();
             }
             __syncthreads();
-            const uint32_t(*rows)[kThetaCols] = stage[s2 & 1];
+            const uint32_t(*rows)[kThetaCols] = stage[s2 % kThetaBufs];
             const int j1 = min(n_own, (s2 + 1) * kStageChannels);
             for (int j = s2 * kStageChannels; j < j1; ++j) {
                 const uint32_t nib =
@@ -1110,7 +1128,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = __ffma2_rn(v[i], w2, acc[i]);
             }
-            __syncthreads();   // buffer s2 & 1 is reloaded two stages on
+            __syncthreads();   // buffer s2 % kThetaBufs is reloaded kThetaBufs stages on
         }
         const int tile = t0 + sub;
         if (tile < S.m_tiles) {
@@ -1427,7 +1445,8 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 }
 
 template <int NS, int GP>
-cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int max_m_keys,
+cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int total_heads,
+                      int max_m_keys,
                       const FetchJob *fetch, int n_fetch, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
 {
@@ -1448,12 +1467,16 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, 
         // exact-path flags)
         static int threshold_smem_set[64];
         auto kern = threshold_kernel<NS, GP>;
-        const size_t dyn = 2 * kThetaStageBytes + (size_t)max_m_keys * sizeof(uint32_t);
+        const size_t dyn = kThetaBufs * kThetaStageBytes + (size_t)max_m_keys * sizeof(uint32_t);
         if ((e = ensure_smem(threshold_smem_set, kern,
-                             2 * kThetaStageBytes + (size_t)kSampleMaxKeys * sizeof(uint32_t))) !=
+                             kThetaBufs * kThetaStageBytes +
+                                 (size_t)kSampleMaxKeys * sizeof(uint32_t))) !=
             cudaSuccess)
             return note_error(e, "threshold set-up");
-        kern<<<total_queries, kSelThreads, dyn, stream>>>(bt, force ? 1u : 0u);
+        // one CTA per query, then (unless the exact path is forced) one per
+        // KV head building its tables
+        const int ctas = total_queries + (force ? 0 : total_heads);
+        kern<<<ctas, kSelThreads, dyn, stream>>>(bt, force ? 1u : 0u, total_queries);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "threshold launch");
         ++launches;
     }
@@ -1509,7 +1532,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, queries = 0, max_m = 0, n_fetch = 0;
+    int groups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
     FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
@@ -1548,18 +1571,20 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.exact_only = z.exact_only;
         D.group_begin = groups;
         D.q_begin = queries;
+        D.head_begin = heads;
+        heads += ix.n_kv_heads;
         groups += D.H * D.col_groups;
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, max_m, fetch, n_fetch, flags,
+    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
-    return run_batch<NS, 8>(bt, groups, queries, max_m, fetch, n_fetch, flags,
+    return run_batch<NS, 8>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
                                            stream, hook);
 }
 
