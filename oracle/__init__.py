@@ -61,6 +61,7 @@ def _load():
             "fo_exact_scores": ([P, P, I, I, P], None),
             "fo_topk": ([P, I, I, P, P], ctypes.c_int),
             "fo_attention": ([P, P, I, I, P, P, I, ctypes.c_double, P], ctypes.c_int),
+            "fo_merge_topk": ([P, P, P, I, I, I, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -323,3 +324,18 @@ def attention_error(o: np.ndarray, o_exact: np.ndarray) -> float:
     o = np.asarray(o, np.float64)
     o_exact = np.asarray(o_exact, np.float64)
     return float(np.linalg.norm(o - o_exact) / np.linalg.norm(o_exact))
+
+
+# ------------------------------------------------------------ sharded keys
+def merge_topk(idx, score, offset, k: int):
+    """Exact top-k over S shard lists (idx int32 [S][k_s] local, score [S][k_s],
+    offset [S]): -> (global idx ascending [k], scores [k])."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    score = np.ascontiguousarray(score, np.float64)
+    offset = np.ascontiguousarray(offset, np.int64)
+    S, k_s = idx.shape
+    out_i = np.empty(k, np.int32)
+    out_s = np.empty(k, np.float64)
+    _check(_load().fo_merge_topk(_p(idx), _p(score), _p(offset), S, k_s, int(k), _p(out_i),
+                                 _p(out_s)), "merge_topk")
+    return out_i, out_s

@@ -511,3 +511,42 @@ int fo_attention(const float *keys_h, const float *values_h, int64_t n, int64_t 
     free(logit);
     return FO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* One KV head's keys split across devices: merging the shards' top-k.  */
+/* ------------------------------------------------------------------ */
+
+/* Exact top-k of the union of S shard lists of one query: shard s holds
+ * keys [offset_s, offset_s + n_s) and lists k_s of them (local index,
+ * score).  Keys rank by (score descending, global index ascending), the
+ * order the single-device top-k uses, so when each shard list is that
+ * shard's top-k the merge is the top-k of all keys.  out_idx receives the k
+ * global indices in ascending order, out_score their scores.
+ * idx, score: [S][k_s]; offset: [S]. */
+int fo_merge_topk(const int32_t *idx, const double *score, const int64_t *offset, int64_t S,
+                  int64_t k_s, int64_t k, int32_t *out_idx, double *out_score)
+{
+    const int64_t m = S * k_s;
+    if (S < 1 || k_s < 1 || k < 1 || k > m) return FO_ERR_ARG;
+    fo_score_item *items = (fo_score_item *)malloc((size_t)m * sizeof *items);
+    if (!items) return FO_ERR_ARG;
+    for (int64_t s = 0; s < S; ++s)
+        for (int64_t i = 0; i < k_s; ++i) {
+            items[s * k_s + i].s = score[s * k_s + i];
+            items[s * k_s + i].j = offset[s] + idx[s * k_s + i];
+        }
+    qsort(items, (size_t)m, sizeof *items, fo_score_cmp);
+    /* the k best, then ascending global index (insertion sort: k is small) */
+    for (int64_t i = 1; i < k; ++i) {
+        fo_score_item x = items[i];
+        int64_t p = i - 1;
+        while (p >= 0 && items[p].j > x.j) { items[p + 1] = items[p]; --p; }
+        items[p + 1] = x;
+    }
+    for (int64_t i = 0; i < k; ++i) {
+        out_idx[i] = (int32_t)items[i].j;
+        out_score[i] = items[i].s;
+    }
+    free(items);
+    return FO_OK;
+}

@@ -37,6 +37,9 @@ MUTATIONS = {
     "marginal_gain_ignores_depth": ("const float gain = w[c] * (1.0f / (float)(1 << (2 * t[c])));",
                                     "const float gain = w[c];"),
     "marginal_gain_halves": ("(float)(1 << (2 * t[c]))", "(float)(1 << t[c])"),
+    "merge_ignores_offset": ("items[s * k_s + i].j = offset[s] + idx[s * k_s + i];",
+                             "items[s * k_s + i].j = idx[s * k_s + i];"),
+    "merge_output_not_index_ordered": ("while (p >= 0 && items[p].j > x.j)", "while (0)"),
     "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
                                "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
 }
@@ -60,6 +63,7 @@ PIN_TESTS = [
     pins.test_attention_special_cases,
     pins.test_marginal_plan_spreads_uniform_importance_round_robin,
     pins.test_marginal_plan_hand_worked,
+    lambda: pins.test_merging_shard_topks_is_the_topk_of_all_keys(3, 999, 64),
 ]
 
 

@@ -494,3 +494,27 @@ def test_marginal_plan_hand_worked():
         [[1, 0], [2, 0], [3, 0], [3, 1], [4, 1]]
     # water-filling instead fills channel 0 to 4 bits before channel 1 gets any
     assert list(oracle.plan_greedy(w, 4)) == [4, 0]
+
+
+# ------------------------------------------------------------ sharded keys
+@pytest.mark.parametrize("S,n,k", [(2, 1000, 50), (3, 999, 64), (4, 4096, 300), (5, 60, 12)])
+def test_merging_shard_topks_is_the_topk_of_all_keys(S, n, k):
+    """Split the keys into S ranges, take each range's top-k, merge: the
+    result is the top-k of all keys (indices ascending), ties included."""
+    rng = np.random.default_rng(S * n + k)
+    s = np.round(rng.standard_normal(n), 1)          # many exact ties
+    cuts = np.sort(rng.choice(np.arange(1, n), S - 1, replace=False))
+    bounds = [0, *cuts.tolist(), n]
+    k_s = max(min(k, b - a) for a, b in zip(bounds, bounds[1:]))
+    idx = np.zeros((S, k_s), np.int32)
+    sc = np.full((S, k_s), -np.inf)
+    for r, (a, b) in enumerate(zip(bounds, bounds[1:])):
+        kk = min(k, b - a)
+        li, ls = oracle.topk(s[a:b], kk)
+        idx[r, :kk], sc[r, :kk] = li, ls
+        idx[r, kk:] = 0                                   # padding rows never win
+    gi, gs = oracle.merge_topk(idx, sc, np.array(bounds[:-1]), k)
+    ref_i, _ = oracle.topk(s, k)
+    assert np.array_equal(gi, np.sort(ref_i))
+    assert np.all(np.diff(gi) > 0)
+    np.testing.assert_array_equal(gs, s[gi])
