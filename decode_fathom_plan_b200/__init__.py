@@ -39,6 +39,7 @@ EXPORTED = (
     "fathom_last_device_status", "fathom_launch_count", "fathom_profile_read",
     "fathom_scan_topk_static", "fathom_link_probe", "fathom_append_keys",
     "fathom_sparse_attention_workspace_bytes", "fathom_sparse_attention", "fathom_plan_marginal",
+    "fathom_merge_topk",
 )
 
 
@@ -86,6 +87,7 @@ def load_library(path: str = LIB_PATH):
         "fathom_plan": ([IX, P, P, P, P, P, P], ctypes.c_int),
         "fathom_fixed_plan": ([IX, P, I32, P, P, P, P], ctypes.c_int),
         "fathom_plan_marginal": ([IX, P, P, P, P, P, P], ctypes.c_int),
+        "fathom_merge_topk": ([P, P, P, I32, I32, I32, I32, P, P, P], ctypes.c_int),
         "fathom_scan_workspace_bytes": ([IX, I32], SZ),
         "fathom_scan_topk": ([IX, P, P, P, I32, P, P, P, SZ, U32, P], ctypes.c_int),
         "fathom_scan_topk_static": ([IX, P, P, P, I32, P, P, U32, P], ctypes.c_int),
@@ -240,6 +242,17 @@ def fathom_sparse_attention(keys, values, n_kv_heads: int, group: int, head_dim:
         _ptr(keys), _ptr(values), int(n_kv_heads), int(group), int(head_dim), int(n_keys),
         _ptr(q_bf16), _ptr(idx), int(k), float(softmax_scale), _ptr(out), _ptr(workspace),
         ws_bytes, _stream(stream)), "fathom_sparse_attention")
+
+
+def fathom_merge_topk(shard_idx, shard_score, shard_offset, k: int, out_idx, out_score,
+                      stream=None):
+    """Exact top-k over S shard lists ([S][Q][k_shard] device tensors) of key
+    ranges starting at shard_offset (S ints, ascending)."""
+    S, Q, k_s = shard_idx.shape
+    offs = (ctypes.c_int64 * S)(*[int(o) for o in shard_offset])
+    _check(load_library().fathom_merge_topk(_ptr(shard_idx), _ptr(shard_score), offs, S, Q, k_s,
+                                            int(k), _ptr(out_idx), _ptr(out_score),
+                                            _stream(stream)), "fathom_merge_topk")
 
 
 def fathom_last_device_status(stream=None) -> int:

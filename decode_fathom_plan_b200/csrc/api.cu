@@ -358,6 +358,30 @@ fathom_status fathom_profile_read(double *scan_kernel_ms, uint64_t *scan_kernel_
     return st;
 }
 
+fathom_status fathom_merge_topk(const int32_t *shard_idx, const float *shard_score,
+                                const int64_t *shard_offset, int32_t n_shards, int32_t n_queries,
+                                int32_t k_shard, int32_t k, int32_t *out_idx, float *out_score,
+                                cudaStream_t stream)
+{
+    if (!shard_idx || !shard_score || !shard_offset || !out_idx || !out_score)
+        return FATHOM_ERR_INVALID_ARG;
+    if (n_shards < 1 || n_shards > kMaxMergeShards || n_queries < 1 || k_shard < 1)
+        return FATHOM_ERR_INVALID_ARG;
+    if ((long long)n_shards * k_shard > kMaxMergeCandidates) return FATHOM_ERR_INVALID_ARG;
+    if (k < 1 || k > kMaxK || (long long)k > (long long)n_shards * k_shard)
+        return FATHOM_ERR_INVALID_ARG;
+    MergeOffsets off{};
+    for (int s = 0; s < n_shards; ++s) {
+        // ascending shard ranges, each holding at least its k_shard listed keys
+        if (shard_offset[s] < 0 || (s > 0 && shard_offset[s] < shard_offset[s - 1] + k_shard))
+            return FATHOM_ERR_INVALID_ARG;
+        off.offset[s] = shard_offset[s];
+    }
+    if (shard_offset[n_shards - 1] + k_shard > (1ll << 31)) return FATHOM_ERR_INVALID_ARG;
+    return cuda_status(launch_merge(shard_idx, shard_score, off, n_shards, n_queries, k_shard, k,
+                                    out_idx, out_score, stream));
+}
+
 size_t fathom_sparse_attention_workspace_bytes(int32_t n_queries, int32_t head_dim, int32_t k)
 {
     return attention_bytes(n_queries, head_dim, k);

@@ -58,6 +58,17 @@ cudaError_t launch_attention(const float *keys, const float *values, int H, int 
                              const uint16_t *q_bf16, const int32_t *idx, int k, float scale,
                              float *out, float *part, cudaStream_t stream);
 
+// ---- merge.cu
+constexpr int kMaxMergeShards = 64;
+constexpr int kMaxMergeCandidates = 16384;   // S * k_s per query (shared memory)
+struct MergeOffsets {
+    long long offset[kMaxMergeShards];       // first global key of each shard
+};
+size_t merge_smem_bytes(int S, int k_s);
+cudaError_t launch_merge(const int32_t *idx, const float *score, const MergeOffsets &off, int S,
+                         int Q, int k_s, int k, int32_t *out_idx, float *out_score,
+                         cudaStream_t stream);
+
 // ---- scan.cu
 struct ScanSessionArgs {
     const fathom_index *ix;

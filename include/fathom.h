@@ -259,6 +259,31 @@ fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_s
                                        uint32_t flags, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
+/* One KV head's keys split across devices.                               */
+/* ---------------------------------------------------------------------- */
+
+/* Exact top-k over the shards of a key range (explainer, 解决什么真问题:
+ * each decode step keeps the top-k of all keys).  Shard s holds the keys
+ * [shard_offset[s], shard_offset[s+1]) of every KV head and returned its
+ * top-k_shard per query (e.g. from fathom_scan_topk on an index of that
+ * range): shard_idx int32 [S][Q][k_shard] local key indices in ascending
+ * order, shard_score float32 [S][Q][k_shard] (device pointers, e.g. one
+ * all-gathered buffer).  Keys rank by (score descending, global index
+ * ascending), the order of the single-device top-k, so the result is the
+ * top-k of all the shards' keys: out_idx int32 [Q][k] global indices in
+ * ascending order, out_score float32 [Q][k].  Shards that are word ranges
+ * of one packed index (same mn, scale, sigma2) score each key exactly as
+ * the whole index does, and the merge reproduces the single-device output.
+ * shard_offset: host array of S ascending key offsets.  1 <= S <= 64,
+ * S*k_shard <= 16384, 1 <= k <= min(S*k_shard, 4096).  A negative index or
+ * non-finite score in the lists sets FATHOM_ERR_INVALID_ARG in the device
+ * status. */
+fathom_status fathom_merge_topk(const int32_t *shard_idx, const float *shard_score,
+                                const int64_t *shard_offset, int32_t n_shards, int32_t n_queries,
+                                int32_t k_shard, int32_t k, int32_t *out_idx, float *out_score,
+                                cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* After the scan: attention over the selected keys.                      */
 /* ---------------------------------------------------------------------- */
 

@@ -144,3 +144,15 @@ def test_sparse_attention_sizes_and_argument_checks(lib):
     assert call(args(G=9)) == F
     assert call(args(idx=None)) == F
     assert call(args(scale=float("nan"))) == F
+
+
+def test_merge_rejects_bad_arguments_before_launching(lib):
+    fake = 0x1000
+    F = fp.FATHOM_ERR_INVALID_ARG
+    merge = lib.fathom_merge_topk
+    offs = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    assert merge(fake, fake, offs(0, 10), 2, 4, 64, 64, fake, fake, None) == F      # overlapping ranges
+    assert merge(fake, fake, offs(100, 0), 2, 4, 64, 64, fake, fake, None) == F     # not ascending
+    assert merge(fake, fake, offs(0, 100), 2, 4, 64, 129, fake, fake, None) == F    # k > S*k_s
+    assert merge(fake, fake, offs(0, 10000), 2, 4, 9000, 64, fake, fake, None) == F  # too many candidates
+    assert merge(None, fake, offs(0, 100), 2, 4, 64, 64, fake, fake, None) == F
