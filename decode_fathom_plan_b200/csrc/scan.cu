@@ -67,6 +67,7 @@ namespace {
 constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-word chunk
 constexpr int kMainStages = 3;
 constexpr int kMaskOrderValues = 16;   // reader sets of up to 4 query heads
+constexpr int kMinChunkGroups = 8;     // smallest chunk of the main scan: 32 words
 
 struct SessionDesc {
     const uint32_t *planes;      // device address of [H][d][4][n_words]
@@ -82,7 +83,8 @@ struct SessionDesc {
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
-    int group_begin, q_begin, head_begin;
+    int chunks, chunk_begin;   // main-scan chunks per KV head, first chunk's CTA
+    int q_begin, head_begin;
 };
 
 template <int NS>
@@ -578,11 +580,11 @@ __device__ __forceinline__ float score_of(const float2 (&a)[4], int m, float bia
 }
 
 template <int NS>
-__device__ __forceinline__ int find_session_by_group(const Batch<NS> &b, int g)
+__device__ __forceinline__ int find_session_by_chunk(const Batch<NS> &b, int ci)
 {
     int si = 0;
     for (int s = 1; s < b.n_sessions; ++s)
-        if (b.s[s].group_begin <= g) si = s;
+        if (b.s[s].chunk_begin <= ci) si = s;
     return si;
 }
 
@@ -611,7 +613,7 @@ __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
 // >= theta to their query's candidate buffer.
 template <int NS, int GP, int STAGES>
 __global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
-scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
+scan_kernel(const __grid_constant__ Batch<NS> b)
 {
     __shared__ ScanMeta<GP> sm;
     __shared__ uint32_t s_theta[GP];
@@ -622,34 +624,25 @@ scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
     const int G = b.G;
     const int col = threadIdx.x >> 2, r = threadIdx.x & 3, lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    int g = blockIdx.x * per_cta;
-    const int g_end = min(total_groups, g + per_cta);
-    int cur_si = -1, cur_h = -1;
-    while (g < g_end) {
-        const int si = find_session_by_group(b, g);
+    {
+        // this CTA's chunk: chunk c of the KV head's S.chunks equal parts of
+        // its column groups (at most 16 groups = 64 words each)
+        const int si = find_session_by_chunk(b, (int)blockIdx.x);
         const SessionDesc &S = b.s[si];
-        const int local = g - S.group_begin;
-        const int h = local / S.col_groups;
-        const int gi = local - h * S.col_groups;
-        // this chunk: balanced split of what is left of the range in this
-        // head, at most 16 groups
-        const int avail = min(g_end - g, S.col_groups - gi);
-        const int col_lo = gi * 4;
-        const int pieces = (avail + kTileGroups - 1) / kTileGroups;
-        const int lim = (avail + pieces - 1) / pieces;
-        const int width = lim * 4;                     // plane words owned by this chunk
+        const int local = (int)blockIdx.x - S.chunk_begin;
+        const int h = local / S.chunks;
+        const int c = local - h * S.chunks;
+        const int g0 = (int)((long long)c * S.col_groups / S.chunks);
+        const int g1 = (int)((long long)(c + 1) * S.col_groups / S.chunks);
+        const int col_lo = g0 * 4;
+        const int width = (g1 - g0) * 4;               // plane words owned by this chunk
         const int col_hi = min(S.n_cols, col_lo + width);
         const int q0 = h * G;
-        if (si != cur_si || h != cur_h) {
-            __syncthreads();   // the previous chunk's epilogue may still read sm
-            if (threadIdx.x < GP)
-                s_theta[threadIdx.x] = (threadIdx.x < G)
-                                           ? S.qstate[(q0 + threadIdx.x) * kQueryStateWords + 0]
-                                           : 0xFFFFFFFFu;
-            load_head<GP>(sm, S.tables, h);
-            cur_si = si;
-            cur_h = h;
-        }
+        if (threadIdx.x < GP)
+            s_theta[threadIdx.x] = (threadIdx.x < G)
+                                       ? S.qstate[(q0 + threadIdx.x) * kQueryStateWords + 0]
+                                       : 0xFFFFFFFFu;
+        load_head<GP>(sm, S.tables, h);
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
 
@@ -718,7 +711,6 @@ scan_kernel(const __grid_constant__ Batch<NS> b, int total_groups, int per_cta)
                 }
             }
         }
-        g += lim;
     }
 }
 
@@ -1282,6 +1274,21 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     return L;
 }
 
+// Multiprocessors of the current device (cached per device).
+inline int sm_count()
+{
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 // Raise a kernel's dynamic shared-memory limit to its largest possible need,
 // once per device.  `done` must belong to that kernel alone.
 template <class Kernel>
@@ -1338,7 +1345,7 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 }
 
 template <int NS, int GP>
-cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, int total_heads,
+cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, int total_heads,
                       int max_m_keys,
                       const FetchJob *fetch, int n_fetch, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
@@ -1373,16 +1380,14 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_groups, int total_queries, 
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "threshold launch");
         ++launches;
     }
-    if (!force && total_groups > 0) {
+    if (!force && total_chunks > 0) {
         const bool timed = hook && hook->enabled && n_fetch == 0;
-        const int per_cta = kTileGroups;   // one 64-word chunk per CTA
-        const int ctas = (total_groups + per_cta - 1) / per_cta;
         static int main_smem_set[64];
         auto kern = scan_kernel<NS, GP, kMainStages>;
         const size_t dyn = kMainStages * kStageBytes;
         if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
         if (timed) record_timing_event(hook->begin, stream);
-        kern<<<ctas, kScanThreads, dyn, stream>>>(bt, total_groups, per_cta);
+        kern<<<total_chunks, kScanThreads, dyn, stream>>>(bt);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
         if (timed) {
             record_timing_event(hook->end, stream);
@@ -1462,13 +1467,32 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.m_keys = z.m_keys;
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
-        D.group_begin = groups;
+        D.chunks = (D.col_groups + kTileGroups - 1) / kTileGroups;   // chunks of <= 64 words
         D.q_begin = queries;
         D.head_begin = heads;
         heads += ix.n_kv_heads;
-        groups += D.H * D.col_groups;
+        groups += D.H * D.chunks;
         queries += D.H * bt.G;
         max_m = std::max(max_m, z.m_keys);
+    }
+    // Below one wave of CTA slots, cut the heads into more, equal chunks (at
+    // least kMinChunkGroups groups each) so the grid fills the slots evenly;
+    // a chunk never spans two heads.
+    const int slots = sm_count() * ((bt.G > 4) ? 2 : 4);
+    if (groups < slots) {
+        const double grow = (double)slots / (double)groups;
+        groups = 0;
+        for (int s = 0; s < n_sessions; ++s) {
+            SessionDesc &D = bt.s[s];
+            const int most = std::max(1, D.col_groups / kMinChunkGroups);
+            D.chunks = std::max(D.chunks, std::min(most, (int)(D.chunks * grow)));
+            groups += D.H * D.chunks;
+        }
+    }
+    groups = 0;
+    for (int s = 0; s < n_sessions; ++s) {
+        bt.s[s].chunk_begin = groups;
+        groups += bt.s[s].H * bt.s[s].chunks;
     }
     const int G = bt.G;
     if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
