@@ -16,47 +16,10 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "plan_warp.cuh"
 
 namespace fathom {
 namespace {
-
-// Sort N composite keys held E = N/32 per lane (element e = lane*E + i)
-// in descending order: bitonic network, strides below E inside the lane,
-// the rest by warp shuffles.
-template <int E>
-__device__ __forceinline__ void warp_sort_desc(unsigned long long (&key)[E])
-{
-    const int lane = threadIdx.x & 31;
-    constexpr int N = 32 * E;
-#pragma unroll
-    for (int size = 2; size <= N; size <<= 1) {
-#pragma unroll
-        for (int j = size >> 1; j > 0; j >>= 1) {
-            if (j < E) {
-#pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    if ((i & j) == 0) {
-                        const int e = lane * E + i;
-                        const bool desc = (e & size) == 0;
-                        const unsigned long long a = key[i], b = key[i ^ j];
-                        if ((a < b) == desc) {
-                            key[i] = b;
-                            key[i ^ j] = a;
-                        }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, key[i], j / E);
-                    const int e = lane * E + i;
-                    const bool desc = (e & size) == 0, low = (e & j) == 0;
-                    key[i] = (low == desc) ? max(key[i], other) : min(key[i], other);
-                }
-            }
-        }
-    }
-}
 
 // One CTA per KV head, one warp per query head.  Each warp sorts its
 // query's channels by (key descending, channel ascending) with a warp
@@ -74,48 +37,13 @@ plan_kernel(const uint16_t *__restrict__ q, const int32_t *__restrict__ budget, 
     const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned long long plane_bytes = 4ull * (unsigned long long)n_words;
     const int qi = h * G + g;
-    unsigned long long key[E];
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int c = lane * E + i;
-        key[i] = 0ull;                                   // padding sorts last
-        if (c < d) {
-            const float qf = bf16_to_float(q[(size_t)qi * d + c]);
-            float k;
-            if (kFixed) {
-                k = fabsf(qf);
-                bad |= !isfinite(qf);
-            } else {
-                k = __fmul_rn(__fmul_rn(qf, qf), sigma2[h * d + c]);
-                bad |= !isfinite(k);
-            }
-            key[i] = ((unsigned long long)order_key(k) << 32) | (0xFFFFFFFFu - (uint32_t)c);
-        }
-    }
-    bad = __any_sync(0xFFFFFFFFu, bad);
-    int B = 0;
-    if (!kFixed) {
-        B = budget[qi];
-        if (B < 0 || B > kBits * d) {
-            if (lane == 0) set_status(status, FATHOM_ERR_INVALID_ARG);
-            B = 0;
-        }
-    }
-    if (bad && lane == 0) set_status(status, FATHOM_ERR_NONFINITE);
-    warp_sort_desc<E>(key);
+    warp_plan<kFixed, E>(q + (size_t)qi * d, sigma2 + h * d, d, kFixed ? 0 : budget[qi], fixed_r,
+                         tt[g], status);
+    __syncwarp();
     unsigned long long my_bytes = 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int rank = lane * E + i;
-        const uint32_t c = 0xFFFFFFFFu - (uint32_t)(key[i] & 0xFFFFFFFFull);
-        if (key[i] != 0ull && c < (uint32_t)d) {
-            int tc = kFixed ? (rank < fixed_r ? kBits : 0) : min(kBits, max(0, B - kBits * rank));
-            if (bad) tc = 0;
-            tt[g][c] = (uint8_t)tc;
-            t[(size_t)qi * d + c] = (uint8_t)tc;
-            my_bytes += (unsigned long long)tc * plane_bytes;
-        }
+    for (int c = lane; c < d; c += 32) {
+        t[(size_t)qi * d + c] = tt[g][c];
+        my_bytes += (unsigned long long)tt[g][c] * plane_bytes;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) my_bytes += __shfl_xor_sync(0xFFFFFFFFu, my_bytes, off);
