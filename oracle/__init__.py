@@ -44,20 +44,20 @@ def _load():
         lib = ctypes.CDLL(_LIB_PATH)
         P, I = ctypes.c_void_p, ctypes.c_int64
         sig = {
-            "fo_quantize": ([P, I, I, I, P, P, P], ctypes.c_int),
-            "fo_pack_planes": ([P, I, I, I, I, P], ctypes.c_int),
-            "fo_unpack_planes": ([P, I, I, I, I, P], ctypes.c_int),
-            "fo_append": ([P, I, I, I, I, I, P, P, P, P, P, P, P], ctypes.c_int),
+            "fo_quantize": ([P, I, I, I, I, P, P, P], ctypes.c_int),
+            "fo_pack_planes": ([P, I, I, I, I, I, P], ctypes.c_int),
+            "fo_unpack_planes": ([P, I, I, I, I, I, P], ctypes.c_int),
+            "fo_append": ([P, I, I, I, I, I, I, P, P, P, P, P, P, P], ctypes.c_int),
             "fo_channel_stats": ([P, I, I, I, P, P, P, P], ctypes.c_int),
             "fo_importance": ([P, P, I, P], ctypes.c_int),
-            "fo_plan_greedy": ([P, I, I, P], ctypes.c_int),
-            "fo_plan_marginal": ([P, I, I, P], ctypes.c_int),
-            "fo_fixed_plan": ([P, I, I, P], ctypes.c_int),
+            "fo_plan_greedy": ([P, I, I, I, P], ctypes.c_int),
+            "fo_plan_marginal": ([P, I, I, I, P], ctypes.c_int),
+            "fo_fixed_plan": ([P, I, I, I, P], ctypes.c_int),
             "fo_union": ([P, I, I, P], None),
             "fo_plan_bytes": ([P, I, I], ctypes.c_uint64),
-            "fo_score_planes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
-            "fo_score_codes": ([P, P, P, P, P, I, I, P], ctypes.c_int),
-            "fo_score_abs_planes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
+            "fo_score_planes": ([P, P, P, P, P, I, I, I, I, P], ctypes.c_int),
+            "fo_score_codes": ([P, P, P, P, P, I, I, I, P], ctypes.c_int),
+            "fo_score_abs_planes": ([P, P, P, P, P, I, I, I, I, P], ctypes.c_int),
             "fo_exact_scores": ([P, P, I, I, P], None),
             "fo_topk": ([P, I, I, P, P], ctypes.c_int),
             "fo_attention": ([P, P, I, I, P, P, I, ctypes.c_double, P], ctypes.c_int),
@@ -87,32 +87,37 @@ def n_words_for(n: int) -> int:
 
 
 # ---------------------------------------------------------------- storage side
-def quantize(keys: np.ndarray):
-    """keys float32 [H][n][d] -> (mn [H][d], scale [H][d], codes uint8 [H][d][n])."""
+def quantize(keys: np.ndarray, bits: int = 4):
+    """keys float32 [H][n][d] -> (mn [H][d], scale [H][d], codes uint8 [H][d][n]),
+    codes of `bits` bits (4: the 4-bit K cache; 8: the 8-plane variant)."""
     keys = np.ascontiguousarray(keys, dtype=np.float32)
     H, n, d = keys.shape
     mn = np.empty((H, d), np.float32)
     scale = np.empty((H, d), np.float32)
     codes = np.empty((H, d, n), np.uint8)
-    _check(_load().fo_quantize(_p(keys), H, n, d, _p(mn), _p(scale), _p(codes)), "quantize")
+    _check(_load().fo_quantize(_p(keys), H, n, d, int(bits), _p(mn), _p(scale), _p(codes)),
+           "quantize")
     return mn, scale, codes
 
 
-def pack_planes(codes: np.ndarray, n_words: Optional[int] = None) -> np.ndarray:
-    """codes uint8 [H][d][n] -> planes uint32 [H][d][4][n_words]."""
+def pack_planes(codes: np.ndarray, n_words: Optional[int] = None, bits: int = 4) -> np.ndarray:
+    """codes uint8 [H][d][n] -> planes uint32 [H][d][bits][n_words]."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     H, d, n = codes.shape
     n_words = n_words_for(n) if n_words is None else n_words
-    planes = np.empty((H, d, 4, n_words), np.uint32)
-    _check(_load().fo_pack_planes(_p(codes), H, n, d, n_words, _p(planes)), "pack_planes")
+    planes = np.empty((H, d, int(bits), n_words), np.uint32)
+    _check(_load().fo_pack_planes(_p(codes), H, n, d, int(bits), n_words, _p(planes)),
+           "pack_planes")
     return planes
 
 
 def unpack_planes(planes: np.ndarray, n: int) -> np.ndarray:
+    """planes uint32 [H][d][bits][n_words] -> codes uint8 [H][d][n]."""
     planes = np.ascontiguousarray(planes, dtype=np.uint32)
-    H, d, _, n_words = planes.shape
+    H, d, bits, n_words = planes.shape
     codes = np.empty((H, d, n), np.uint8)
-    _check(_load().fo_unpack_planes(_p(planes), H, n, d, n_words, _p(codes)), "unpack_planes")
+    _check(_load().fo_unpack_planes(_p(planes), H, n, d, bits, n_words, _p(codes)),
+           "unpack_planes")
     return codes
 
 
@@ -123,12 +128,12 @@ def append(index: Dict[str, np.ndarray], keys: np.ndarray, clamped=None):
     keys = np.ascontiguousarray(keys, dtype=np.float32)
     H, m, d = keys.shape
     n = index["n"]
-    n_words = index["planes"].shape[-1]
+    bits, n_words = index["planes"].shape[-2:]
     for name in ("planes", "s1", "s2", "sigma2"):
         assert index[name].flags["C_CONTIGUOUS"]
     if clamped is not None:
         assert clamped.dtype == np.uint32 and clamped.flags["C_CONTIGUOUS"]
-    _check(_load().fo_append(_p(keys), H, n, m, d, n_words, _p(index["mn"]), _p(index["scale"]),
+    _check(_load().fo_append(_p(keys), H, n, m, d, bits, n_words, _p(index["mn"]), _p(index["scale"]),
                              _p(index["planes"]), _p(index["s1"]), _p(index["s2"]),
                              _p(index["sigma2"]), None if clamped is None else _p(clamped)),
            "append")
@@ -160,25 +165,27 @@ def importance(q_bf16: np.ndarray, sigma2: np.ndarray) -> np.ndarray:
     return w
 
 
-def plan_greedy(w: np.ndarray, B: int) -> np.ndarray:
+def plan_greedy(w: np.ndarray, B: int, bits: int = 4) -> np.ndarray:
+    """Reverse water-filling with at most `bits` bits per channel."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     t = np.empty(w.shape[0], np.uint8)
-    _check(_load().fo_plan_greedy(_p(w), w.shape[0], int(B), _p(t)), "plan_greedy")
+    _check(_load().fo_plan_greedy(_p(w), w.shape[0], int(B), int(bits), _p(t)), "plan_greedy")
     return t
 
 
-def plan_marginal(w: np.ndarray, B: int) -> np.ndarray:
+def plan_marginal(w: np.ndarray, B: int, bits: int = 4) -> np.ndarray:
     """Marginal-gain plan: bits one at a time to the largest w_c * 4^-t_c."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     t = np.empty(w.shape[0], np.uint8)
-    _check(_load().fo_plan_marginal(_p(w), w.shape[0], int(B), _p(t)), "plan_marginal")
+    _check(_load().fo_plan_marginal(_p(w), w.shape[0], int(B), int(bits), _p(t)),
+           "plan_marginal")
     return t
 
 
-def fixed_plan(q_bf16: np.ndarray, r: int) -> np.ndarray:
+def fixed_plan(q_bf16: np.ndarray, r: int, bits: int = 4) -> np.ndarray:
     q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
     t = np.empty(q.shape[0], np.uint8)
-    _check(_load().fo_fixed_plan(_p(q), q.shape[0], int(r), _p(t)), "fixed_plan")
+    _check(_load().fo_fixed_plan(_p(q), q.shape[0], int(r), int(bits), _p(t)), "fixed_plan")
     return t
 
 
@@ -197,30 +204,30 @@ def plan_bytes(t: np.ndarray, n_words: int) -> int:
 
 def score_planes(planes_h, mn_h, scale_h, q_bf16, t, n: int) -> np.ndarray:
     planes_h = np.ascontiguousarray(planes_h, dtype=np.uint32)
-    d, _, n_words = planes_h.shape
+    d, bits, n_words = planes_h.shape
     mn_h = np.ascontiguousarray(mn_h, np.float32)
     scale_h = np.ascontiguousarray(scale_h, np.float32)
     q = np.ascontiguousarray(q_bf16, np.uint16)
     t = np.ascontiguousarray(t, np.uint8)
     s = np.empty(n, np.float64)
     _check(_load().fo_score_planes(_p(planes_h), _p(mn_h), _p(scale_h), _p(q), _p(t),
-                                   d, n, n_words, _p(s)), "score_planes")
+                                   d, bits, n, n_words, _p(s)), "score_planes")
     return s
 
 
 def score_abs_planes(planes_h, mn_h, scale_h, q_bf16, t, n: int) -> np.ndarray:
     planes_h = np.ascontiguousarray(planes_h, dtype=np.uint32)
-    d, _, n_words = planes_h.shape
+    d, bits, n_words = planes_h.shape
     a = np.empty(n, np.float64)
     _check(_load().fo_score_abs_planes(
         _p(planes_h), _p(np.ascontiguousarray(mn_h, np.float32)),
         _p(np.ascontiguousarray(scale_h, np.float32)),
         _p(np.ascontiguousarray(q_bf16, np.uint16)), _p(np.ascontiguousarray(t, np.uint8)),
-        d, n, n_words, _p(a)), "score_abs_planes")
+        d, bits, n, n_words, _p(a)), "score_abs_planes")
     return a
 
 
-def score_codes(codes_h, mn_h, scale_h, q_bf16, t) -> np.ndarray:
+def score_codes(codes_h, mn_h, scale_h, q_bf16, t, bits: int = 4) -> np.ndarray:
     codes_h = np.ascontiguousarray(codes_h, dtype=np.uint8)
     d, n = codes_h.shape
     s = np.empty(n, np.float64)
@@ -228,7 +235,7 @@ def score_codes(codes_h, mn_h, scale_h, q_bf16, t) -> np.ndarray:
         _p(codes_h), _p(np.ascontiguousarray(mn_h, np.float32)),
         _p(np.ascontiguousarray(scale_h, np.float32)),
         _p(np.ascontiguousarray(q_bf16, np.uint16)), _p(np.ascontiguousarray(t, np.uint8)),
-        d, n, _p(s)), "score_codes")
+        d, int(bits), n, _p(s)), "score_codes")
     return s
 
 
@@ -257,31 +264,34 @@ def recall(selected, reference) -> float:
 
 
 # --------------------------------------------------------------- whole pipeline
-def build_index(keys: np.ndarray, capacity: Optional[int] = None) -> Dict[str, np.ndarray]:
+def build_index(keys: np.ndarray, capacity: Optional[int] = None,
+                bits: int = 4) -> Dict[str, np.ndarray]:
     """Storage side for one session: quantise, pack, channel statistics.
-    capacity: keys the planes can hold (for appends); default n."""
-    mn, scale, codes = quantize(keys)
+    capacity: keys the planes can hold (for appends); default n.
+    bits: planes per channel (4, or 8 for an 8-bit K cache)."""
+    mn, scale, codes = quantize(keys, bits)
     n = keys.shape[1]
-    planes = pack_planes(codes, n_words_for(max(n, capacity or n)))
+    planes = pack_planes(codes, n_words_for(max(n, capacity or n)), bits)
     s1, s2, sigma2 = channel_stats(codes, scale)
     return dict(mn=mn, scale=scale, codes=codes, planes=planes, s1=s1, s2=s2,
-                sigma2=sigma2, n=n, n_words=planes.shape[-1])
+                sigma2=sigma2, n=n, n_words=planes.shape[-1], bits=int(bits))
 
 
 def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
                  fixed_r: Optional[int] = None, marginal: bool = False):
     """-> (t uint8 [Q][d], T uint8 [H][d], bytes uint64 [Q+H])."""
     H, d = index["mn"].shape
+    bits = index["planes"].shape[-2]
     Q = H * group
     t = np.empty((Q, d), np.uint8)
     for q in range(Q):
         h = q // group
         if fixed_r is not None:
-            t[q] = fixed_plan(q_bf16[q], fixed_r)
+            t[q] = fixed_plan(q_bf16[q], fixed_r, bits)
         elif marginal:
-            t[q] = plan_marginal(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
+            t[q] = plan_marginal(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]), bits)
         else:
-            t[q] = plan_greedy(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]))
+            t[q] = plan_greedy(importance(q_bf16[q], index["sigma2"][h]), int(budgets[q]), bits)
     T = np.stack([union(t[h * group:(h + 1) * group]) for h in range(H)])
     nb = np.array([plan_bytes(t[q], index["n_words"]) for q in range(Q)]
                   + [plan_bytes(T[h], index["n_words"]) for h in range(H)], np.uint64)

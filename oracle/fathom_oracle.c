@@ -14,20 +14,23 @@
  * Caches", Summary).  Every choice the pages leave open is a stated reading:
  *
  *   quantiser   per (head, channel) asymmetric min/max over all n keys,
- *               scale = (max-min)/15, code = clamp(floor((k-min)/scale+0.5),
- *               0, 15) in float32 round-to-nearest with no fused ops; a
- *               constant channel gets scale 0 and code 0.
+ *               scale = (max-min)/L with L = 2^b - 1 levels for a b-bit K
+ *               cache (b = 4; b = 8 for the 8-plane variant the page's
+ *               部署前必读 item 3 asks for when the upstream K is 8-bit),
+ *               code = clamp(floor((k-min)/scale+0.5), 0, L) in float32
+ *               round-to-nearest with no fused ops; a constant channel
+ *               gets scale 0 and code 0.
  *   planes      bit p of a code (p = 0 least significant, as on the page)
- *               is stored in slot 3-p, so reading slots 0..t-1 reads the
+ *               is stored in slot b-1-p, so reading slots 0..t-1 reads the
  *               t most significant bits ("the first t planes are the t-bit
  *               quantiser" only holds MSB-first).
- *   variance    sigma^2 = population variance of the dequantised 4-bit keys,
+ *   variance    sigma^2 = population variance of the dequantised keys,
  *               from exact integer sums of codes.
  *   importance  w_c = (q_c*q_c)*sigma^2_c in float32, q widened from bf16.
  *   plan        channels in order of (w descending, channel ascending); each
- *               takes min(4, remaining budget) bits until the budget is
+ *               takes min(b, remaining budget) bits until the budget is
  *               spent, so channels of zero importance still take leftovers.
- *   score       reading t bits gives u = code >> (4-t); the key is rebuilt
+ *   score       reading t bits gives u = code >> (b-t); the key is rebuilt
  *               at the middle of that coarse bin and dotted with q in fp64.
  *   top-k       score descending, ties to the lower key index.
  *
@@ -45,19 +48,21 @@
 #define FO_ERR_ARG 1
 #define FO_ERR_NONFINITE 3
 
-#define FO_BITS 4   /* 4-bit K cache (storage side) */
-#define FO_LEVELS 15
+/* Planes per channel: b = 4 for the 4-bit K cache; the oracle takes any
+ * b in 1..8 so that the 8-plane variant is the same code. */
+static int fo_bits_ok(int64_t bits) { return bits >= 1 && bits <= 8; }
 
 /* ------------------------------------------------------------------ */
-/* Storage side: 4-bit quantisation of each channel.                    */
+/* Storage side: b-bit quantisation of each channel.                    */
 /* ------------------------------------------------------------------ */
 
 /* keys: float32 [H][n][d] (token-major, as a K cache holds them).
  * Outputs: mn, scale float32 [H][d]; codes uint8 [H][d][n] (channel-major). */
-int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d,
+int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d, int64_t bits,
                 float *mn, float *scale, uint8_t *codes)
 {
-    if (H <= 0 || n <= 0 || d <= 0) return FO_ERR_ARG;
+    if (H <= 0 || n <= 0 || d <= 0 || !fo_bits_ok(bits)) return FO_ERR_ARG;
+    const int levels = (1 << bits) - 1;
     for (int64_t h = 0; h < H; ++h) {
         const float *kh = keys + h * n * d;
         for (int64_t c = 0; c < d; ++c) {
@@ -75,7 +80,7 @@ int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d,
                 memset(out, 0, (size_t)n);
                 continue;
             }
-            float sc = (hi - lo) / (float)FO_LEVELS;
+            float sc = (hi - lo) / (float)levels;
             scale[h * d + c] = sc;
             for (int64_t j = 0; j < n; ++j) {
                 float diff = kh[j * d + c] - lo;
@@ -84,7 +89,7 @@ int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d,
                 float level = floorf(shifted);
                 int v = (int)level;
                 if (v < 0) v = 0;
-                if (v > FO_LEVELS) v = FO_LEVELS;
+                if (v > levels) v = levels;
                 out[j] = (uint8_t)v;
             }
         }
@@ -92,49 +97,51 @@ int fo_quantize(const float *keys, int64_t H, int64_t n, int64_t d,
     return FO_OK;
 }
 
-/* Channel-major bit planes: planes uint32 [H][d][4][n_words]; slot s holds
- * bit (3-s) of the code; bit i of word w belongs to key 32*w+i; words past
- * the last key are zero.  n_words >= ceil(n/32). */
-int fo_pack_planes(const uint8_t *codes, int64_t H, int64_t n, int64_t d,
+/* Channel-major bit planes: planes uint32 [H][d][b][n_words]; slot s holds
+ * bit (b-1-s) of the code; bit i of word w belongs to key 32*w+i; words
+ * past the last key are zero.  n_words >= ceil(n/32). */
+int fo_pack_planes(const uint8_t *codes, int64_t H, int64_t n, int64_t d, int64_t bits,
                    int64_t n_words, uint32_t *planes)
 {
-    if (n_words * 32 < n) return FO_ERR_ARG;
-    memset(planes, 0, (size_t)(H * d * FO_BITS * n_words) * sizeof(uint32_t));
+    if (n_words * 32 < n || !fo_bits_ok(bits)) return FO_ERR_ARG;
+    memset(planes, 0, (size_t)(H * d * bits * n_words) * sizeof(uint32_t));
     for (int64_t h = 0; h < H; ++h)
         for (int64_t c = 0; c < d; ++c) {
             const uint8_t *cc = codes + (h * d + c) * n;
-            uint32_t *pc = planes + (h * d + c) * FO_BITS * n_words;
+            uint32_t *pc = planes + (h * d + c) * bits * n_words;
             for (int64_t j = 0; j < n; ++j)
-                for (int p = 0; p < FO_BITS; ++p)
+                for (int p = 0; p < bits; ++p)
                     if ((cc[j] >> p) & 1u)
-                        pc[(FO_BITS - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
+                        pc[(bits - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
         }
     return FO_OK;
 }
 
 /* Append m keys per KV head to an index holding n keys: the decode step's
- * new keys enter the 4-bit K cache the explainer's read side scans
+ * new keys enter the b-bit K cache the explainer's read side scans
  * (核心方法 / 存储侧; the cache comes from the serving stack, 适用边界).
  * Reading: the new keys are quantised with the index's existing mn and
  * scale, in the quantiser's own float32 steps, and the level is clamped to
- * 0..15 (a key outside the stored range takes the nearest level); their
+ * 0..2^b-1 (a key outside the stored range takes the nearest level); their
  * bits go to key positions n..n+m-1 of the planes; S1 and S2 grow by the
  * new codes and sigma^2 is recomputed from them with n+m keys.
  * clamped[h][c] (may be NULL) is incremented once per new key whose level
- * fell outside 0..15 (for a constant channel: any key other than mn), the
+ * fell outside 0..2^b-1 (for a constant channel: any key other than mn), the
  * measure of range drift a caller re-quantises on.
- * keys float32 [H][m][d]; planes [H][d][4][n_words], 32*n_words >= n+m,
+ * keys float32 [H][m][d]; planes [H][d][b][n_words], 32*n_words >= n+m,
  * words past key n zero. */
-int fo_append(const float *keys, int64_t H, int64_t n, int64_t m, int64_t d, int64_t n_words,
-              const float *mn, const float *scale, uint32_t *planes, int64_t *s1, int64_t *s2,
-              float *sigma2, uint32_t *clamped)
+int fo_append(const float *keys, int64_t H, int64_t n, int64_t m, int64_t d, int64_t bits,
+              int64_t n_words, const float *mn, const float *scale, uint32_t *planes,
+              int64_t *s1, int64_t *s2, float *sigma2, uint32_t *clamped)
 {
-    if (H <= 0 || n < 0 || m <= 0 || d <= 0 || n_words * 32 < n + m) return FO_ERR_ARG;
+    if (H <= 0 || n < 0 || m <= 0 || d <= 0 || n_words * 32 < n + m || !fo_bits_ok(bits))
+        return FO_ERR_ARG;
+    const int levels = (1 << bits) - 1;
     for (int64_t h = 0; h < H; ++h)
         for (int64_t c = 0; c < d; ++c) {
             const int64_t hc = h * d + c;
             const float lo = mn[hc], sc = scale[hc];
-            uint32_t *pc = planes + hc * FO_BITS * n_words;
+            uint32_t *pc = planes + hc * bits * n_words;
             for (int64_t i = 0; i < m; ++i) {
                 const float x = keys[(h * m + i) * d + c];
                 if (!isfinite(x)) return FO_ERR_NONFINITE;
@@ -148,13 +155,13 @@ int fo_append(const float *keys, int64_t H, int64_t n, int64_t m, int64_t d, int
                     float ratio = diff / sc;
                     float shifted = ratio + 0.5f;
                     float level = floorf(shifted);
-                    out_of_range = level < 0.0f || level > (float)FO_LEVELS;
-                    v = level < 0.0f ? 0 : (level > (float)FO_LEVELS ? FO_LEVELS : (int)level);
+                    out_of_range = level < 0.0f || level > (float)levels;
+                    v = level < 0.0f ? 0 : (level > (float)levels ? levels : (int)level);
                 }
                 const int64_t j = n + i;
-                for (int p = 0; p < FO_BITS; ++p)
+                for (int p = 0; p < bits; ++p)
                     if ((v >> p) & 1)
-                        pc[(FO_BITS - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
+                        pc[(bits - 1 - p) * n_words + j / 32] |= 1u << (j % 32);
                 s1[hc] += v;
                 s2[hc] += (int64_t)v * v;
                 if (clamped && out_of_range) clamped[hc] += 1;
@@ -167,26 +174,26 @@ int fo_append(const float *keys, int64_t H, int64_t n, int64_t m, int64_t d, int
     return FO_OK;
 }
 
-/* Inverse of fo_pack_planes (reads all four slots). */
-int fo_unpack_planes(const uint32_t *planes, int64_t H, int64_t n, int64_t d,
+/* Inverse of fo_pack_planes (reads all b slots). */
+int fo_unpack_planes(const uint32_t *planes, int64_t H, int64_t n, int64_t d, int64_t bits,
                      int64_t n_words, uint8_t *codes)
 {
-    if (n_words * 32 < n) return FO_ERR_ARG;
+    if (n_words * 32 < n || !fo_bits_ok(bits)) return FO_ERR_ARG;
     for (int64_t h = 0; h < H; ++h)
         for (int64_t c = 0; c < d; ++c) {
-            const uint32_t *pc = planes + (h * d + c) * FO_BITS * n_words;
+            const uint32_t *pc = planes + (h * d + c) * bits * n_words;
             uint8_t *cc = codes + (h * d + c) * n;
             for (int64_t j = 0; j < n; ++j) {
                 int v = 0;
-                for (int p = 0; p < FO_BITS; ++p)
-                    v |= (int)((pc[(FO_BITS - 1 - p) * n_words + j / 32] >> (j % 32)) & 1u) << p;
+                for (int p = 0; p < bits; ++p)
+                    v |= (int)((pc[(bits - 1 - p) * n_words + j / 32] >> (j % 32)) & 1u) << p;
                 cc[j] = (uint8_t)v;
             }
         }
     return FO_OK;
 }
 
-/* Per-channel statistics of the stored 4-bit keys: S1 = sum code,
+/* Per-channel statistics of the stored b-bit keys: S1 = sum code,
  * S2 = sum code^2 (exact int64) and the population variance of the
  * dequantised keys mn + scale*code:
  *   sigma^2 = scale^2 * (n*S2 - S1^2) / n^2,
@@ -252,11 +259,11 @@ static int fo_rank_cmp(const void *pa, const void *pb)
 }
 
 /* Reverse water-filling: visit channels from the most important down and
- * give each min(4, remaining) bits; once the budget is gone the rest get 0.
- * B must lie in [0, 4d]. */
-int fo_plan_greedy(const float *w, int64_t d, int64_t B, uint8_t *t)
+ * give each min(b, remaining) bits; once the budget is gone the rest get 0.
+ * B must lie in [0, b*d]. */
+int fo_plan_greedy(const float *w, int64_t d, int64_t B, int64_t bits, uint8_t *t)
 {
-    if (B < 0 || B > FO_BITS * d) return FO_ERR_ARG;
+    if (!fo_bits_ok(bits) || B < 0 || B > bits * d) return FO_ERR_ARG;
     fo_rank_item *order = (fo_rank_item *)malloc((size_t)d * sizeof *order);
     if (!order) return FO_ERR_ARG;
     for (int64_t c = 0; c < d; ++c) {
@@ -269,7 +276,7 @@ int fo_plan_greedy(const float *w, int64_t d, int64_t B, uint8_t *t)
     for (int64_t i = 0; i < d; ++i) {
         int64_t take = 0;
         if (left > 0) {
-            take = left < FO_BITS ? left : FO_BITS;
+            take = left < bits ? left : bits;
             left -= take;
         }
         t[order[i].c] = (uint8_t)take;
@@ -283,11 +290,11 @@ int fo_plan_greedy(const float *w, int64_t d, int64_t B, uint8_t *t)
  * channels, 核心方法 / 读侧, and notes that finer handling is possible).
  * Reading: the distortion of a channel read at t bits falls as 4^-t, so
  * bit t+1 of channel c is worth w_c * 4^-t; the B bits go one at a time to
- * the channel of largest w_c * 4^-t_c (t_c < 4), ties to the lower channel.
- * 4^-t is a power of two, so the float gains are exact.  B in [0, 4d]. */
-int fo_plan_marginal(const float *w, int64_t d, int64_t B, uint8_t *t)
+ * the channel of largest w_c * 4^-t_c (t_c < b), ties to the lower channel.
+ * 4^-t is a power of two, so the float gains are exact.  B in [0, b*d]. */
+int fo_plan_marginal(const float *w, int64_t d, int64_t B, int64_t bits, uint8_t *t)
 {
-    if (B < 0 || B > FO_BITS * d) return FO_ERR_ARG;
+    if (!fo_bits_ok(bits) || B < 0 || B > bits * d) return FO_ERR_ARG;
     for (int64_t c = 0; c < d; ++c) {
         if (!isfinite(w[c])) return FO_ERR_NONFINITE;
         t[c] = 0;
@@ -296,7 +303,7 @@ int fo_plan_marginal(const float *w, int64_t d, int64_t B, uint8_t *t)
         int64_t best = -1;
         float best_gain = 0.0f;
         for (int64_t c = 0; c < d; ++c) {
-            if (t[c] >= FO_BITS) continue;
+            if (t[c] >= bits) continue;
             const float gain = w[c] * (1.0f / (float)(1 << (2 * t[c])));
             if (best < 0 || gain > best_gain) {
                 best = c;
@@ -309,10 +316,10 @@ int fo_plan_marginal(const float *w, int64_t d, int64_t B, uint8_t *t)
 }
 
 /* Fixed-width baseline plan: the r channels of largest |q_c| (ties to the
- * lower channel) are read at all 4 bits, the rest not at all. */
-int fo_fixed_plan(const uint16_t *q_bf16, int64_t d, int64_t r, uint8_t *t)
+ * lower channel) are read at all b bits, the rest not at all. */
+int fo_fixed_plan(const uint16_t *q_bf16, int64_t d, int64_t r, int64_t bits, uint8_t *t)
 {
-    if (r < 0 || r > d) return FO_ERR_ARG;
+    if (r < 0 || r > d || !fo_bits_ok(bits)) return FO_ERR_ARG;
     fo_rank_item *order = (fo_rank_item *)malloc((size_t)d * sizeof *order);
     if (!order) return FO_ERR_ARG;
     for (int64_t c = 0; c < d; ++c) {
@@ -320,7 +327,7 @@ int fo_fixed_plan(const uint16_t *q_bf16, int64_t d, int64_t r, uint8_t *t)
         order[c].c = c;
     }
     qsort(order, (size_t)d, sizeof *order, fo_rank_cmp);
-    for (int64_t i = 0; i < d; ++i) t[order[i].c] = (uint8_t)(i < r ? FO_BITS : 0);
+    for (int64_t i = 0; i < d; ++i) t[order[i].c] = (uint8_t)(i < r ? bits : 0);
     free(order);
     return FO_OK;
 }
@@ -349,53 +356,58 @@ uint64_t fo_plan_bytes(const uint8_t *t, int64_t d, int64_t n_words)
 /* Scoring from the selected planes.                                    */
 /* ------------------------------------------------------------------ */
 
-/* A key read at t bits with value u = code >> (4-t) lies in the coarse bin
- * of fine levels [u*2^(4-t), u*2^(4-t) + 2^(4-t) - 1]; it is rebuilt at the
- * bin's middle.  t = 4 gives mn + scale*code; t = 0 gives mn + 7.5*scale. */
-static double fo_coarse_midpoint(float mn, float scale, int t, int u)
+/* A key read at t of b bits with value u = code >> (b-t) lies in the coarse
+ * bin of fine levels [u*2^(b-t), u*2^(b-t) + 2^(b-t) - 1]; it is rebuilt at
+ * the bin's middle.  t = b gives mn + scale*code; t = 0 gives
+ * mn + scale*(2^b-1)/2 (7.5*scale for b = 4). */
+static double fo_coarse_midpoint(float mn, float scale, int t, int u, int bits)
 {
-    int width = 1 << (FO_BITS - t);
+    int width = 1 << (bits - t);
     double level = (double)(width * u) + (double)(width - 1) / 2.0;
     return (double)mn + (double)scale * level;
 }
 
 /* Score every key of one KV head for one query from its plan t:
- * planes_h uint32 [d][4][n_words]; mn, scale [d]; q bf16 [d]; t [d];
+ * planes_h uint32 [d][b][n_words]; mn, scale [d]; q bf16 [d]; t [d];
  * s float64 [n].  Reads slots 0..t_c-1 of each channel (MSB first). */
 int fo_score_planes(const uint32_t *planes_h, const float *mn, const float *scale,
-                    const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
-                    int64_t n_words, double *s)
+                    const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t bits,
+                    int64_t n, int64_t n_words, double *s)
 {
+    if (!fo_bits_ok(bits)) return FO_ERR_ARG;
     for (int64_t j = 0; j < n; ++j) {
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c) {
             int tc = t[c];
-            if (tc < 0 || tc > FO_BITS) return FO_ERR_ARG;
+            if (tc < 0 || tc > bits) return FO_ERR_ARG;
             int u = 0;
             for (int slot = 0; slot < tc; ++slot) {
-                uint32_t word = planes_h[(c * FO_BITS + slot) * n_words + j / 32];
+                uint32_t word = planes_h[(c * bits + slot) * n_words + j / 32];
                 u = (u << 1) | (int)((word >> (j % 32)) & 1u);
             }
-            acc += (double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u);
+            acc += (double)bf16_value(q_bf16[c]) *
+                   fo_coarse_midpoint(mn[c], scale[c], tc, u, (int)bits);
         }
         s[j] = acc;
     }
     return FO_OK;
 }
 
-/* The same score from the 4-bit codes by re-quantising to t bits:
+/* The same score from the b-bit codes by re-quantising to t bits:
  * codes_h uint8 [d][n]. */
 int fo_score_codes(const uint8_t *codes_h, const float *mn, const float *scale,
-                   const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
-                   double *s)
+                   const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t bits,
+                   int64_t n, double *s)
 {
+    if (!fo_bits_ok(bits)) return FO_ERR_ARG;
     for (int64_t j = 0; j < n; ++j) {
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c) {
             int tc = t[c];
-            if (tc < 0 || tc > FO_BITS) return FO_ERR_ARG;
-            int u = codes_h[c * n + j] >> (FO_BITS - tc);
-            acc += (double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u);
+            if (tc < 0 || tc > bits) return FO_ERR_ARG;
+            int u = codes_h[c * n + j] >> (bits - tc);
+            acc += (double)bf16_value(q_bf16[c]) *
+                   fo_coarse_midpoint(mn[c], scale[c], tc, u, (int)bits);
         }
         s[j] = acc;
     }
@@ -405,19 +417,22 @@ int fo_score_codes(const uint8_t *codes_h, const float *mn, const float *scale,
 /* sum_c |q_c * khat_c,j| for the same reading: the scale a score's
  * rounding error is measured against. */
 int fo_score_abs_planes(const uint32_t *planes_h, const float *mn, const float *scale,
-                        const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t n,
-                        int64_t n_words, double *a)
+                        const uint16_t *q_bf16, const uint8_t *t, int64_t d, int64_t bits,
+                        int64_t n, int64_t n_words, double *a)
 {
+    if (!fo_bits_ok(bits)) return FO_ERR_ARG;
     for (int64_t j = 0; j < n; ++j) {
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c) {
             int tc = t[c];
+            if (tc < 0 || tc > bits) return FO_ERR_ARG;
             int u = 0;
             for (int slot = 0; slot < tc; ++slot) {
-                uint32_t word = planes_h[(c * FO_BITS + slot) * n_words + j / 32];
+                uint32_t word = planes_h[(c * bits + slot) * n_words + j / 32];
                 u = (u << 1) | (int)((word >> (j % 32)) & 1u);
             }
-            acc += fabs((double)bf16_value(q_bf16[c]) * fo_coarse_midpoint(mn[c], scale[c], tc, u));
+            acc += fabs((double)bf16_value(q_bf16[c]) *
+                        fo_coarse_midpoint(mn[c], scale[c], tc, u, (int)bits));
         }
         a[j] = acc;
     }

@@ -13,24 +13,24 @@ from tests.conftest import read_golden
 
 MUTATIONS = {
     "dropped_half_in_rounding": ("float shifted = ratio + 0.5f;", "float shifted = ratio;"),
-    "scale_over_16": ("(hi - lo) / (float)FO_LEVELS", "(hi - lo) / 16.0f"),
-    "lsb_first_planes": ("pc[(FO_BITS - 1 - p) * n_words + j / 32] |=", "pc[p * n_words + j / 32] |="),
+    "scale_over_16": ("(hi - lo) / (float)levels", "(hi - lo) / (float)(levels + 1)"),
+    "lsb_first_planes": ("pc[(bits - 1 - p) * n_words + j / 32] |=", "pc[p * n_words + j / 32] |="),
     "variance_missing_square": ("double sc2 = sc * sc;", "double sc2 = sc;"),
     "importance_uses_abs_q": ("float qq = qc * qc;", "float qq = fabsf(qc);"),
     "plan_ascending_importance": ("if (a->key > b->key) return -1;\n    if (a->key < b->key) return 1;",
                                   "if (a->key < b->key) return -1;\n    if (a->key > b->key) return 1;"),
-    "plan_cap_3_bits": ("take = left < FO_BITS ? left : FO_BITS;", "take = left < 3 ? left : 3;"),
+    "plan_cap_3_bits": ("take = left < bits ? left : bits;", "take = left < 3 ? left : 3;"),
     "bin_low_edge_not_middle": ("(double)(width - 1) / 2.0", "0.0"),
     "planes_read_lsb_first": ("u = (u << 1) | (int)((word >> (j % 32)) & 1u);",
                               "u = u | (int)(((word >> (j % 32)) & 1u) << slot);"),
     "topk_ties_to_higher_index": ("return (a->j < b->j) ? -1 : (a->j > b->j);",
                                   "return (a->j > b->j) ? -1 : (a->j < b->j);"),
     "union_takes_min": ("if (t[g * d + c] > m) m = t[g * d + c];", "if (g == 0) m = t[g * d + c];"),
-    "append_lsb_first": ("if ((v >> p) & 1)\n                        pc[(FO_BITS - 1 - p) * n_words",
+    "append_lsb_first": ("if ((v >> p) & 1)\n                        pc[(bits - 1 - p) * n_words",
                          "if ((v >> p) & 1)\n                        pc[p * n_words"),
     "append_ignores_min": ("float diff = x - lo;", "float diff = x;"),
     "append_variance_old_count": ("const int64_t nn = n + m;", "const int64_t nn = n;"),
-    "append_no_high_clamp_count": ("out_of_range = level < 0.0f || level > (float)FO_LEVELS;",
+    "append_no_high_clamp_count": ("out_of_range = level < 0.0f || level > (float)levels;",
                                    "out_of_range = level < 0.0f;"),
     "attention_no_max_shift": ("const double p = exp(logit[i] - mx);", "const double p = exp(logit[i]);"),
     "attention_unscaled_logits": ("logit[i] = scale * acc;", "logit[i] = acc;"),
@@ -40,6 +40,13 @@ MUTATIONS = {
     "merge_ignores_offset": ("items[s * k_s + i].j = offset[s] + idx[s * k_s + i];",
                              "items[s * k_s + i].j = idx[s * k_s + i];"),
     "merge_output_not_index_ordered": ("while (p >= 0 && items[p].j > x.j)", "while (0)"),
+    "quantize_levels_stay_15": ("const int levels = (1 << bits) - 1;", "const int levels = 15;"),
+    "plan_cap_stays_4_bits": ("take = left < bits ? left : bits;", "take = left < 4 ? left : 4;"),
+    "fixed_plan_reads_4_bits": ("(uint8_t)(i < r ? bits : 0)", "(uint8_t)(i < r ? 4 : 0)"),
+    "unpack_reads_4_slots": ("for (int p = 0; p < bits; ++p)\n                    v |=",
+                             "for (int p = 0; p < bits && p < 4; ++p)\n                    v |="),
+    "midpoint_of_4bit_bins": ("double level = (double)(width * u) + (double)(width - 1) / 2.0;",
+                              "double level = (double)(width * u) + (double)((width < 16 ? width : 16) - 1) / 2.0;"),
     "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
                                "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
 }
@@ -64,6 +71,14 @@ PIN_TESTS = [
     pins.test_marginal_plan_spreads_uniform_importance_round_robin,
     pins.test_marginal_plan_hand_worked,
     lambda: pins.test_merging_shard_topks_is_the_topk_of_all_keys(3, 999, 64),
+    pins.test_quantize_8bit_hand_worked,
+    pins.test_quantize_8bit_error_bound_and_extremes,
+    pins.test_plane_layout_8bit_hand_worked,
+    lambda: pins.test_planes_8bit_round_trip_and_size(1000),
+    pins.test_coarse_bin_8bit_is_mean_of_its_fine_levels,
+    lambda: pins.test_plan_8bit_is_optimal_by_brute_force(2),
+    pins.test_fixed_plan_8bit_reads_whole_channels,
+    pins.test_append_8bit_in_range_equals_repacking_and_clamps,
 ]
 
 

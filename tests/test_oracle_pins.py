@@ -518,3 +518,156 @@ def test_merging_shard_topks_is_the_topk_of_all_keys(S, n, k):
     assert np.array_equal(gi, np.sort(ref_i))
     assert np.all(np.diff(gi) > 0)
     np.testing.assert_array_equal(gs, s[gi])
+
+
+# -------------------------------------------------------- 8-plane variant
+# The explainer's deployment notes (部署前必读, item 3) say an 8-bit upstream K
+# cache needs the index adapted to 8 planes per channel.  Reading: the same
+# quantiser with 255 levels, slots MSB first, plans capped at 8 bits, and the
+# same coarse-bin midpoint rebuild.  These pins fix that reading.
+def test_quantize_8bit_hand_worked():
+    """max - min = 255 makes scale exactly 1, so each code is
+    floor(k - min + 0.5): worked by hand."""
+    keys = np.array([-100.0, 155.0, 27.25, 27.75, 0.5, 130.5, 154.4], np.float32)
+    mn, scale, codes = oracle.quantize(keys[None, :, None], bits=8)
+    assert mn[0, 0] == -100.0 and scale[0, 0] == 1.0
+    assert list(codes[0, 0]) == [0, 255, 127, 128, 101, 231, 254]
+    s1, s2, _ = oracle.channel_stats(codes, scale)
+    assert s1[0, 0] == 0 + 255 + 127 + 128 + 101 + 231 + 254
+    assert s2[0, 0] == 255 ** 2 + 127 ** 2 + 128 ** 2 + 101 ** 2 + 231 ** 2 + 254 ** 2
+
+
+def test_quantize_8bit_error_bound_and_extremes():
+    ses = synth.make_session(13, 2, 1, 3000, 16)
+    mn, scale, codes = oracle.quantize(ses.keys, bits=8)
+    k = ses.keys.transpose(0, 2, 1).astype(np.float64)
+    deq = mn[..., None].astype(np.float64) + scale[..., None].astype(np.float64) * codes
+    assert np.all(np.abs(deq - k) <= scale[..., None] * (0.5 + 1e-4) + 1e-6)
+    jmin, jmax = np.argmin(k, axis=2), np.argmax(k, axis=2)
+    assert np.all(np.take_along_axis(codes, jmin[..., None], 2) == 0)
+    assert np.all(np.take_along_axis(codes, jmax[..., None], 2) == 255)
+    assert len(np.unique(codes[0, 0])) >= 150          # far more than 16 levels
+    _, _, sigma2 = oracle.channel_stats(codes, scale)
+    np.testing.assert_allclose(sigma2, deq.var(axis=2), rtol=1e-6)
+    ratio = sigma2 / (ses.sigma ** 2)                   # 8-bit noise is scale^2/12
+    assert np.all((ratio > 0.9) & (ratio < 1.1))
+
+
+def test_plane_layout_8bit_hand_worked():
+    """Code 177 = 0b10110001 at key 0 sets slots 0, 2, 3, 7 of word 0, bit 0;
+    code 66 = 0b01000010 at key 37 sets slots 1 and 6 of word 1, bit 5."""
+    codes = np.zeros((1, 1, 64), np.uint8)
+    codes[0, 0, 0], codes[0, 0, 37] = 177, 66
+    planes = oracle.pack_planes(codes, bits=8)
+    assert planes.shape == (1, 1, 8, 4)
+    expect = np.zeros((8, 4), np.uint32)
+    for s in (0, 2, 3, 7):
+        expect[s, 0] = 1
+    for s in (1, 6):
+        expect[s, 1] = 1 << 5
+    assert np.array_equal(planes[0, 0], expect)
+
+
+@pytest.mark.parametrize("n", [1, 33, 128, 1000])
+def test_planes_8bit_round_trip_and_size(n):
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 256, size=(2, 3, n), dtype=np.uint8)
+    planes = oracle.pack_planes(codes, bits=8)
+    assert planes.shape == (2, 3, 8, oracle.n_words_for(n))
+    assert np.array_equal(oracle.unpack_planes(planes, n), codes)
+    assert not oracle.unpack_planes(planes, planes.shape[-1] * 32)[..., n:].any()
+    # one byte per key per channel when n is a multiple of 128
+    if n % 128 == 0:
+        assert planes.nbytes == 2 * 3 * n
+
+
+def test_coarse_bin_8bit_is_mean_of_its_fine_levels():
+    mn, sc = np.float32(0.75), np.float32(0.0625)
+    one = synth.f32_to_bf16_bits(np.array([1.0], np.float32))
+    codes = np.arange(256, dtype=np.uint8)[None, None, :]
+    planes = oracle.pack_planes(codes, bits=8)
+    for t in range(9):
+        s = oracle.score_planes(planes[0], np.array([mn]), np.array([sc]), one,
+                                np.array([t], np.uint8), 256)
+        width = 1 << (8 - t)
+        for code in range(0, 256, 7):
+            lo = (code // width) * width
+            levels = float(mn) + float(sc) * np.arange(lo, lo + width, dtype=np.float64)
+            assert s[code] == pytest.approx(levels.mean(), rel=1e-15, abs=1e-15)
+
+
+def test_8bit_scores_full_zero_and_prefix_depths():
+    ses = synth.make_session(21, 1, 2, 600, 300)
+    ix = oracle.build_index(ses.keys, bits=8)
+    assert ix["planes"].shape[-2] == 8
+    deq = ix["mn"][0][:, None].astype(np.float64) + \
+        ix["scale"][0][:, None].astype(np.float64) * ix["codes"][0]
+    rng = np.random.default_rng(3)
+    for g in range(2):
+        q = ses.q_bf16[g]
+        qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+        full = oracle.score_planes(ix["planes"][0], ix["mn"][0], ix["scale"][0], q,
+                                   np.full(128, 8, np.uint8), 600)
+        mag = np.abs(qf) @ np.abs(deq)
+        assert np.all(np.abs(full - qf @ deq) <= 1e-13 * mag)
+        zero = oracle.score_planes(ix["planes"][0], ix["mn"][0], ix["scale"][0], q,
+                                   np.zeros(128, np.uint8), 600)
+        const = qf @ (ix["mn"][0].astype(np.float64) + 127.5 * ix["scale"][0].astype(np.float64))
+        assert np.allclose(zero, const, rtol=1e-13, atol=0)
+        t = rng.integers(0, 9, size=128).astype(np.uint8)
+        a = oracle.score_planes(ix["planes"][0], ix["mn"][0], ix["scale"][0], q, t, 600)
+        b = oracle.score_codes(ix["codes"][0], ix["mn"][0], ix["scale"][0], q, t, bits=8)
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("d", [1, 2, 3])
+def test_plan_8bit_is_optimal_by_brute_force(d):
+    rng = np.random.default_rng(200 + d)
+    allocs = np.array(list(itertools.product(range(9), repeat=d)), dtype=np.int64)
+    for trial in range(5):
+        w = rng.lognormal(0, 1, size=d).astype(np.float32)
+        vals = allocs @ w.astype(np.float64)
+        for B in range(0, 8 * d + 1):
+            t = oracle.plan_greedy(w, B, bits=8)
+            assert int(t.sum()) == B and t.max() <= 8
+            best = vals[allocs.sum(axis=1) <= B].max()
+            assert float(np.dot(w.astype(np.float64), t)) == pytest.approx(best, rel=1e-12)
+    with pytest.raises(ValueError):
+        oracle.plan_greedy(np.ones(d, np.float32), 8 * d + 1, bits=8)
+
+
+def test_marginal_plan_8bit_is_optimal_by_brute_force():
+    d = 3
+    rng = np.random.default_rng(33)
+    allocs = list(itertools.product(range(9), repeat=d))
+    for trial in range(4):
+        w = rng.lognormal(0.0, 2.0, d).astype(np.float32)
+        for B in range(0, 8 * d + 1):
+            t = oracle.plan_marginal(w, B, bits=8)
+            assert int(t.sum()) == B and t.max() <= 8
+            best = max(_distortion_drop(w, c) for c in allocs if sum(c) == B)
+            assert abs(_distortion_drop(w, t) - best) <= 1e-9 * max(1.0, best)
+
+
+def test_fixed_plan_8bit_reads_whole_channels():
+    q = synth.make_session(0, 1, 1, 128, 16).q_bf16[0]
+    for r in (0, 17, 34, 128):
+        t = oracle.fixed_plan(q, r, bits=8)
+        assert int(t.sum()) == 8 * r and set(np.unique(t)) <= {0, 8}
+        assert np.array_equal(t > 0, oracle.fixed_plan(q, r) > 0)
+
+
+def test_append_8bit_in_range_equals_repacking_and_clamps():
+    first, new = _split_in_range(77, 2, 300, 45, 16)
+    ix = oracle.build_index(first, capacity=345, bits=8)
+    clamped = np.zeros((2, 16), np.uint32)
+    oracle.append(ix, new, clamped)
+    full = oracle.build_index(np.concatenate([first, new], axis=1), bits=8)
+    for name in ("planes", "s1", "s2", "sigma2"):
+        assert np.array_equal(ix[name], full[name]), name
+    assert clamped.sum() == 0
+    keys = np.arange(256, dtype=np.float32)[None, :, None]      # scale 1
+    ix = oracle.build_index(keys, capacity=384, bits=8)
+    clamped = np.zeros((1, 1), np.uint32)
+    oracle.append(ix, np.array([[[-3.0], [300.0], [17.4]]], np.float32), clamped)
+    assert list(ix["codes"][0, 0, 256:]) == [0, 255, 17] and clamped[0, 0] == 2
