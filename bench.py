@@ -2,7 +2,8 @@
 """Benchmark of the Fathom per-query read-depth top-k key scan on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
-                    [--workload qwen3_8b_layer_128k|plan_variants_128k|host_1m|host_256k|fixed_vs_wf_1m|
+                    [--workload qwen3_8b_layer_128k|qwen3_8b_layer_128k_8plane|
+                               plan_variants_128k|host_1m|host_256k|fixed_vs_wf_1m|
                                agent_16_sessions|append_layer_128k|
                                attention_layer_128k]
 
@@ -47,12 +48,17 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
 # plans: ("wf", B) = reverse water-filling at B bits per key; ("mg", B) = the
-# marginal-gain variant; ("fixed", r) = the top-r channels by |q_c| at 4 bits.  "device_keys": keys drawn on the
-# GPU (synth.device_keys) instead of numpy, for sizes numpy would take
-# minutes on.  agent_16_sessions scans its sessions in one batched call.
+# marginal-gain variant; ("fixed", r) = the top-r channels by |q_c| at all
+# b bits.  "bits": b, the stored code width (4 unless given; 8 = the 8-plane
+# variant for an 8-bit K cache).  "device_keys": keys drawn on the GPU
+# (synth.device_keys) instead of numpy, for sizes numpy would take minutes
+# on.  agent_16_sessions scans its sessions in one batched call.
 WORKLOADS = {
     "qwen3_8b_layer_128k": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
                                 plans=(("wf", 68), ("wf", 92), ("wf", 136))),
+    # the same layer with an 8-bit K cache (8 planes per channel), same budgets
+    "qwen3_8b_layer_128k_8plane": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
+                                       bits=8, plans=(("wf", 68), ("wf", 92), ("wf", 136))),
     "host_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                     plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
     # the host path at a quarter of the keys: the profiling case of the fetch
@@ -84,9 +90,9 @@ def plan_name(spec):
     return f"{spec[0]}{spec[1]}"
 
 
-def plan_bits(spec):
-    """Bits per key a query of this plan reads."""
-    return 4 * spec[1] if spec[0] == "fixed" else spec[1]
+def plan_bits(spec, bits=4):
+    """Bits per key a query of this plan reads (bits = the code width b)."""
+    return bits * spec[1] if spec[0] == "fixed" else spec[1]
 
 
 def parse_args():
@@ -126,7 +132,7 @@ def config_of(wl_name, wl, flush_note, sessions=None):
     c = {"workload": wl_name, "kv_heads": wl["H"], "query_heads_per_kv": wl["G"],
          "head_dim": wl["d"], "k": wl["k"],
          "residency": "hbm" if wl["residency"] == "device" else "host_pinned_mapped",
-         "l2": flush_note}
+         "code_bits": wl.get("bits", 4), "l2": flush_note}
     if sessions is None:
         c["n_keys"] = wl["n"]
         c["plans"] = [plan_name(p) for p in wl["plans"]]
@@ -215,7 +221,7 @@ def measure_host_link(fp, torch, nbytes=1 << 30, reps=10):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0):
+def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bits=4):
     """Time the oracle (plan + fp64 score + full-sort top-k per query) over
     the given KV heads' keys (float32 [h][n][d]) at every plan spec, cycling
     over (head, plan) until at least min_seconds have passed (one round at
@@ -223,7 +229,7 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0):
     timed.  Returns (seconds, head-scans, keys)."""
     import oracle
     if ref is None:
-        ref = oracle.build_index(keys_heads)
+        ref = oracle.build_index(keys_heads, bits=bits)
     n = keys_heads.shape[1]
     pairs = [(hi, spec) for hi in range(keys_heads.shape[0]) for spec in plans]
     t0 = time.perf_counter()
@@ -233,11 +239,13 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0):
         for g in range(G):
             qrow = q_bf16[hi * G + g]
             if spec[0] == "wf":
-                tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1])
+                tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1],
+                                        bits)
             elif spec[0] == "mg":
-                tq = oracle.plan_marginal(oracle.importance(qrow, ref["sigma2"][hi]), spec[1])
+                tq = oracle.plan_marginal(oracle.importance(qrow, ref["sigma2"][hi]), spec[1],
+                                          bits)
             else:
-                tq = oracle.fixed_plan(qrow, spec[1])
+                tq = oracle.fixed_plan(qrow, spec[1], bits)
             s = oracle.score_planes(ref["planes"][hi], ref["mn"][hi], ref["scale"][hi],
                                     qrow, tq, n)
             oracle.topk(s, k)
@@ -248,10 +256,10 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0):
 CPU_BASELINE_SECONDS = 12.0
 
 
-def cpu_baseline(keys_heads, q_bf16, G, plans, k):
+def cpu_baseline(keys_heads, q_bf16, G, plans, k, bits=4):
     """About 12 s of single-thread oracle work on a few KV heads."""
     secs, scans, keys = oracle_sample(keys_heads, q_bf16, G, plans, k,
-                                      min_seconds=CPU_BASELINE_SECONDS)
+                                      min_seconds=CPU_BASELINE_SECONDS, bits=bits)
     return {"value": keys / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{scans} scans of one KV head ({G} query heads, {keys_heads.shape[1]} "
                       f"keys) cycling over {keys_heads.shape[0]} KV head(s) x plans "
@@ -270,13 +278,14 @@ def run_reference(args, wl_name, wl):
         return
     n = wl["n"] if (wl["n"] and wl["residency"] == "device") else min(wl["n"] or (1 << 18), 1 << 18)
     plans = reference_plans(wl)
-    ses = synth.make_session(0, 1, wl["G"], n, plan_bits(plans[0]), head_dim=wl["d"])
+    bits = wl.get("bits", 4)
+    ses = synth.make_session(0, 1, wl["G"], n, plan_bits(plans[0], bits), head_dim=wl["d"])
     import oracle
-    ref = oracle.build_index(ses.keys[:1])
+    ref = oracle.build_index(ses.keys[:1], bits=bits)
     times = []
     for i in range(args.warmup + args.steps):
         secs, _, _ = oracle_sample(ses.keys[:1], ses.q_bf16, wl["G"], (plans[i % len(plans)],),
-                                   wl["k"], ref)
+                                   wl["k"], ref, bits=bits)
         if i >= args.warmup:
             times.append(secs)
     keys_per_step = n                      # one KV head, one plan, per step
@@ -309,7 +318,10 @@ def recorded_traffic(wl_name, wl, kernel):
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)[kernel]
+            recs = json.load(f)
+        # a capture of this very workload ("kernel@workload") before the
+        # kernel's default one
+        rec = recs.get(f"{kernel}@{wl_name}") or recs[kernel]
         with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
                 return None, "kernel changed since the recorded capture"
@@ -367,7 +379,7 @@ def build_sessions(wl, rank, torch, fp):
         else:
             ses = synth.make_session(p["seed"], H, G, p["n"], 64, head_dim=d)
             keys = torch.from_numpy(ses.keys).cuda()
-        index = fp.KeyIndex(H, G, p["n"], d, wl["residency"])
+        index = fp.KeyIndex(H, G, p["n"], d, wl["residency"], bits=wl.get("bits", 4))
         index.pack(keys)
         plans = wl["plans"] if wl.get("plans") else (("wf", p["budget"]),)
         out.append(dict(n=p["n"], budget=p["budget"], keys=keys, index=index, plans=plans))
@@ -402,7 +414,7 @@ def run_fathom(args, wl_name, wl):
         S["q"] = torch.from_numpy(synth.draw_queries(10_000 + 100 * rank + si, Q, d,
                                                      count=W + K).view(np.int16)).cuda()
         for spec in S["plans"]:
-            B = plan_bits(spec)
+            B = plan_bits(spec, wl.get("bits", 4))
             jobs.append(dict(s=si, spec=spec, buf=fp.ScanBuffers(S["index"], k),
                              bvec=torch.full((Q,), B, dtype=torch.int32, device="cuda")))
     ws_batch = None
@@ -517,7 +529,7 @@ def run_fathom(args, wl_name, wl):
                     inter = np.intersect1d(exact[g].cpu().numpy(), got[h, g].cpu().numpy())
                     rec.append(len(inter) / k)
             per_plan.append({"plan": plan_name(j["spec"]), "session": j["s"], "n_keys": S["n"],
-                             "bits_per_key": plan_bits(j["spec"]),
+                             "bits_per_key": plan_bits(j["spec"], wl.get("bits", 4)),
                              "bytes_per_query": float(qb.mean()),
                              "union_bytes_per_kv_head": float(ub.mean()),
                              "union_factor": float(ub.sum() / (qb.sum() / G)),
@@ -593,7 +605,7 @@ def run_fathom(args, wl_name, wl):
         nh = max(1, min(H, (8 * 131072) // S0["n"]))
         line["cpu_baseline"] = cpu_baseline(S0["keys"][:nh].cpu().numpy(),
                                             S0["q"][0].cpu().numpy().view(np.uint16), G,
-                                            S0["plans"], k)
+                                            S0["plans"], k, wl.get("bits", 4))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -57,7 +57,7 @@ class fathom_index(ctypes.Structure):
         ("n_words", ctypes.c_int32), ("residency", ctypes.c_int32),
         ("planes", ctypes.c_void_p), ("mn", ctypes.c_void_p), ("scale", ctypes.c_void_p),
         ("sigma2", ctypes.c_void_p), ("sum_code", ctypes.c_void_p),
-        ("sum_code2", ctypes.c_void_p),
+        ("sum_code2", ctypes.c_void_p), ("bits", ctypes.c_int32),
     ]
 
 
@@ -284,16 +284,19 @@ class KeyIndex:
 
     residency "device" keeps the planes in HBM; "host_mapped" keeps them in
     pinned host memory read zero-copy by the scan.  Statistics stay on the
-    device either way."""
+    device either way.  bits: 4 (the 4-bit K cache) or 8 (the 8-plane
+    variant for an 8-bit K cache)."""
 
     def __init__(self, n_kv_heads: int, group: int, n_keys: int, head_dim: int = 128,
                  residency: str = "device", device: Optional[int] = None,
-                 capacity: Optional[int] = None):
+                 capacity: Optional[int] = None, bits: int = 4):
         import torch
+        if bits not in (4, 8):
+            raise ValueError(f"bits must be 4 or 8, not {bits}")
         dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
         self.n_words = fathom_n_words(max(n_keys, capacity or n_keys))
         H, d = n_kv_heads, head_dim
-        shape = (H, d, 4, self.n_words)
+        shape = (H, d, bits, self.n_words)
         if residency == "device":
             self.planes = torch.empty(shape, dtype=torch.int32, device=dev)
             res = FATHOM_RES_DEVICE
@@ -311,7 +314,7 @@ class KeyIndex:
         self.desc = fathom_index(H, group, d, n_keys, self.n_words, res,
                                  self.planes.data_ptr(), self.mn.data_ptr(),
                                  self.scale.data_ptr(), self.sigma2.data_ptr(),
-                                 self.sum_code.data_ptr(), self.sum_code2.data_ptr())
+                                 self.sum_code.data_ptr(), self.sum_code2.data_ptr(), bits)
         self.device = dev
 
     @property
@@ -329,6 +332,10 @@ class KeyIndex:
     @property
     def n_keys(self):
         return self.desc.n_keys
+
+    @property
+    def bits(self):
+        return self.desc.bits
 
     @property
     def capacity(self):

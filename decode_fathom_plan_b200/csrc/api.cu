@@ -67,9 +67,49 @@ bool index_shape_ok(const fathom_index *ix)
     if (ix->n_keys < 1 || ix->n_words < 4 || ix->n_words % 4) return false;
     if ((long long)ix->n_words * 32 < (long long)ix->n_keys) return false;
     if (ix->residency != FATHOM_RES_DEVICE && ix->residency != FATHOM_RES_HOST_MAPPED) return false;
+    if (ix->bits != 0 && ix->bits != 4 && ix->bits != 8) return false;
+    const int bits = index_bits(*ix);
+    // 8 planes: the scan's 2d nibble channels fit its head_dim limit
+    if (bits == 8 && 2 * ix->head_dim > kMaxHeadDim) return false;
+    // n * sum_code2 <= n^2 * (2^b - 1)^2 must fit in int64
+    if ((long long)ix->n_words * 32 > (bits == 8 ? (1ll << 23) : (1ll << 27))) return false;
     // global plane row indices must fit in 32 bits
-    if ((long long)ix->n_kv_heads * ix->head_dim * kBits >= (1ll << 31)) return false;
+    if ((long long)ix->n_kv_heads * ix->head_dim * bits >= (1ll << 31)) return false;
     return true;
+}
+
+size_t align16(size_t b) { return (b + 15) & ~(size_t)15; }
+
+// The descriptor the 4-plane scan sees: an 8-plane index is 2d nibble
+// channels of 4 planes each (same planes; mn and scale are replaced by the
+// lifted arrays before a launch).
+fathom_index scan_view(const fathom_index &ix)
+{
+    fathom_index v = ix;
+    if (index_bits(ix) == 8) {
+        v.head_dim = 2 * ix.head_dim;
+        v.bits = 4;
+    }
+    return v;
+}
+
+// Workspace of a scan call: the scan's own part (16-byte rounded), then the
+// lifted arrays of every 8-plane session.
+size_t scan_part_bytes(const fathom_index *sessions, int n_sessions, int k)
+{
+    std::vector<fathom_index> views(n_sessions);
+    for (int s = 0; s < n_sessions; ++s) views[s] = scan_view(sessions[s]);
+    return align16(scan_workspace_bytes(views.data(), n_sessions, k));
+}
+
+size_t scan_total_bytes(const fathom_index *sessions, int n_sessions, int k)
+{
+    size_t total = scan_part_bytes(sessions, n_sessions, k);
+    for (int s = 0; s < n_sessions; ++s)
+        if (index_bits(sessions[s]) == 8)
+            total += lift_bytes(sessions[s].n_kv_heads, sessions[s].n_kv_heads * sessions[s].group,
+                                sessions[s].head_dim);
+    return total;
 }
 
 // Resolve the planes pointer to a device address for the residency mode.
@@ -133,17 +173,43 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
     for (int s = 0; s < n_sessions; ++s) {
         const fathom_index *ix = &sessions[s];
         if (!index_shape_ok(ix) || !ix->mn || !ix->scale) return FATHOM_ERR_INVALID_ARG;
-        if (ix->head_dim != sessions[0].head_dim || ix->group != sessions[0].group)
+        if (ix->head_dim != sessions[0].head_dim || ix->group != sessions[0].group ||
+            index_bits(*ix) != index_bits(sessions[0]))
             return FATHOM_ERR_INVALID_ARG;
         if (k > ix->n_keys) return FATHOM_ERR_INVALID_ARG;
         if (!q[s] || !t[s] || !tu[s] || !out_idx[s] || !out_score[s]) return FATHOM_ERR_INVALID_ARG;
-        resolved[s] = *ix;
+        resolved[s] = scan_view(*ix);
         fathom_status st = resolve_planes(ix, &resolved[s].planes);
         if (st != FATHOM_OK) return st;
         args[s] = ScanSessionArgs{&resolved[s], q[s], t[s], tu[s], out_idx[s], out_score[s]};
     }
-    const size_t need = scan_workspace_bytes(sessions, n_sessions, k);
-    if (!ws || !aligned16(ws) || ws_bytes < need) return FATHOM_ERR_WORKSPACE;
+    const size_t scan_part = scan_part_bytes(sessions, n_sessions, k);
+    if (!ws || !aligned16(ws) || ws_bytes < scan_total_bytes(sessions, n_sessions, k))
+        return FATHOM_ERR_WORKSPACE;
+    if (index_bits(sessions[0]) == 8) {
+        // 8-plane sessions: write the nibble-channel arguments behind the
+        // scan's own workspace and point the scan at them
+        unsigned char *at = static_cast<unsigned char *>(ws) + scan_part;
+        for (int s = 0; s < n_sessions; ++s) {
+            const fathom_index &ix = sessions[s];
+            const int H = ix.n_kv_heads, Q = H * ix.group, d = ix.head_dim;
+            LiftArgs la{};
+            la.mn = ix.mn;
+            la.scale = ix.scale;
+            la.q = q[s];
+            la.t = t[s];
+            la.tu = tu[s];
+            lift_carve(at, H, Q, d, &la);
+            at += lift_bytes(H, Q, d);
+            const cudaError_t e = launch_lift(la, stream);
+            if (e != cudaSuccess) return cuda_status(note_error(e, "lift"));
+            resolved[s].mn = la.mn2;
+            resolved[s].scale = la.scale2;
+            args[s].q = la.q2;
+            args[s].t = la.t2;
+            args[s].t_union = la.tu2;
+        }
+    }
 
     ScanProfileHook hook{false, nullptr, nullptr, false};
     EventPair ev{};
@@ -151,7 +217,7 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
         ev = take_event_pair();
         hook = ScanProfileHook{true, ev.begin, ev.end, false};
     }
-    cudaError_t e = launch_scan(args.data(), n_sessions, k, ws, ws_bytes, flags, stream, &hook);
+    cudaError_t e = launch_scan(args.data(), n_sessions, k, ws, scan_part, flags, stream, &hook);
     if (flags & FATHOM_SCAN_PROFILE) {
         std::lock_guard<std::mutex> lock(g_mu);
         if (hook.recorded)
@@ -281,7 +347,7 @@ fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf1
 size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k)
 {
     if (!index_shape_ok(index) || k < 1 || k > kMaxK) return 0;
-    return scan_workspace_bytes(index, 1, k);
+    return scan_total_bytes(index, 1, k);
 }
 
 fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,
@@ -298,8 +364,9 @@ size_t fathom_scan_batched_workspace_bytes(const fathom_index *sessions, int32_t
 {
     if (!sessions || n_sessions < 1 || n_sessions > kMaxSessions || k < 1 || k > kMaxK) return 0;
     for (int s = 0; s < n_sessions; ++s)
-        if (!index_shape_ok(&sessions[s])) return 0;
-    return scan_workspace_bytes(sessions, n_sessions, k);
+        if (!index_shape_ok(&sessions[s]) || index_bits(sessions[s]) != index_bits(sessions[0]))
+            return 0;
+    return scan_total_bytes(sessions, n_sessions, k);
 }
 
 fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_sessions,

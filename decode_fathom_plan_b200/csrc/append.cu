@@ -1,11 +1,12 @@
-// Append path: the decode step's new keys into an existing 4-bit K index.
+// Append path: the decode step's new keys into an existing b-bit K index
+// (b = 4, or 8 for the 8-plane variant).
 //
 // Source: Fathom explainer (papers.ananclaw.com, arXiv 2609.17652),
 // section 核心方法 / 存储侧 (per-channel 4-bit quantisation stored as
 // MSB-first bit planes) and 适用边界 (the 4-bit K cache comes from the
 // serving stack, which grows it by one key per decode step).  A new key is
 // quantised with the index's stored min and scale in the quantiser's own
-// float32 steps, its level clamped to 0..15 (a key outside the stored
+// float32 steps, its level clamped to 0..2^b-1 (a key outside the stored
 // range takes the nearest level, and the clamp is counted per channel as
 // the measure of range drift), its bits are ORed into the zero padding
 // words past the last key, the exact sums S1, S2 grow, and sigma^2 is
@@ -21,6 +22,7 @@
 namespace fathom {
 namespace {
 
+template <int BITS>
 __global__ void __launch_bounds__(256)
 append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_words,
               const float *__restrict__ mn, const float *__restrict__ scale, uint32_t *planes,
@@ -37,7 +39,10 @@ append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_
     const int j_lo = max(n, w * 32), j_hi = min(n + m, w * 32 + 32);
     const int hc = h * d + c;
     const float lo = mn[hc], sc = scale[hc];
-    uint32_t slot[kBits] = {0u, 0u, 0u, 0u};
+    constexpr int kLevels = (1 << BITS) - 1;
+    uint32_t slot[BITS];
+#pragma unroll
+    for (int s = 0; s < BITS; ++s) slot[s] = 0u;
     unsigned long long a1 = 0, a2 = 0;
     unsigned n_clamped = 0;
     bool bad = false;
@@ -49,13 +54,13 @@ append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_
             n_clamped += (x != lo);
         } else {
             const float level = floorf(__fadd_rn(__fdiv_rn(__fsub_rn(x, lo), sc), 0.5f));
-            const bool out = level < 0.0f || level > 15.0f;
+            const bool out = level < 0.0f || level > (float)kLevels;
             n_clamped += out;
-            v = level < 0.0f ? 0 : (level > 15.0f ? 15 : static_cast<int>(level));
+            v = level < 0.0f ? 0 : (level > (float)kLevels ? kLevels : static_cast<int>(level));
         }
 #pragma unroll
-        for (int s = 0; s < kBits; ++s)   // slot s holds bit 3-s
-            slot[s] |= (uint32_t)((v >> (kBits - 1 - s)) & 1) << (j & 31);
+        for (int s = 0; s < BITS; ++s)   // slot s holds bit BITS-1-s
+            slot[s] |= (uint32_t)((v >> (BITS - 1 - s)) & 1) << (j & 31);
         a1 += (unsigned long long)v;
         a2 += (unsigned long long)(v * v);
     };
@@ -73,9 +78,9 @@ append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_
     } else {
         for (int j = j_lo; j < j_hi; ++j) take(j, kc[(size_t)(j - n) * d]);
     }
-    uint32_t *pw = planes + (size_t)hc * kBits * n_words + w;
+    uint32_t *pw = planes + (size_t)hc * BITS * n_words + w;
 #pragma unroll
-    for (int s = 0; s < kBits; ++s)
+    for (int s = 0; s < BITS; ++s)
         if (slot[s]) pw[(size_t)s * n_words] |= slot[s];
     const unsigned long long o1 = atomicAdd(reinterpret_cast<unsigned long long *>(&s1[hc]), a1);
     const unsigned long long o2 = atomicAdd(reinterpret_cast<unsigned long long *>(&s2[hc]), a2);
@@ -97,10 +102,10 @@ cudaError_t launch_append(const float *keys, const fathom_index &ix, int m, uint
     const long long threads = (long long)H * words * d;
     const int block = 256;
     const long long grid = (threads + block - 1) / block;
-    append_kernel<<<(unsigned)grid, block, 0, stream>>>(keys, H, n, m, d, ix.n_words, ix.mn,
-                                                        ix.scale, ix.planes, ix.sum_code,
-                                                        ix.sum_code2, ix.sigma2, clamped,
-                                                        device_status_ptr());
+    auto kern = index_bits(ix) == 8 ? append_kernel<8> : append_kernel<4>;
+    kern<<<(unsigned)grid, block, 0, stream>>>(keys, H, n, m, d, ix.n_words, ix.mn, ix.scale,
+                                               ix.planes, ix.sum_code, ix.sum_code2, ix.sigma2,
+                                               clamped, device_status_ptr());
     note_launch(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || words == 1) return e;

@@ -17,6 +17,10 @@ void note_launch(int n = 1);
 // by the C-ABI layer) and return it.
 cudaError_t note_error(cudaError_t e, const char *site);
 
+// Code width b of an index: 4, or 8 for the 8-plane variant (the C ABI
+// reads 0 as 4 and rejects anything else before a launcher runs).
+inline int index_bits(const fathom_index &ix) { return ix.bits == 8 ? 8 : 4; }
+
 // ---- pack.cu
 cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_minmax,
                         cudaStream_t stream);
@@ -36,6 +40,25 @@ cudaError_t launch_plan(const fathom_index &ix, const uint16_t *q, const int32_t
 cudaError_t launch_plan_marginal(const fathom_index &ix, const uint16_t *q, const int32_t *budget,
                                  uint8_t *t, uint8_t *t_union, uint64_t *bytes,
                                  cudaStream_t stream);
+
+// ---- lift.cu
+// An 8-plane index's scan arguments rewritten for the 4-plane scan over 2d
+// nibble channels (the planes themselves need no change).
+struct LiftArgs {
+    const float *mn, *scale;     // [H][d]
+    const uint16_t *q;           // [Q][d]
+    const uint8_t *t, *tu;       // [Q][d], [H][d]
+    float *mn2, *scale2;         // [H][2d]
+    uint16_t *q2;                // [Q][2d]
+    uint8_t *t2, *tu2;           // [Q][2d], [H][2d]
+    int H, Q, d;
+};
+// Workspace bytes of the primed arrays (each rounded up to 16 bytes).
+size_t lift_bytes(int H, int Q, int d);
+// Points the primed arrays of *a into ws (lift_bytes(H, Q, d) bytes, 16-byte
+// aligned) and sets its sizes; the caller sets the inputs.
+void lift_carve(void *ws, int H, int Q, int d, LiftArgs *a);
+cudaError_t launch_lift(const LiftArgs &a, cudaStream_t stream);
 
 // ---- fetch.cu
 // One host-resident index to fetch: for each of its n_channels = H*d

@@ -1,17 +1,19 @@
-// Storage side of the Fathom scan: per-channel 4-bit min/max quantisation,
-// channel-major MSB-first bit planes and exact channel statistics.
+// Storage side of the Fathom scan: per-channel b-bit min/max quantisation
+// (b = 4, or 8 for the 8-plane variant), channel-major MSB-first bit planes
+// and exact channel statistics.
 //
 // Source: Fathom explainer (papers.ananclaw.com, arXiv 2609.17652),
 // section 核心方法 / 存储侧: the K cache is quantised to 4 bits, laid out
 // channel-major, and each channel's 4 bits are split into bit planes so that
-// the first t planes of a channel are its t-bit quantiser.
+// the first t planes of a channel are its t-bit quantiser; 部署前必读 item 3:
+// an 8-bit upstream K cache needs the index adapted to 8 planes.
 //
 // Four small kernels (the index build is off the decode path):
 //   init    ordered-key min/max accumulators, zero the integer sums
 //   minmax  per (h, c) min and max over all n keys (exact, via atomics on
 //           order-preserving integer keys)
-//   range   mn and scale = (max - min) / 15 per (h, c)
-//   quant   codes -> 4 ballots per 32-key word -> plane rows staged in shared
+//   range   mn and scale = (max - min) / (2^b - 1) per (h, c)
+//   quant   codes -> b ballots per 32-key word -> plane rows staged in shared
 //           memory and written 128 bytes at a time; code sums from popcounts
 //   stats   sigma^2 = scale^2 * (n*S2 - S1^2) / n^2 in fp64
 #include "common.cuh"
@@ -62,35 +64,38 @@ __global__ void pack_minmax_kernel(const float *__restrict__ keys, int n, int d,
 }
 
 __global__ void pack_range_kernel(const uint32_t *ws_min, const uint32_t *ws_max, float *mn,
-                                  float *scale, int count)
+                                  float *scale, int count, int levels)
 {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= count) return;
     float lo = order_key_to_float(ws_min[i]);
     float hi = order_key_to_float(ws_max[i]);
     mn[i] = lo;
-    scale[i] = (hi == lo) ? 0.0f : __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    scale[i] = (hi == lo) ? 0.0f : __fdiv_rn(__fsub_rn(hi, lo), (float)levels);
 }
 
+template <int BITS>
 __device__ __forceinline__ uint32_t quantize_code(float x, float lo, float sc)
 {
+    constexpr int kLevels = (1 << BITS) - 1;
     if (sc == 0.0f) return 0u;
     float ratio = __fdiv_rn(__fsub_rn(x, lo), sc);
     float level = floorf(__fadd_rn(ratio, 0.5f));
     int v = static_cast<int>(level);
-    v = v < 0 ? 0 : (v > 15 ? 15 : v);
+    v = v < 0 ? 0 : (v > kLevels ? kLevels : v);
     return static_cast<uint32_t>(v);
 }
 
 // grid (ceil(n_words / 32), H), block 256 = 8 warps; a warp quantises one
 // 32-key word at a time (lane = key) over all d channels; dynamic shared
-// memory holds the CTA's 32-word slice of every plane row (d*4 rows).
+// memory holds the CTA's 32-word slice of every plane row (d*BITS rows).
+template <int BITS>
 __global__ void __launch_bounds__(kQuantThreads)
 pack_quant_kernel(const float *__restrict__ keys, int n, int d, int n_words,
                   const float *__restrict__ mn, const float *__restrict__ scale,
                   uint32_t *planes, int64_t *s1, int64_t *s2)
 {
-    extern __shared__ uint32_t rows[];               // [d*4][32]
+    extern __shared__ uint32_t rows[];               // [d*BITS][32]
     __shared__ unsigned long long sum1[kMaxHeadDim], sum2[kMaxHeadDim];
     const int h = blockIdx.y;
     const int w0 = blockIdx.x * kQuantWordsPerBlock;
@@ -106,25 +111,26 @@ pack_quant_kernel(const float *__restrict__ keys, int n, int d, int n_words,
         const bool live = j < n;
         const float *krow = kh + (size_t)(live ? j : 0) * d;
         for (int c = 0; c < d; ++c) {
-            uint32_t code = live ? quantize_code(krow[c], mnh[c], sch[c]) : 0u;
-            uint32_t b0 = __ballot_sync(0xFFFFFFFFu, code & 1u);
-            uint32_t b1 = __ballot_sync(0xFFFFFFFFu, code & 2u);
-            uint32_t b2 = __ballot_sync(0xFFFFFFFFu, code & 4u);
-            uint32_t b3 = __ballot_sync(0xFFFFFFFFu, code & 8u);
-            // slot s holds bit 3-s (slot 0 = most significant)
-            if (lane < 4) {
-                uint32_t word = lane == 0 ? b3 : lane == 1 ? b2 : lane == 2 ? b1 : b0;
-                rows[(c * kBits + lane) * kQuantWordsPerBlock + wl] = word;
+            const uint32_t code = live ? quantize_code<BITS>(krow[c], mnh[c], sch[c]) : 0u;
+            uint32_t b[BITS];   // b[p]: ballot of bit p
+#pragma unroll
+            for (int p = 0; p < BITS; ++p) b[p] = __ballot_sync(0xFFFFFFFFu, (code >> p) & 1u);
+            // slot s holds bit BITS-1-s (slot 0 = most significant)
+            if (lane < BITS) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int p = 0; p < BITS; ++p)
+                    if (lane == BITS - 1 - p) word = b[p];
+                rows[(c * BITS + lane) * kQuantWordsPerBlock + wl] = word;
             }
             if (lane == (c & 31)) {
                 // sum code = sum_p 2^p popc(b_p); sum code^2 = sum_{p,p'} 2^(p+p') popc(b_p & b_p')
-                const uint32_t b[4] = {b0, b1, b2, b3};
                 unsigned long long a1 = 0, a2 = 0;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
+                for (int p = 0; p < BITS; ++p) {
                     a1 += (unsigned long long)__popc(b[p]) << p;
 #pragma unroll
-                    for (int pp = 0; pp < 4; ++pp)
+                    for (int pp = 0; pp < BITS; ++pp)
                         a2 += (unsigned long long)__popc(b[p] & b[pp]) << (p + pp);
                 }
                 atomicAdd(&sum1[c], a1);
@@ -134,7 +140,7 @@ pack_quant_kernel(const float *__restrict__ keys, int n, int d, int n_words,
     }
     __syncthreads();
     // 128-byte row segments: thread -> (row, word)
-    const int n_rows = d * kBits;
+    const int n_rows = d * BITS;
     for (int e = threadIdx.x; e < n_rows * kQuantWordsPerBlock; e += blockDim.x) {
         const int row = e / kQuantWordsPerBlock, wl = e % kQuantWordsPerBlock;
         const int w = w0 + wl;
@@ -161,6 +167,7 @@ cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_
                         cudaStream_t stream)
 {
     const int H = ix.n_kv_heads, d = ix.head_dim, n = ix.n_keys, n_words = ix.n_words;
+    const int bits = index_bits(ix);
     const int count = H * d;
     uint32_t *ws_min = ws_minmax, *ws_max = ws_minmax + count;
     int *status = device_status_ptr();
@@ -169,14 +176,16 @@ cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_
     pack_init_kernel<<<eg, eb, 0, stream>>>(ws_min, ws_max, ix.sum_code, ix.sum_code2, count);
     dim3 g1((n + kMinMaxKeysPerBlock - 1) / kMinMaxKeysPerBlock, H);
     pack_minmax_kernel<<<g1, d, 0, stream>>>(keys, n, d, ws_min, ws_max, status);
-    pack_range_kernel<<<eg, eb, 0, stream>>>(ws_min, ws_max, ix.mn, ix.scale, count);
-    const size_t smem = (size_t)d * kBits * kQuantWordsPerBlock * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(pack_quant_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    pack_range_kernel<<<eg, eb, 0, stream>>>(ws_min, ws_max, ix.mn, ix.scale, count,
+                                             (1 << bits) - 1);
+    const size_t smem = (size_t)d * bits * kQuantWordsPerBlock * sizeof(uint32_t);
+    auto kern = bits == 8 ? pack_quant_kernel<8> : pack_quant_kernel<4>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     dim3 g2((n_words + kQuantWordsPerBlock - 1) / kQuantWordsPerBlock, H);
-    pack_quant_kernel<<<g2, kQuantThreads, smem, stream>>>(keys, n, d, n_words, ix.mn, ix.scale,
-                                                          ix.planes, ix.sum_code, ix.sum_code2);
+    kern<<<g2, kQuantThreads, smem, stream>>>(keys, n, d, n_words, ix.mn, ix.scale, ix.planes,
+                                              ix.sum_code, ix.sum_code2);
     note_launch(4);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return launch_channel_stats(ix, n, stream);

@@ -1,12 +1,12 @@
-// Reverse water-filling of one query by one warp (shared by the plan
-// kernels and the fused plan+scan path).
+// Reverse water-filling of one query by one warp (the plan kernels' core).
 //
 // Source: Fathom explainer (papers.ananclaw.com, arXiv 2609.17652),
 // section 核心方法 / 读侧: channels are visited in order of importance
-// w_c = q_c^2 sigma_c^2 and each takes min(4, remaining budget) bits, so with
-// rank_c the position of channel c in (w descending, channel ascending)
-// order, t_c = min(4, max(0, B - 4*rank_c)).  The fixed-width baselines
-// instead read the top-r channels by |q_c| at 4 bits.
+// w_c = q_c^2 sigma_c^2 and each takes min(b, remaining budget) bits (b = 4;
+// 8 for the 8-plane variant), so with rank_c the position of channel c in
+// (w descending, channel ascending) order, t_c = min(b, max(0, B - b*rank_c)).
+// The fixed-width baselines instead read the top-r channels by |q_c| at all
+// b bits.
 #pragma once
 
 #include "common.cuh"
@@ -54,12 +54,13 @@ __device__ __forceinline__ void warp_sort_desc(unsigned long long (&key)[E])
 
 // One warp plans query row q_row of a KV head whose channel variances are
 // sigma2_h: writes t_c to tt_row[c] for c < d (shared or global memory).
-// E = head_dim padded to a power of two, / 32.  A budget outside [0, 4d] sets
-// FATHOM_ERR_INVALID_ARG (the query reads nothing); a non-finite importance
-// (or |q|) sets FATHOM_ERR_NONFINITE (likewise).
+// E = head_dim padded to a power of two, / 32; bits = b.  A budget outside
+// [0, b*d] sets FATHOM_ERR_INVALID_ARG (the query reads nothing); a
+// non-finite importance (or |q|) sets FATHOM_ERR_NONFINITE (likewise).
 template <bool kFixed, int E>
 __device__ __forceinline__ void warp_plan(const uint16_t *q_row, const float *sigma2_h, int d,
-                                          int B, int fixed_r, uint8_t *tt_row, int *status)
+                                          int bits, int B, int fixed_r, uint8_t *tt_row,
+                                          int *status)
 {
     const int lane = threadIdx.x & 31;
     unsigned long long key[E];
@@ -82,7 +83,7 @@ __device__ __forceinline__ void warp_plan(const uint16_t *q_row, const float *si
         }
     }
     bad = __any_sync(0xFFFFFFFFu, bad);
-    if (!kFixed && (B < 0 || B > kBits * d)) {
+    if (!kFixed && (B < 0 || B > bits * d)) {
         if (lane == 0) set_status(status, FATHOM_ERR_INVALID_ARG);
         B = 0;
     }
@@ -93,7 +94,7 @@ __device__ __forceinline__ void warp_plan(const uint16_t *q_row, const float *si
         const int rank = lane * E + i;
         const uint32_t c = 0xFFFFFFFFu - (uint32_t)(key[i] & 0xFFFFFFFFull);
         if (key[i] != 0ull && c < (uint32_t)d) {
-            int tc = kFixed ? (rank < fixed_r ? kBits : 0) : min(kBits, max(0, B - kBits * rank));
+            int tc = kFixed ? (rank < fixed_r ? bits : 0) : min(bits, max(0, B - bits * rank));
             if (bad) tc = 0;
             tt_row[c] = (uint8_t)tc;
         }

@@ -26,24 +26,31 @@
  *     recorded in a per-device status word read by
  *     fathom_last_device_status().
  *   - Layouts (H = KV heads, G = query heads per KV head, Q = H*G,
- *     d = head_dim, n = keys, n_words = words per plane):
+ *     d = head_dim, n = keys, n_words = words per plane, b = bits per
+ *     stored code: 4, or 8 for the 8-plane variant):
  *       keys      float32 [H][n][d]            (token-major, as a K cache)
- *       planes    uint32  [H][d][4][n_words]   slot s holds bit 3-s of the
- *                 4-bit code (slot 0 = most significant); bit i of word w
- *                 belongs to key 32*w+i; words past the last key are zero
+ *       planes    uint32  [H][d][b][n_words]   slot s holds bit b-1-s of
+ *                 the b-bit code (slot 0 = most significant); bit i of word
+ *                 w belongs to key 32*w+i; words past the last key are zero
  *       mn, scale, sigma2  float32 [H][d]; sum_code, sum_code2 int64 [H][d]
  *       q         bfloat16 bits (uint16) [Q][d], query q served by KV head
  *                 q / G
- *       budget    int32 [Q] bits per key, 0 <= B <= 4*d
- *       t         uint8 [Q][d] bits read per channel; t_union uint8 [H][d]
+ *       budget    int32 [Q] bits per key, 0 <= B <= b*d
+ *       t         uint8 [Q][d] bits read per channel (0..b);
+ *                 t_union uint8 [H][d]
  *       bytes     uint64 [Q + H]: per query, then per KV head (union)
  *       out_idx   int32 [Q][k], out_score float32 [Q][k]: the k keys of
  *                 largest score (ties to the lower key index), listed in
  *                 ascending key index (the order a gather of their K/V rows
  *                 wants), each with its score
- *   - head_dim is a multiple of 32 and at most 256; G is 1..8;
- *     n_words is a multiple of 4 (16-byte plane rows) with 32*n_words >= n;
- *     1 <= k <= min(n, 4096).
+ *   - head_dim is a multiple of 32 and at most 256 (at most 128 when
+ *     b = 8); G is 1..8; n_words is a multiple of 4 (16-byte plane rows)
+ *     with 32*n_words >= n and 32*n_words <= 2^27 keys (2^23 when b = 8, so
+ *     that n*sum_code2 fits in 64 bits); 1 <= k <= min(n, 4096).
+ *   - The 8-plane variant (b = 8) is the adaptation the explainer's
+ *     deployment notes (部署前必读, item 3) call for when the upstream K
+ *     cache is 8-bit: the same quantiser with 255 levels, plans capped at 8
+ *     bits per channel, the same coarse-bin rebuild.
  */
 #ifndef FATHOM_H
 #define FATHOM_H
@@ -80,7 +87,9 @@ typedef enum {
 /* A packed K index of one session (one layer).  Plain descriptor; every
  * pointer is caller-owned.  planes is a device pointer (DEVICE) or a pinned,
  * device-mapped host pointer (HOST_MAPPED); the statistics are device
- * pointers. */
+ * pointers.  bits is the code width b: 4 (the 4-bit K cache) or 8 (the
+ * 8-plane variant); 0 is read as 4, so a zero-initialised field keeps the
+ * 4-bit index. */
 typedef struct {
     int32_t n_kv_heads;       /* H */
     int32_t group;            /* G query heads per KV head */
@@ -88,12 +97,13 @@ typedef struct {
     int32_t n_keys;           /* n */
     int32_t n_words;          /* words per plane */
     int32_t residency;        /* fathom_residency */
-    uint32_t *planes;         /* [H][d][4][n_words] */
+    uint32_t *planes;         /* [H][d][b][n_words] */
     float *mn;                /* [H][d] channel minimum */
-    float *scale;             /* [H][d] (max - min) / 15, 0 if max == min */
+    float *scale;             /* [H][d] (max - min) / (2^b - 1), 0 if max == min */
     float *sigma2;            /* [H][d] variance of the dequantised keys */
     int64_t *sum_code;        /* [H][d] sum of codes */
     int64_t *sum_code2;       /* [H][d] sum of squared codes */
+    int32_t bits;             /* b: 4 or 8 (0 means 4) */
 } fathom_index;
 
 /* Scan flags. */
@@ -119,12 +129,13 @@ const char *fathom_status_str(fathom_status status);
 /* Workspace bytes fathom_pack_keys needs for `index` (8*H*d). */
 size_t fathom_pack_workspace_bytes(const fathom_index *index);
 
-/* Quantise keys to 4 bits per (KV head, channel) and write the bit planes
+/* Quantise keys to b bits per (KV head, channel) and write the bit planes
  * and channel statistics into `index` (explainer, 核心方法 / 存储侧).
- * Per (h, c) over all n keys: mn = min, scale = (max-min)/15 (0 if the
- * channel is constant), code = clamp(floor((k-mn)/scale + 0.5), 0, 15) in
- * IEEE float32; sum_code, sum_code2 exact; sigma2 = scale^2*(n*S2-S1^2)/n^2
- * in fp64 rounded to float32 (the variance of the stored 4-bit keys, the
+ * Per (h, c) over all n keys: mn = min, scale = (max-min)/L with
+ * L = 2^b - 1 (0 if the channel is constant), code = clamp(floor((k-mn)/scale
+ * + 0.5), 0, L) in IEEE float32; sum_code, sum_code2 exact;
+ * sigma2 = scale^2*(n*S2-S1^2)/n^2 in fp64 rounded to float32 (the variance
+ * of the stored b-bit keys, the
  * importance weight the read side uses).
  * keys: device float32 [H][n][d].  Every output array of `index` is
  * written; planes may be a mapped host pointer (written zero-copy).
@@ -134,11 +145,11 @@ fathom_status fathom_pack_keys(const float *keys, const fathom_index *index,
                                cudaStream_t stream);
 
 /* Append m new keys per KV head at positions n..n+m-1 of an index holding
- * n = index->n_keys keys: the decode step's keys entering the 4-bit K
+ * n = index->n_keys keys: the decode step's keys entering the b-bit K
  * cache the read side scans (explainer, 核心方法 / 存储侧; the cache comes
  * from the serving stack, 适用边界).  Each new key is quantised with the
  * index's stored mn and scale exactly as fathom_pack_keys quantises, its
- * level clamped to 0..15 (a key outside the stored range takes the nearest
+ * level clamped to 0..2^b-1 (a key outside the stored range takes the nearest
  * level; a constant channel stores code 0); its bits go to key positions
  * n..n+m-1 of the planes; sum_code, sum_code2 grow by the new codes and
  * sigma2 is recomputed for n+m keys.  Keys inside the stored range give
@@ -161,12 +172,12 @@ fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t
 
 /* Reverse water-filling (explainer, 核心方法 / 读侧): for each query,
  * w_c = (q_c*q_c)*sigma2_c in float32; channels are visited by w descending
- * (ties to the lower channel) and each takes min(4, remaining budget) bits,
- * so t_c = min(4, max(0, B - 4*rank_c)) and sum_c t_c = B.  Also writes the
+ * (ties to the lower channel) and each takes min(b, remaining budget) bits,
+ * so t_c = min(b, max(0, B - b*rank_c)) and sum_c t_c = B.  Also writes the
  * GQA union t_union[h][c] = max over the G queries of KV head h, and the
  * bytes each query (and each KV head's union) reads: sum_c t_c * 4*n_words.
  * q_bf16, budget, t, t_union, bytes: device pointers.
- * A budget outside [0, 4d] sets FATHOM_ERR_INVALID_ARG in the device status
+ * A budget outside [0, b*d] sets FATHOM_ERR_INVALID_ARG in the device status
  * (that query reads nothing); a non-finite w sets FATHOM_ERR_NONFINITE. */
 fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
                           const int32_t *budget, uint8_t *t, uint8_t *t_union,
@@ -179,14 +190,14 @@ fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
  * reads its B most valuable (channel, bit) pairs, ties to the lower channel
  * then the lower bit -- the same as handing the bits out one at a time to
  * the channel of largest w_c * 4^-t_c.  Same arguments, outputs and errors
- * as fathom_plan; sum_c t_c = B and t_c <= 4. */
+ * as fathom_plan; sum_c t_c = B and t_c <= b. */
 fathom_status fathom_plan_marginal(const fathom_index *index, const uint16_t *q_bf16,
                                    const int32_t *budget, uint8_t *t, uint8_t *t_union,
                                    uint64_t *bytes, cudaStream_t stream);
 
 /* Fixed-width baseline plan (the 136-bit / 68-bit key scans the explainer
  * compares against): the r channels of largest |q_c| (ties to the lower
- * channel) are read at 4 bits, the rest at 0.  Same outputs as
+ * channel) are read at all b bits, the rest at 0.  Same outputs as
  * fathom_plan.  0 <= r <= d. */
 fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf16,
                                 int32_t r, uint8_t *t, uint8_t *t_union,
@@ -203,11 +214,20 @@ size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k);
  * and select the top-k (explainer, 核心方法 and 解决什么真问题).
  * Each KV head reads the union of its G queries' planes once; query g's
  * score of key j is
- *   s_gj = sum_c q_gc * (mn_c + scale_c*(2^(4-t)*u + (2^(4-t)-1)/2)),
- *   t = t_gc, u = code_cj >> (4-t)
+ *   s_gj = sum_c q_gc * (mn_c + scale_c*(2^(b-t)*u + (2^(b-t)-1)/2)),
+ *   t = t_gc, u = code_cj >> (b-t)
  * (the key rebuilt at the middle of its coarse t-bit bin), accumulated in
  * float32.  Outputs the k keys of largest s, ties to the lower index,
  * listed in ascending key index.
+ * An 8-plane index (b = 8) is scored as 2d nibble channels: the high and
+ * low nibbles of channel c (planes 0-3 and 4-7, which the layout already
+ * stores as two 4-plane channels) with scales 16*scale_c and scale_c and
+ * minima mn_c and 0, read to min(t, 4) and max(t - 4, 0) planes -- the
+ * same rebuilt key, since the high nibble's bin middle plus the low
+ * nibble's is the 8-bit bin middle.  This adds one small launch and
+ * (9*H + 3*Q)*2d bytes of workspace (each array rounded up to 16 bytes) for
+ * the nibble-channel arguments.
+ * All sessions of a batched call have the same b.
  * q_bf16, t, t_union, out_idx, out_score, workspace: device pointers.
  * flags: FATHOM_SCAN_* bits. */
 fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,

@@ -75,7 +75,8 @@ def test_host_resident_workspace_holds_a_plane_mirror(lib):
 
 @pytest.mark.parametrize("field,value", [("head_dim", 48), ("head_dim", 512), ("group", 9),
                                          ("group", 0), ("n_words", 6), ("n_keys", 0),
-                                         ("residency", 7)])
+                                         ("residency", 7), ("bits", 5), ("bits", 2),
+                                         ("n_words", (1 << 22) + 4)])
 def test_bad_index_shapes_are_rejected(lib, field, value):
     ix = _desc()
     setattr(ix, field, value)
@@ -156,3 +157,34 @@ def test_merge_rejects_bad_arguments_before_launching(lib):
     assert merge(fake, fake, offs(0, 100), 2, 4, 64, 129, fake, fake, None) == F    # k > S*k_s
     assert merge(fake, fake, offs(0, 10000), 2, 4, 9000, 64, fake, fake, None) == F  # too many candidates
     assert merge(None, fake, offs(0, 100), 2, 4, 64, 64, fake, fake, None) == F
+
+
+def test_eight_plane_index_sizes_and_limits(lib):
+    """An 8-plane index scans as 2d nibble channels of 4 planes: its workspace
+    is that of a 4-plane index of head_dim 2d plus the nibble-channel
+    arguments (mn', scale' float [H][2d], q' bf16 [Q][2d], t' [Q][2d],
+    t_union' [H][2d], each rounded up to 16 bytes)."""
+    for H, G, d, n, res in ((2, 4, 128, 4096, 0), (8, 4, 128, 1 << 20, 0), (1, 1, 32, 100, 1)):
+        ix8 = _desc(H=H, G=G, d=d, n=n, residency=res)
+        ix8.bits = 8
+        ix4 = _desc(H=H, G=G, d=2 * d, n=n, residency=res)
+        a16 = lambda b: (b + 15) // 16 * 16
+        Q, d2 = H * G, 2 * d
+        lift = 2 * a16(H * d2 * 4) + a16(Q * d2 * 2) + a16(Q * d2) + a16(H * d2)
+        assert fp.fathom_scan_workspace_bytes(ix8, 64) == \
+            fp.fathom_scan_workspace_bytes(ix4, 64) + lift
+        assert fp.fathom_pack_workspace_bytes(ix8) == 8 * H * d
+    wide = _desc(d=256)
+    wide.bits = 8                              # 2d = 512 nibble channels: too wide
+    assert fp.fathom_scan_workspace_bytes(wide, 64) == 0
+    long8 = _desc(n=(1 << 23) + 128)
+    long8.bits = 8                             # n * sum_code2 would overflow int64
+    assert fp.fathom_scan_workspace_bytes(long8, 64) == 0
+    long8.bits = 4
+    assert fp.fathom_scan_workspace_bytes(long8, 64) > 0
+    a, b = _desc(), _desc()
+    b.bits = 8                                 # one batch, one code width
+    assert fp.fathom_scan_batched_workspace_bytes([a, b], 64) == 0
+    a.bits = 8
+    assert fp.fathom_scan_batched_workspace_bytes([a, b], 64) == \
+        2 * fp.fathom_scan_workspace_bytes(b, 64)
