@@ -49,6 +49,7 @@ def _load():
             "fo_unpack_planes": ([P, I, I, I, I, I, P], ctypes.c_int),
             "fo_append": ([P, I, I, I, I, I, I, P, P, P, P, P, P, P], ctypes.c_int),
             "fo_channel_stats": ([P, I, I, I, P, P, P, P], ctypes.c_int),
+            "fo_blocked_sigma2": ([P, P, P, P, I, I, I, P], ctypes.c_int),
             "fo_importance": ([P, P, I, P], ctypes.c_int),
             "fo_plan_greedy": ([P, I, I, I, P], ctypes.c_int),
             "fo_plan_marginal": ([P, I, I, I, P], ctypes.c_int),
@@ -153,6 +154,23 @@ def channel_stats(codes: np.ndarray, scale: np.ndarray):
     _check(_load().fo_channel_stats(_p(codes), H, n, d, _p(scale), _p(s1), _p(s2),
                                     _p(sigma2)), "channel_stats")
     return s1, s2, sigma2
+
+
+def blocked_sigma2(mn_h, scale_h, s1_h, s2_h, n: int, block: int) -> np.ndarray:
+    """sigma^2 [d] of one KV head of a block-scaled index: the variance of
+    all n dequantised keys from the blocks' sums (mn_h ... s2_h [nb][d])."""
+    mn_h = np.ascontiguousarray(mn_h, np.float32)
+    d = mn_h.shape[-1]
+    out = np.empty(d, np.float32)
+    _check(_load().fo_blocked_sigma2(_p(mn_h), _p(np.ascontiguousarray(scale_h, np.float32)),
+                                     _p(np.ascontiguousarray(s1_h, np.int64)),
+                                     _p(np.ascontiguousarray(s2_h, np.int64)), d, int(n),
+                                     int(block), _p(out)), "blocked_sigma2")
+    return out
+
+
+def n_blocks_for(n: int, block: int) -> int:
+    return (n + block - 1) // block
 
 
 # ------------------------------------------------------------------- read side
@@ -265,16 +283,68 @@ def recall(selected, reference) -> float:
 
 # --------------------------------------------------------------- whole pipeline
 def build_index(keys: np.ndarray, capacity: Optional[int] = None,
-                bits: int = 4) -> Dict[str, np.ndarray]:
+                bits: int = 4, block_keys: int = 0) -> Dict[str, np.ndarray]:
     """Storage side for one session: quantise, pack, channel statistics.
     capacity: keys the planes can hold (for appends); default n.
-    bits: planes per channel (4, or 8 for an 8-bit K cache)."""
-    mn, scale, codes = quantize(keys, bits)
+    bits: planes per channel (4, or 8 for an 8-bit K cache).
+    block_keys: 0 for one scale per channel over all keys; else grouped
+    per-token-block scales, each block of block_keys tokens quantised on
+    its own (mn, scale, s1, s2 then hold [H][n_blocks][d], n_blocks counted
+    over the capacity; blocks past the keys stay zero)."""
     n = keys.shape[1]
-    planes = pack_planes(codes, n_words_for(max(n, capacity or n)), bits)
-    s1, s2, sigma2 = channel_stats(codes, scale)
+    n_words = n_words_for(max(n, capacity or n))
+    if not block_keys:
+        mn, scale, codes = quantize(keys, bits)
+        planes = pack_planes(codes, n_words, bits)
+        s1, s2, sigma2 = channel_stats(codes, scale)
+        return dict(mn=mn, scale=scale, codes=codes, planes=planes, s1=s1, s2=s2,
+                    sigma2=sigma2, n=n, n_words=n_words, bits=int(bits), block_keys=0)
+    H, _, d = keys.shape
+    nb_cap = n_blocks_for(32 * n_words, block_keys)
+    mn = np.zeros((H, nb_cap, d), np.float32)
+    scale = np.zeros_like(mn)
+    s1 = np.zeros((H, nb_cap, d), np.int64)
+    s2 = np.zeros_like(s1)
+    codes = np.empty((H, d, n), np.uint8)
+    for b in range(n_blocks_for(n, block_keys)):
+        j0, j1 = b * block_keys, min(n, (b + 1) * block_keys)
+        mn[:, b], scale[:, b], codes[:, :, j0:j1] = quantize(keys[:, j0:j1], bits)
+        s1[:, b], s2[:, b], _ = channel_stats(codes[:, :, j0:j1], scale[:, b])
+    planes = pack_planes(codes, n_words, bits)
+    sigma2 = np.stack([blocked_sigma2(mn[h], scale[h], s1[h], s2[h], n, block_keys)
+                       for h in range(H)])
     return dict(mn=mn, scale=scale, codes=codes, planes=planes, s1=s1, s2=s2,
-                sigma2=sigma2, n=n, n_words=planes.shape[-1], bits=int(bits))
+                sigma2=sigma2, n=n, n_words=n_words, bits=int(bits), block_keys=int(block_keys))
+
+
+def append_blocks(index: Dict[str, np.ndarray], keys: np.ndarray) -> int:
+    """Append keys float32 [H][m][d] to a block-scaled index whose key count
+    is a whole number of blocks: each new block is quantised on its own, as
+    packing all keys would.  Returns the new key count."""
+    block = index["block_keys"]
+    n = index["n"]
+    assert block and n % block == 0, "appends start a new block"
+    H, m, d = keys.shape
+    bits, n_words = index["planes"].shape[-2:]
+    assert n + m <= 32 * n_words
+    new_codes = np.empty((H, d, m), np.uint8)
+    for i0 in range(0, m, block):
+        b = (n + i0) // block
+        i1 = min(m, i0 + block)
+        mb, sb, cb = quantize(keys[:, i0:i1], bits)
+        index["mn"][:, b], index["scale"][:, b] = mb, sb
+        index["s1"][:, b], index["s2"][:, b], _ = channel_stats(cb, sb)
+        new_codes[:, :, i0:i1] = cb
+    words = pack_planes(new_codes, None, bits)
+    w0 = n // 32
+    nw = min(words.shape[-1], n_words - w0)
+    index["planes"][..., w0:w0 + nw] |= words[..., :nw]
+    index["n"] = n + m
+    index["codes"] = np.concatenate([index["codes"], new_codes], axis=2)
+    for h in range(H):
+        index["sigma2"][h] = blocked_sigma2(index["mn"][h], index["scale"][h], index["s1"][h],
+                                            index["s2"][h], n + m, block)
+    return n + m
 
 
 def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
@@ -298,11 +368,32 @@ def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
     return t, T, nb
 
 
+def _head_blocks(index, h: int):
+    """(key range, planes, mn, scale) of each scale block of KV head h."""
+    n, block = index["n"], index.get("block_keys", 0)
+    if not block:
+        return [((0, n), index["planes"][h], index["mn"][h], index["scale"][h])]
+    out = []
+    for b in range(n_blocks_for(n, block)):
+        j0, j1 = b * block, min(n, (b + 1) * block)
+        out.append(((j0, j1), np.ascontiguousarray(index["planes"][h][..., j0 // 32:]),
+                    index["mn"][h, b], index["scale"][h, b]))
+    return out
+
+
+def score_head(index, h: int, q_bf16_row, t_row, absolute: bool = False) -> np.ndarray:
+    """Scores [n] of one query against KV head h from its plan t (each key
+    with the scales of its block); absolute=True gives sum_c |q_c khat_cj|."""
+    fn = score_abs_planes if absolute else score_planes
+    parts = [fn(planes, mn, sc, q_bf16_row, t_row, j1 - j0)
+             for (j0, j1), planes, mn, sc in _head_blocks(index, h)]
+    return np.concatenate(parts)
+
+
 def scan_query(index, q_bf16_row, t_row, h: int, k: int):
     """Score one query against KV head h and select its top-k.
-    -> (idx [k], top scores [k], all scores [n], abs sums [n])."""
-    n = index["n"]
-    s = score_planes(index["planes"][h], index["mn"][h], index["scale"][h], q_bf16_row, t_row, n)
+    -> (idx [k], top scores [k], all scores [n])."""
+    s = score_head(index, h, q_bf16_row, t_row)
     idx, top = topk(s, k)
     return idx, top, s
 

@@ -222,6 +222,47 @@ int fo_channel_stats(const uint8_t *codes, int64_t H, int64_t n, int64_t d,
     return FO_OK;
 }
 
+/* Grouped per-token-block scales: the keys of a channel are cut into
+ * blocks of `block` tokens, each quantised on its own (its own mn, scale,
+ * S1, S2; the last block may hold fewer keys), the grouping quantised K
+ * caches of serving stacks use (the explainer, 亮点 and 适用边界: the index
+ * is the serving stack's quantised K).  sigma^2 stays one number per
+ * channel: the population variance of all n dequantised keys, combined
+ * from the blocks' exact sums in fp64, block by block in order, with the
+ * pairwise update of Chan, Golub and LeVeque (1979):
+ *   mean_b = mn_b + scale_b * (S1_b / n_b)
+ *   M2_b   = (scale_b * scale_b) * ((n_b*S2_b - S1_b^2) / n_b)
+ *   N' = N + n_b;  delta = mean_b - mean;  mean += delta * (n_b / N');
+ *   M2 += M2_b + (delta * delta) * ((N * n_b) / N');  N = N'
+ *   sigma^2 = (float)(M2 / n).
+ * mn, scale float [nb][d]; s1, s2 int64 [nb][d] of one KV head;
+ * sigma2 float [d]. */
+int fo_blocked_sigma2(const float *mn, const float *scale, const int64_t *s1, const int64_t *s2,
+                      int64_t d, int64_t n, int64_t block, float *sigma2)
+{
+    if (d <= 0 || n <= 0 || block <= 0) return FO_ERR_ARG;
+    const int64_t nb = (n + block - 1) / block;
+    for (int64_t c = 0; c < d; ++c) {
+        double N = 0.0, mean = 0.0, M2 = 0.0;
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t nbk = (b + 1) * block <= n ? block : n - b * block;
+            const int64_t i = b * d + c;
+            const double nbd = (double)nbk;
+            const double sc = (double)scale[i];
+            const double mean_b = (double)mn[i] + sc * ((double)s1[i] / nbd);
+            const int64_t num = nbk * s2[i] - s1[i] * s1[i];
+            const double m2_b = (sc * sc) * ((double)num / nbd);
+            const double Nn = N + nbd;
+            const double delta = mean_b - mean;
+            mean = mean + delta * (nbd / Nn);
+            M2 = M2 + m2_b + (delta * delta) * ((N * nbd) / Nn);
+            N = Nn;
+        }
+        sigma2[c] = (float)(M2 / (double)n);
+    }
+    return FO_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* Read side: importance, reverse water-filling, union, bytes.          */
 /* ------------------------------------------------------------------ */

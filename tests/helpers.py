@@ -15,9 +15,8 @@ def to_np_u32(t):
 
 def oracle_query(ix, q_row, t_row, h, k):
     """-> (idx, top, all scores, abs sums) of one query against KV head h."""
-    n = ix["n"]
-    s = oracle.score_planes(ix["planes"][h], ix["mn"][h], ix["scale"][h], q_row, t_row, n)
-    a = oracle.score_abs_planes(ix["planes"][h], ix["mn"][h], ix["scale"][h], q_row, t_row, n)
+    s = oracle.score_head(ix, h, q_row, t_row)
+    a = oracle.score_head(ix, h, q_row, t_row, absolute=True)
     idx, top = oracle.topk(s, k)
     return idx, top, s, a
 

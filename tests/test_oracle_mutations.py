@@ -47,6 +47,10 @@ MUTATIONS = {
                              "for (int p = 0; p < bits && p < 4; ++p)\n                    v |="),
     "midpoint_of_4bit_bins": ("double level = (double)(width * u) + (double)(width - 1) / 2.0;",
                               "double level = (double)(width * u) + (double)((width < 16 ? width : 16) - 1) / 2.0;"),
+    "blocked_sigma2_no_between_block_term": (
+        "M2 = M2 + m2_b + (delta * delta) * ((N * nbd) / Nn);", "M2 = M2 + m2_b;"),
+    "blocked_sigma2_mean_ignores_min": ("const double mean_b = (double)mn[i] + sc *",
+                                        "const double mean_b = 0.0 + sc *"),
     "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
                                "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
 }
@@ -79,6 +83,8 @@ PIN_TESTS = [
     lambda: pins.test_plan_8bit_is_optimal_by_brute_force(2),
     pins.test_fixed_plan_8bit_reads_whole_channels,
     pins.test_append_8bit_in_range_equals_repacking_and_clamps,
+    pins.test_blocked_sigma2_is_the_variance_of_all_dequantised_keys,
+    pins.test_blocks_as_large_as_the_keys_are_the_global_quantiser,
 ]
 
 

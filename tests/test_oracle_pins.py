@@ -671,3 +671,114 @@ def test_append_8bit_in_range_equals_repacking_and_clamps():
     clamped = np.zeros((1, 1), np.uint32)
     oracle.append(ix, np.array([[[-3.0], [300.0], [17.4]]], np.float32), clamped)
     assert list(ix["codes"][0, 0, 256:]) == [0, 255, 17] and clamped[0, 0] == 2
+
+
+# ------------------------------------------- grouped per-token-block scales
+# Reading: the keys of each channel are cut into blocks of block_keys tokens
+# and each block is quantised on its own, as grouped quantised K caches of
+# serving stacks are (the explainer's index is the serving stack's quantised
+# K, 亮点 / 适用边界); sigma^2 stays the variance of all dequantised keys.
+def _drifting_keys(seed, H, n, d, shift_every, shift):
+    """Keys whose channel means move by `shift` every `shift_every` tokens."""
+    ses = synth.make_session(seed, H, 2, n, 64, head_dim=d)
+    keys = ses.keys.copy()
+    keys += (np.arange(n) // shift_every)[None, :, None].astype(np.float32) * np.float32(shift)
+    return ses, keys
+
+
+def test_blocks_as_large_as_the_keys_are_the_global_quantiser():
+    ses = synth.make_session(31, 2, 2, 3000, 64)
+    g = oracle.build_index(ses.keys)
+    b = oracle.build_index(ses.keys, block_keys=4096)
+    assert b["mn"].shape == (2, 1, 128)
+    for name in ("planes", "codes"):
+        assert np.array_equal(g[name], b[name])
+    for name in ("mn", "scale", "s1", "s2"):
+        assert np.array_equal(g[name], b[name][:, 0]), name
+    np.testing.assert_allclose(b["sigma2"], g["sigma2"], rtol=1e-6)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_block_quantiser_error_bound_and_extremes_per_block(bits):
+    """Every key is within half a step of its level, the step being its own
+    block's range / (2^b - 1) (numpy min/max per block); each block's min key
+    maps to level 0 and its max to the top level."""
+    n, block, top = 5000, 2048, (1 << bits) - 1
+    _, keys = _drifting_keys(32, 2, n, 16, 1000, 3.0)
+    ix = oracle.build_index(keys, block_keys=block, bits=bits)
+    for b in range(3):
+        j0, j1 = b * block, min(n, (b + 1) * block)
+        kb = keys[:, j0:j1].transpose(0, 2, 1).astype(np.float64)      # [H][d][nb]
+        lo, hi = kb.min(axis=2), kb.max(axis=2)
+        step = (hi - lo) / top
+        np.testing.assert_allclose(ix["mn"][:, b], lo, rtol=0, atol=0)
+        np.testing.assert_allclose(ix["scale"][:, b], step, rtol=1e-6)
+        cb = ix["codes"][:, :, j0:j1]
+        deq = lo[..., None] + ix["scale"][:, b][..., None].astype(np.float64) * cb
+        assert np.all(np.abs(deq - kb) <= step[..., None] * (0.5 + 1e-4) + 1e-6)
+        assert np.all(np.take_along_axis(cb, np.argmin(kb, 2)[..., None], 2) == 0)
+        assert np.all(np.take_along_axis(cb, np.argmax(kb, 2)[..., None], 2) == top)
+
+
+def _dequantised_blocked(ix, h):
+    n, block = ix["n"], ix["block_keys"]
+    blk = np.arange(n) // block
+    mn = ix["mn"][h][blk].T.astype(np.float64)          # [d][n]
+    sc = ix["scale"][h][blk].T.astype(np.float64)
+    return mn + sc * ix["codes"][h]
+
+
+def test_blocked_sigma2_is_the_variance_of_all_dequantised_keys():
+    """Drifting means make the between-block term large: numpy's two-pass
+    variance over all keys (a different algorithm) must agree."""
+    _, keys = _drifting_keys(33, 2, 7000, 32, 2048, 2.5)
+    ix = oracle.build_index(keys, block_keys=2048)
+    for h in range(2):
+        ref = _dequantised_blocked(ix, h).var(axis=1)
+        np.testing.assert_allclose(ix["sigma2"][h], ref, rtol=1e-6)
+    # a block's own variance alone would miss the drift
+    within = ix["sigma2"][0] / _dequantised_blocked(ix, 0)[:, :2048].var(axis=1)
+    assert np.median(within) > 1.5
+
+
+def test_blocked_scores_full_zero_and_prefix_depths():
+    ses, keys = _drifting_keys(34, 1, 5000, 128, 1500, 1.0)
+    ix = oracle.build_index(keys, block_keys=2048)
+    deq = _dequantised_blocked(ix, 0)
+    q = ses.q_bf16[0]
+    qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+    full = oracle.score_head(ix, 0, q, np.full(128, 4, np.uint8))
+    assert np.all(np.abs(full - qf @ deq) <= 1e-13 * (np.abs(qf) @ np.abs(deq)))
+    zero = oracle.score_head(ix, 0, q, np.zeros(128, np.uint8))
+    blk = np.arange(5000) // 2048
+    const = np.array([qf @ (ix["mn"][0, b].astype(np.float64) +
+                            7.5 * ix["scale"][0, b].astype(np.float64)) for b in range(3)])
+    np.testing.assert_allclose(zero, const[blk], rtol=1e-13)
+    assert len(np.unique(zero)) == 3                      # one constant per block
+    t = np.random.default_rng(5).integers(0, 5, size=128).astype(np.uint8)
+    by_codes = np.concatenate([
+        oracle.score_codes(np.ascontiguousarray(ix["codes"][0][:, j0:j0 + 2048]),
+                           ix["mn"][0, b], ix["scale"][0, b], q, t)
+        for b, j0 in enumerate(range(0, 5000, 2048))])
+    assert np.array_equal(oracle.score_head(ix, 0, q, t), by_codes)
+
+
+def test_blocked_append_of_whole_blocks_equals_packing_everything():
+    _, keys = _drifting_keys(35, 2, 2048 * 3 + 500, 16, 2048, 4.0)
+    ix = oracle.build_index(keys[:, :4096], capacity=keys.shape[1], block_keys=2048)
+    oracle.append_blocks(ix, keys[:, 4096:])
+    full = oracle.build_index(keys, capacity=keys.shape[1], block_keys=2048)
+    for name in ("planes", "mn", "scale", "s1", "s2", "sigma2", "codes"):
+        assert np.array_equal(ix[name], full[name]), name
+
+
+def test_blocks_follow_a_drifting_key_range():
+    """What the grouping is for: when the keys drift, per-block scales keep the
+    quantisation error near one block's range instead of the whole range."""
+    _, keys = _drifting_keys(36, 1, 8192, 32, 2048, 6.0)
+    g = oracle.build_index(keys)
+    b = oracle.build_index(keys, block_keys=2048)
+    k = keys[0].T.astype(np.float64)
+    err_g = np.abs(g["mn"][0][:, None] + g["scale"][0][:, None].astype(np.float64) * g["codes"][0] - k)
+    err_b = np.abs(_dequantised_blocked(b, 0) - k)
+    assert err_b.mean() < 0.5 * err_g.mean()
