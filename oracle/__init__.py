@@ -350,7 +350,7 @@ def append_blocks(index: Dict[str, np.ndarray], keys: np.ndarray) -> int:
 def plan_session(index, q_bf16: np.ndarray, budgets: np.ndarray, group: int,
                  fixed_r: Optional[int] = None, marginal: bool = False):
     """-> (t uint8 [Q][d], T uint8 [H][d], bytes uint64 [Q+H])."""
-    H, d = index["mn"].shape
+    H, d = index["sigma2"].shape
     bits = index["planes"].shape[-2]
     Q = H * group
     t = np.empty((Q, d), np.uint8)

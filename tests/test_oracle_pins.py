@@ -782,3 +782,14 @@ def test_blocks_follow_a_drifting_key_range():
     err_g = np.abs(g["mn"][0][:, None] + g["scale"][0][:, None].astype(np.float64) * g["codes"][0] - k)
     err_b = np.abs(_dequantised_blocked(b, 0) - k)
     assert err_b.mean() < 0.5 * err_g.mean()
+
+
+def test_plans_of_a_blocked_index_use_its_channel_variance():
+    """The read side sees one sigma^2 per channel whatever the grouping."""
+    ses, keys = _drifting_keys(37, 2, 5000, 32, 2048, 2.0)
+    ix = oracle.build_index(keys, block_keys=2048)
+    t, T, nb = oracle.plan_session(ix, ses.q_bf16, np.full(4, 40), 2)
+    for q in range(4):
+        w = oracle.importance(ses.q_bf16[q], ix["sigma2"][q // 2])
+        assert np.array_equal(t[q], oracle.plan_greedy(w, 40))
+    assert T.shape == (2, 32) and int(nb[0]) == 40 * oracle.n_words_for(5000) * 4
