@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fathom|reference]
                     [--workload qwen3_8b_layer_128k|qwen3_8b_layer_128k_8plane|
+                               qwen3_8b_layer_128k_blocked|
                                plan_variants_128k|host_1m|host_256k|fixed_vs_wf_1m|
                                agent_16_sessions|append_layer_128k|
                                attention_layer_128k]
@@ -50,7 +51,9 @@ L2_FLUSH_BYTES = 256 << 20
 # plans: ("wf", B) = reverse water-filling at B bits per key; ("mg", B) = the
 # marginal-gain variant; ("fixed", r) = the top-r channels by |q_c| at all
 # b bits.  "bits": b, the stored code width (4 unless given; 8 = the 8-plane
-# variant for an 8-bit K cache).  "device_keys": keys drawn on the GPU
+# variant for an 8-bit K cache).  "block_keys": grouped per-token-block
+# scales over blocks of that many tokens (0 unless given).  "device_keys":
+# keys drawn on the GPU
 # (synth.device_keys) instead of numpy, for sizes numpy would take minutes
 # on.  agent_16_sessions scans its sessions in one batched call.
 WORKLOADS = {
@@ -59,6 +62,10 @@ WORKLOADS = {
     # the same layer with an 8-bit K cache (8 planes per channel), same budgets
     "qwen3_8b_layer_128k_8plane": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
                                        bits=8, plans=(("wf", 68), ("wf", 92), ("wf", 136))),
+    # the same layer with grouped per-token-block scales (blocks of 2048 keys)
+    "qwen3_8b_layer_128k_blocked": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
+                                        block_keys=2048,
+                                        plans=(("wf", 68), ("wf", 92), ("wf", 136))),
     "host_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
                     plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
     # the host path at a quarter of the keys: the profiling case of the fetch
@@ -132,7 +139,8 @@ def config_of(wl_name, wl, flush_note, sessions=None):
     c = {"workload": wl_name, "kv_heads": wl["H"], "query_heads_per_kv": wl["G"],
          "head_dim": wl["d"], "k": wl["k"],
          "residency": "hbm" if wl["residency"] == "device" else "host_pinned_mapped",
-         "code_bits": wl.get("bits", 4), "l2": flush_note}
+         "code_bits": wl.get("bits", 4), "scale_block_keys": wl.get("block_keys", 0),
+         "l2": flush_note}
     if sessions is None:
         c["n_keys"] = wl["n"]
         c["plans"] = [plan_name(p) for p in wl["plans"]]
@@ -221,7 +229,8 @@ def measure_host_link(fp, torch, nbytes=1 << 30, reps=10):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bits=4):
+def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bits=4,
+                  block_keys=0):
     """Time the oracle (plan + fp64 score + full-sort top-k per query) over
     the given KV heads' keys (float32 [h][n][d]) at every plan spec, cycling
     over (head, plan) until at least min_seconds have passed (one round at
@@ -229,7 +238,7 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bi
     timed.  Returns (seconds, head-scans, keys)."""
     import oracle
     if ref is None:
-        ref = oracle.build_index(keys_heads, bits=bits)
+        ref = oracle.build_index(keys_heads, bits=bits, block_keys=block_keys)
     n = keys_heads.shape[1]
     pairs = [(hi, spec) for hi in range(keys_heads.shape[0]) for spec in plans]
     t0 = time.perf_counter()
@@ -246,8 +255,7 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bi
                                           bits)
             else:
                 tq = oracle.fixed_plan(qrow, spec[1], bits)
-            s = oracle.score_planes(ref["planes"][hi], ref["mn"][hi], ref["scale"][hi],
-                                    qrow, tq, n)
+            s = oracle.score_head(ref, hi, qrow, tq)
             oracle.topk(s, k)
         scans += 1
     return time.perf_counter() - t0, scans, scans * n
@@ -256,10 +264,11 @@ def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bi
 CPU_BASELINE_SECONDS = 12.0
 
 
-def cpu_baseline(keys_heads, q_bf16, G, plans, k, bits=4):
+def cpu_baseline(keys_heads, q_bf16, G, plans, k, bits=4, block_keys=0):
     """About 12 s of single-thread oracle work on a few KV heads."""
     secs, scans, keys = oracle_sample(keys_heads, q_bf16, G, plans, k,
-                                      min_seconds=CPU_BASELINE_SECONDS, bits=bits)
+                                      min_seconds=CPU_BASELINE_SECONDS, bits=bits,
+                                      block_keys=block_keys)
     return {"value": keys / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{scans} scans of one KV head ({G} query heads, {keys_heads.shape[1]} "
                       f"keys) cycling over {keys_heads.shape[0]} KV head(s) x plans "
@@ -281,7 +290,7 @@ def run_reference(args, wl_name, wl):
     bits = wl.get("bits", 4)
     ses = synth.make_session(0, 1, wl["G"], n, plan_bits(plans[0], bits), head_dim=wl["d"])
     import oracle
-    ref = oracle.build_index(ses.keys[:1], bits=bits)
+    ref = oracle.build_index(ses.keys[:1], bits=bits, block_keys=wl.get("block_keys", 0))
     times = []
     for i in range(args.warmup + args.steps):
         secs, _, _ = oracle_sample(ses.keys[:1], ses.q_bf16, wl["G"], (plans[i % len(plans)],),
@@ -379,7 +388,8 @@ def build_sessions(wl, rank, torch, fp):
         else:
             ses = synth.make_session(p["seed"], H, G, p["n"], 64, head_dim=d)
             keys = torch.from_numpy(ses.keys).cuda()
-        index = fp.KeyIndex(H, G, p["n"], d, wl["residency"], bits=wl.get("bits", 4))
+        index = fp.KeyIndex(H, G, p["n"], d, wl["residency"], bits=wl.get("bits", 4),
+                            block_keys=wl.get("block_keys", 0))
         index.pack(keys)
         plans = wl["plans"] if wl.get("plans") else (("wf", p["budget"]),)
         out.append(dict(n=p["n"], budget=p["budget"], keys=keys, index=index, plans=plans))
@@ -605,7 +615,8 @@ def run_fathom(args, wl_name, wl):
         nh = max(1, min(H, (8 * 131072) // S0["n"]))
         line["cpu_baseline"] = cpu_baseline(S0["keys"][:nh].cpu().numpy(),
                                             S0["q"][0].cpu().numpy().view(np.uint16), G,
-                                            S0["plans"], k, wl.get("bits", 4))
+                                            S0["plans"], k, wl.get("bits", 4),
+                                            wl.get("block_keys", 0))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -58,6 +58,7 @@ class fathom_index(ctypes.Structure):
         ("planes", ctypes.c_void_p), ("mn", ctypes.c_void_p), ("scale", ctypes.c_void_p),
         ("sigma2", ctypes.c_void_p), ("sum_code", ctypes.c_void_p),
         ("sum_code2", ctypes.c_void_p), ("bits", ctypes.c_int32),
+        ("block_keys", ctypes.c_int32),
     ]
 
 
@@ -285,14 +286,19 @@ class KeyIndex:
     residency "device" keeps the planes in HBM; "host_mapped" keeps them in
     pinned host memory read zero-copy by the scan.  Statistics stay on the
     device either way.  bits: 4 (the 4-bit K cache) or 8 (the 8-plane
-    variant for an 8-bit K cache)."""
+    variant for an 8-bit K cache).  block_keys: 0 for one scale per channel,
+    or grouped per-token-block scales over blocks of that many tokens (a
+    multiple of 2048); mn, scale, sum_code and sum_code2 are then
+    [H][n_blocks][d] with n_blocks counted over the capacity."""
 
     def __init__(self, n_kv_heads: int, group: int, n_keys: int, head_dim: int = 128,
                  residency: str = "device", device: Optional[int] = None,
-                 capacity: Optional[int] = None, bits: int = 4):
+                 capacity: Optional[int] = None, bits: int = 4, block_keys: int = 0):
         import torch
         if bits not in (4, 8):
             raise ValueError(f"bits must be 4 or 8, not {bits}")
+        if block_keys < 0 or block_keys % 2048:
+            raise ValueError(f"block_keys must be 0 or a multiple of 2048, not {block_keys}")
         dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
         self.n_words = fathom_n_words(max(n_keys, capacity or n_keys))
         H, d = n_kv_heads, head_dim
@@ -305,16 +311,20 @@ class KeyIndex:
             res = FATHOM_RES_HOST_MAPPED
         else:
             raise ValueError(f"unknown residency {residency!r}")
-        self.mn = torch.empty((H, d), dtype=torch.float32, device=dev)
+        stat = (H, d)
+        if block_keys:
+            stat = (H, -(-32 * self.n_words // block_keys), d)
+        self.mn = torch.empty(stat, dtype=torch.float32, device=dev)
         self.scale = torch.empty_like(self.mn)
-        self.sigma2 = torch.empty_like(self.mn)
-        self.sum_code = torch.empty((H, d), dtype=torch.int64, device=dev)
+        self.sigma2 = torch.empty((H, d), dtype=torch.float32, device=dev)
+        self.sum_code = torch.empty(stat, dtype=torch.int64, device=dev)
         self.sum_code2 = torch.empty_like(self.sum_code)
         self.residency = residency
         self.desc = fathom_index(H, group, d, n_keys, self.n_words, res,
                                  self.planes.data_ptr(), self.mn.data_ptr(),
                                  self.scale.data_ptr(), self.sigma2.data_ptr(),
-                                 self.sum_code.data_ptr(), self.sum_code2.data_ptr(), bits)
+                                 self.sum_code.data_ptr(), self.sum_code2.data_ptr(), bits,
+                                 block_keys)
         self.device = dev
 
     @property
@@ -336,6 +346,10 @@ class KeyIndex:
     @property
     def bits(self):
         return self.desc.bits
+
+    @property
+    def block_keys(self):
+        return self.desc.block_keys
 
     @property
     def capacity(self):

@@ -68,6 +68,8 @@ bool index_shape_ok(const fathom_index *ix)
     if ((long long)ix->n_words * 32 < (long long)ix->n_keys) return false;
     if (ix->residency != FATHOM_RES_DEVICE && ix->residency != FATHOM_RES_HOST_MAPPED) return false;
     if (ix->bits != 0 && ix->bits != 4 && ix->bits != 8) return false;
+    // grouped scales: blocks of whole 2048-key scan tiles
+    if (ix->block_keys < 0 || ix->block_keys % kTileKeys) return false;
     const int bits = index_bits(*ix);
     // 8 planes: the scan's 2d nibble channels fit its head_dim limit
     if (bits == 8 && 2 * ix->head_dim > kMaxHeadDim) return false;
@@ -105,10 +107,12 @@ size_t scan_part_bytes(const fathom_index *sessions, int n_sessions, int k)
 size_t scan_total_bytes(const fathom_index *sessions, int n_sessions, int k)
 {
     size_t total = scan_part_bytes(sessions, n_sessions, k);
-    for (int s = 0; s < n_sessions; ++s)
-        if (index_bits(sessions[s]) == 8)
-            total += lift_bytes(sessions[s].n_kv_heads, sessions[s].n_kv_heads * sessions[s].group,
-                                sessions[s].head_dim);
+    for (int s = 0; s < n_sessions; ++s) {
+        const fathom_index &ix = sessions[s];
+        if (index_bits(ix) == 8)
+            total += lift_bytes(ix.n_kv_heads, ix.n_kv_heads * ix.group, ix.head_dim,
+                                ix.n_kv_heads * index_blocks(ix));
+    }
     return total;
 }
 
@@ -174,7 +178,8 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
         const fathom_index *ix = &sessions[s];
         if (!index_shape_ok(ix) || !ix->mn || !ix->scale) return FATHOM_ERR_INVALID_ARG;
         if (ix->head_dim != sessions[0].head_dim || ix->group != sessions[0].group ||
-            index_bits(*ix) != index_bits(sessions[0]))
+            index_bits(*ix) != index_bits(sessions[0]) ||
+            (ix->block_keys != 0) != (sessions[0].block_keys != 0))
             return FATHOM_ERR_INVALID_ARG;
         if (k > ix->n_keys) return FATHOM_ERR_INVALID_ARG;
         if (!q[s] || !t[s] || !tu[s] || !out_idx[s] || !out_score[s]) return FATHOM_ERR_INVALID_ARG;
@@ -193,14 +198,15 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
         for (int s = 0; s < n_sessions; ++s) {
             const fathom_index &ix = sessions[s];
             const int H = ix.n_kv_heads, Q = H * ix.group, d = ix.head_dim;
+            const int rows = H * index_blocks(ix);
             LiftArgs la{};
             la.mn = ix.mn;
             la.scale = ix.scale;
             la.q = q[s];
             la.t = t[s];
             la.tu = tu[s];
-            lift_carve(at, H, Q, d, &la);
-            at += lift_bytes(H, Q, d);
+            lift_carve(at, H, Q, d, rows, &la);
+            at += lift_bytes(H, Q, d, rows);
             const cudaError_t e = launch_lift(la, stream);
             if (e != cudaSuccess) return cuda_status(note_error(e, "lift"));
             resolved[s].mn = la.mn2;
@@ -311,7 +317,13 @@ fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t
     fathom_index ix = *index;
     fathom_status st = resolve_planes(index, &ix.planes);
     if (st != FATHOM_OK) return st;
-    st = cuda_status(launch_append(keys, ix, m, clamped, stream));
+    if (ix.block_keys) {
+        // grouped scales: new keys open new blocks, each quantised on its own
+        if (ix.n_keys % ix.block_keys) return FATHOM_ERR_INVALID_ARG;
+        st = cuda_status(launch_append_blocks(keys, ix, m, stream));
+    } else {
+        st = cuda_status(launch_append(keys, ix, m, clamped, stream));
+    }
     if (st == FATHOM_OK) index->n_keys += m;
     return st;
 }
@@ -364,7 +376,8 @@ size_t fathom_scan_batched_workspace_bytes(const fathom_index *sessions, int32_t
 {
     if (!sessions || n_sessions < 1 || n_sessions > kMaxSessions || k < 1 || k > kMaxK) return 0;
     for (int s = 0; s < n_sessions; ++s)
-        if (!index_shape_ok(&sessions[s]) || index_bits(sessions[s]) != index_bits(sessions[0]))
+        if (!index_shape_ok(&sessions[s]) || index_bits(sessions[s]) != index_bits(sessions[0]) ||
+            (sessions[s].block_keys != 0) != (sessions[0].block_keys != 0))
             return 0;
     return scan_total_bytes(sessions, n_sessions, k);
 }

@@ -20,12 +20,25 @@ cudaError_t note_error(cudaError_t e, const char *site);
 // Code width b of an index: 4, or 8 for the 8-plane variant (the C ABI
 // reads 0 as 4 and rejects anything else before a launcher runs).
 inline int index_bits(const fathom_index &ix) { return ix.bits == 8 ? 8 : 4; }
+// Statistics rows per KV head: 1, or the blocks the planes can hold when the
+// index has grouped per-token-block scales (block_keys > 0).
+inline int index_blocks(const fathom_index &ix)
+{
+    return ix.block_keys ? (int)(((long long)ix.n_words * 32 + ix.block_keys - 1) / ix.block_keys)
+                         : 1;
+}
 
 // ---- pack.cu
 cudaError_t launch_pack(const float *keys, const fathom_index &ix, uint32_t *ws_minmax,
                         cudaStream_t stream);
-// sigma^2 of every (head, channel) from its exact sums and the key count n.
+// sigma^2 of every (head, channel) from its exact sums and the key count n
+// (combined over the blocks of a block-scaled index).
 cudaError_t launch_channel_stats(const fathom_index &ix, int n, cudaStream_t stream);
+// Appends m keys (device float32 [H][m][d]) to a block-scaled index whose
+// ix.n_keys is a whole number of blocks: the new blocks are packed on their
+// own, sigma^2 is recomputed for ix.n_keys + m keys.
+cudaError_t launch_append_blocks(const float *keys, const fathom_index &ix, int m,
+                                 cudaStream_t stream);
 
 // ---- append.cu
 // Appends m keys (device float32 [H][m][d]) at positions ix.n_keys.. and
@@ -45,19 +58,19 @@ cudaError_t launch_plan_marginal(const fathom_index &ix, const uint16_t *q, cons
 // An 8-plane index's scan arguments rewritten for the 4-plane scan over 2d
 // nibble channels (the planes themselves need no change).
 struct LiftArgs {
-    const float *mn, *scale;     // [H][d]
+    const float *mn, *scale;     // [stat_rows][d]: one row per (head, scale block)
     const uint16_t *q;           // [Q][d]
     const uint8_t *t, *tu;       // [Q][d], [H][d]
-    float *mn2, *scale2;         // [H][2d]
+    float *mn2, *scale2;         // [stat_rows][2d]
     uint16_t *q2;                // [Q][2d]
     uint8_t *t2, *tu2;           // [Q][2d], [H][2d]
-    int H, Q, d;
+    int H, Q, d, stat_rows;
 };
 // Workspace bytes of the primed arrays (each rounded up to 16 bytes).
-size_t lift_bytes(int H, int Q, int d);
-// Points the primed arrays of *a into ws (lift_bytes(H, Q, d) bytes, 16-byte
+size_t lift_bytes(int H, int Q, int d, int stat_rows);
+// Points the primed arrays of *a into ws (lift_bytes(...) bytes, 16-byte
 // aligned) and sets its sizes; the caller sets the inputs.
-void lift_carve(void *ws, int H, int Q, int d, LiftArgs *a);
+void lift_carve(void *ws, int H, int Q, int d, int stat_rows, LiftArgs *a);
 cudaError_t launch_lift(const LiftArgs &a, cudaStream_t stream);
 
 // ---- fetch.cu

@@ -19,7 +19,9 @@
 //   q'   = (q_c, q_c), t' = (min(t,4), max(t-4,0))   [likewise the union]
 // scores every key exactly as the 8-plane definition does (16*scale is a
 // power-of-two multiple, so W' = q*scale' is the same product scaled).
-// This kernel writes those primed arrays; the planes are not touched.
+// This kernel writes those primed arrays; the planes are not touched.  With
+// grouped per-token-block scales, mn and scale have a row per (head, block)
+// and are lifted row by row the same way.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,7 +31,7 @@ namespace {
 __global__ void __launch_bounds__(256)
 lift_kernel(LiftArgs a)
 {
-    const int total = max(a.Q, a.H) * a.d;
+    const int total = max(max(a.Q, a.H), a.stat_rows) * a.d;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
         if (i < a.Q * a.d) {   // query row i / d, channel i % d -> nibble channels 2i, 2i+1
             const uint16_t qv = a.q[i];
@@ -39,12 +41,14 @@ lift_kernel(LiftArgs a)
             a.t2[2 * i] = (uint8_t)min(t, 4);
             a.t2[2 * i + 1] = (uint8_t)max(t - 4, 0);
         }
-        if (i < a.H * a.d) {
+        if (i < a.stat_rows * a.d) {
             const float sc = a.scale[i];
             a.mn2[2 * i] = a.mn[i];
             a.mn2[2 * i + 1] = 0.0f;
             a.scale2[2 * i] = __fmul_rn(16.0f, sc);
             a.scale2[2 * i + 1] = sc;
+        }
+        if (i < a.H * a.d) {
             const int tu = min((int)a.tu[i], 8);
             a.tu2[2 * i] = (uint8_t)min(tu, 4);
             a.tu2[2 * i + 1] = (uint8_t)max(tu - 4, 0);
@@ -54,23 +58,23 @@ lift_kernel(LiftArgs a)
 
 }  // namespace
 
-size_t lift_bytes(int H, int Q, int d)
+size_t lift_bytes(int H, int Q, int d, int stat_rows)
 {
     auto a16 = [](size_t b) { return (b + 15) & ~(size_t)15; };
     const size_t d2 = 2 * (size_t)d;
-    return 2 * a16((size_t)H * d2 * sizeof(float)) + a16((size_t)Q * d2 * sizeof(uint16_t)) +
-           a16((size_t)Q * d2) + a16((size_t)H * d2);
+    return 2 * a16((size_t)stat_rows * d2 * sizeof(float)) +
+           a16((size_t)Q * d2 * sizeof(uint16_t)) + a16((size_t)Q * d2) + a16((size_t)H * d2);
 }
 
-void lift_carve(void *ws, int H, int Q, int d, LiftArgs *a)
+void lift_carve(void *ws, int H, int Q, int d, int stat_rows, LiftArgs *a)
 {
     auto a16 = [](size_t b) { return (b + 15) & ~(size_t)15; };
     const size_t d2 = 2 * (size_t)d;
     unsigned char *p = static_cast<unsigned char *>(ws);
     a->mn2 = reinterpret_cast<float *>(p);
-    p += a16((size_t)H * d2 * sizeof(float));
+    p += a16((size_t)stat_rows * d2 * sizeof(float));
     a->scale2 = reinterpret_cast<float *>(p);
-    p += a16((size_t)H * d2 * sizeof(float));
+    p += a16((size_t)stat_rows * d2 * sizeof(float));
     a->q2 = reinterpret_cast<uint16_t *>(p);
     p += a16((size_t)Q * d2 * sizeof(uint16_t));
     a->t2 = p;
@@ -79,11 +83,13 @@ void lift_carve(void *ws, int H, int Q, int d, LiftArgs *a)
     a->H = H;
     a->Q = Q;
     a->d = d;
+    a->stat_rows = stat_rows;
 }
 
 cudaError_t launch_lift(const LiftArgs &a, cudaStream_t stream)
 {
-    const int total = (a.Q > a.H ? a.Q : a.H) * a.d;
+    const int rows = a.Q > a.H ? a.Q : a.H;
+    const int total = (rows > a.stat_rows ? rows : a.stat_rows) * a.d;
     const int block = 256;
     const int grid = (total + block - 1) / block;
     lift_kernel<<<grid, block, 0, stream>>>(a);

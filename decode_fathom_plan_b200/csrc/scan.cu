@@ -68,6 +68,11 @@ constexpr int kTileGroups = kTileCols / 4;   // 16-byte column groups per 64-wor
 constexpr int kMainStages = 3;
 constexpr int kMaskOrderValues = 16;   // reader sets of up to 4 query heads
 constexpr int kMinChunkGroups = 8;     // smallest chunk of the main scan: 32 words
+// Sampled tiles of a session with grouped per-token-block scales (Qwen3-8B
+// layer, 128K keys in 2048-key blocks: 2 tiles sent some queries to the
+// exact fallback, 4 kept all on the fast path, 8 and 16 cost more threshold
+// passes than the fallbacks they saved).
+constexpr int kBlockedSampleTiles = 4;
 
 struct SessionDesc {
     const uint32_t *planes;      // device address of [H][d][4][n_words]
@@ -81,6 +86,10 @@ struct SessionDesc {
     uint32_t *qstate;            // [Q][4]: theta, count, fallback flag, spare
     unsigned long long *cand;    // [Q][cap]
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
+    float *bias_blk;             // grouped scales: [H][nb][G] bias per (head, block, query)
+    int block_words;             // grouped scales: plane words per scale block (0: none)
+    int nb, n_filled;            // statistics rows per head; blocks holding keys
+    int blk_begin;               // first CTA of this session in block_bias_kernel
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
     int chunks, chunk_begin;   // main-scan chunks per KV head, first chunk's CTA
@@ -207,7 +216,10 @@ __device__ __forceinline__ double bin_offset(int t)
 // up to 4 query heads; channel order otherwise), plane-row table, weights
 // (zero for a query that does not read the channel at full union depth) and
 // biases for query heads q_rows[0..G) of KV head h.
-// tu_row: the union plan to read; t_rows: each query's own plan.
+// tu_row: the union plan to read; t_rows: each query's own plan.  With
+// mn_h and sc_h null (grouped per-token-block scales) the tables hold the
+// unscaled weights w = q and the bias of mn = 0, scale = 1; each scanning
+// CTA then applies its own block's scales.
 // Thread c handles channel c: at least 256 threads, d <= 256.  Ends with a
 // barrier.
 template <int GP>
@@ -226,8 +238,8 @@ __device__ void setup_head(ScanMeta<GP> &sm, int h, int G, int d, const uint8_t 
     float qf[GP];
     if (in) {
         T = min((int)tu_row[c], kBits);
-        sc = sc_h[c];
-        mn = mn_h[c];
+        sc = sc_h ? sc_h[c] : 1.0f;
+        mn = mn_h ? mn_h[c] : 0.0f;
     }
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -606,12 +618,89 @@ __device__ __forceinline__ int find_session_by_query(const Batch<NS> &b, int gq)
     return si;
 }
 
+template <int NS>
+__device__ __forceinline__ int find_session_by_block(const Batch<NS> &b, int gi)
+{
+    int si = 0;
+    for (int s = 1; s < b.n_sessions; ++s)
+        if (b.s[s].blk_begin <= gi) si = s;
+    return si;
+}
+
+// ------------------------------------------------ grouped per-block biases
+// One CTA per (session, KV head, scale block holding keys): the bias of
+// each query head of the KV head with that block's scales,
+//   bias_g = sum_c q_gc * (mn_bc + scale_bc * (2^(4-t)-1)/2),
+// t the query's depth clamped to the union, summed exactly as setup_head
+// sums the bias of a one-block index (fp64 terms, warp shuffles, warps in
+// order).  Thread c handles channel c.
+template <int NS>
+__global__ void __launch_bounds__(kScanThreads) block_bias_kernel(const __grid_constant__ Batch<NS> b)
+{
+    __shared__ double part[kScanThreads / 32][kMaxGroup];
+    const int gi = blockIdx.x;
+    const SessionDesc &S = b.s[find_session_by_block(b, gi)];
+    const int local = gi - S.blk_begin;
+    const int h = local / S.n_filled, blk = local - h * S.n_filled;
+    const int G = b.G, d = b.d;
+    const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+    const bool in = c < d;
+    int T = 0;
+    float mn = 0.0f, sc = 0.0f;
+    if (in) {
+        T = min((int)S.tu[h * d + c], kBits);
+        const size_t e = ((size_t)h * S.nb + blk) * d + c;
+        mn = S.mn[e];
+        sc = S.scale[e];
+    }
+    for (int g = 0; g < G; ++g) {
+        double term = 0.0;
+        if (in) {
+            const int tg = min((int)S.t[(size_t)(h * G + g) * d + c], T);
+            const float qf = bf16_to_float(S.q[(size_t)(h * G + g) * d + c]);
+            term = (double)qf * ((double)mn + (double)sc * bin_offset(tg));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
+        if (lane == 0) part[warp][g] = term;
+    }
+    __syncthreads();
+    if (c < G) {
+        double acc = 0.0;
+#pragma unroll
+        for (int w = 0; w < kScanThreads / 32; ++w) acc += part[w][c];
+        S.bias_blk[((size_t)h * S.nb + blk) * G + c] = (float)acc;
+    }
+}
+
+// The CTA's block: scale the unscaled weights of the head's tables by the
+// block's channel scales and take the block's biases.  Ends with a barrier.
+template <int GP>
+__device__ __forceinline__ void apply_block(ScanMeta<GP> &sm, const SessionDesc &S, int h, int blk,
+                                            int G, int d)
+{
+    const int U = sm.U;
+    const float *sc_row = S.scale + ((size_t)h * S.nb + blk) * d;
+    for (int i = threadIdx.x; i < U * GP; i += blockDim.x) {
+        const int u = i / GP, g = i - u * GP;
+        const int c = (int)(sm.row_g[u * kBits] / kBits) - h * d;   // slot 0 of every union channel
+        const float sc = sc_row[c];
+        const float2 w2 = sm.W2[u][g];
+        sm.W2[u][g] = make_float2(__fmul_rn(w2.x, sc), __fmul_rn(w2.y, sc));
+        sm.Wp[u][g] = __fmul_rn(sm.Wp[u][g], sc);
+    }
+    if (threadIdx.x < GP)
+        sm.bias[threadIdx.x] =
+            (threadIdx.x < G) ? S.bias_blk[((size_t)h * S.nb + blk) * G + threadIdx.x] : 0.0f;
+    __syncthreads();
+}
+
 // ------------------------------------------------------- filtered scan
 // CTA i owns column groups [i*per_cta, (i+1)*per_cta) of the linear
 // (session, KV head, column group) space (one 64-word chunk, or two pieces
 // where the range crosses a KV head's end) and appends the keys scoring
 // >= theta to their query's candidate buffer.
-template <int NS, int GP, int STAGES>
+template <int NS, int GP, int STAGES, bool kBlocked>
 __global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
 scan_kernel(const __grid_constant__ Batch<NS> b)
 {
@@ -632,8 +721,21 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
         const int local = (int)blockIdx.x - S.chunk_begin;
         const int h = local / S.chunks;
         const int c = local - h * S.chunks;
-        const int g0 = (int)((long long)c * S.col_groups / S.chunks);
-        const int g1 = (int)((long long)(c + 1) * S.col_groups / S.chunks);
+        int g0, g1, blk = 0;
+        if constexpr (kBlocked) {
+            // S.chunks / S.n_filled equal chunks per scale block: a chunk
+            // never spans two blocks
+            const int cpb = S.chunks / S.n_filled;
+            blk = c / cpb;
+            const int sub = c - blk * cpb;
+            const int gb0 = blk * (S.block_words / 4);
+            const int gbn = min(S.col_groups, gb0 + S.block_words / 4) - gb0;
+            g0 = gb0 + (int)((long long)sub * gbn / cpb);
+            g1 = gb0 + (int)((long long)(sub + 1) * gbn / cpb);
+        } else {
+            g0 = (int)((long long)c * S.col_groups / S.chunks);
+            g1 = (int)((long long)(c + 1) * S.col_groups / S.chunks);
+        }
         const int col_lo = g0 * 4;
         const int width = (g1 - g0) * 4;               // plane words owned by this chunk
         const int col_hi = min(S.n_cols, col_lo + width);
@@ -643,6 +745,7 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
                                        ? S.qstate[(q0 + threadIdx.x) * kQueryStateWords + 0]
                                        : 0xFFFFFFFFu;
         load_head<GP>(sm, S.tables, h);
+        if constexpr (kBlocked) apply_block<GP>(sm, S, h, blk, G, b.d);
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
 
@@ -880,7 +983,7 @@ constexpr size_t kThetaStageBytes = (size_t)kStageRows * kThetaCols * sizeof(uin
 constexpr int kThetaResolutionBits = 2 * kSelBits;
 constexpr int kThetaBufs = 3;   // stages in flight
 
-template <int NS, int GP>
+template <int NS, int GP, bool kBlocked>
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_constant__ Batch<NS> b,
                                                                 uint32_t force_exact,
                                                                 int total_queries)
@@ -890,9 +993,12 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     __shared__ SelShared ss;
     __shared__ uint16_t own_c[kMaxHeadDim];   // the query's channels (t > 0) ...
     __shared__ uint8_t own_t[kMaxHeadDim];    // ... their depths ...
-    __shared__ float own_w[kMaxHeadDim];      // ... and weights q*scale
+    __shared__ float own_w[kMaxHeadDim];      // ... and weights q*scale (q with grouped scales)
     __shared__ double bias_part[kSelThreads / 32];
     __shared__ float bias_s;
+    // grouped scales: the weights and bias of the pass's two tiles' blocks
+    __shared__ float tile_w[kBlocked ? kThetaTilesPerPass : 1][kBlocked ? kMaxHeadDim : 1];
+    __shared__ float tile_bias[kThetaTilesPerPass];
     ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
     uint32_t *vals = th_dyn + kThetaBufs * kStageRows * kThetaCols;
     const int G = b.G, d = b.d;
@@ -901,7 +1007,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
         const SessionDesc &S = b.s[find_session_by_head(b, gh)];
         const int h = gh - S.head_begin;
         setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)h * G * d, S.q + (size_t)h * G * d,
-                       S.mn + h * d, S.scale + h * d);
+                       kBlocked ? nullptr : S.mn + h * d, kBlocked ? nullptr : S.scale + h * d);
         constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
         const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
         uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
@@ -932,9 +1038,13 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
             const int T = min((int)S.tu[h * d + c], kBits);
             tq = min((int)S.t[(size_t)qq * d + c], T);
             const float qf = bf16_to_float(S.q[(size_t)qq * d + c]);
-            const float sc = S.scale[h * d + c];
-            w = __fmul_rn(qf, sc);
-            term = (double)qf * ((double)S.mn[h * d + c] + (double)sc * bin_offset(tq));
+            if constexpr (kBlocked) {
+                w = qf;   // scaled per sampled tile below; the bias is per block
+            } else {
+                const float sc = S.scale[h * d + c];
+                w = __fmul_rn(qf, sc);
+                term = (double)qf * ((double)S.mn[h * d + c] + (double)sc * bin_offset(tq));
+            }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
@@ -989,6 +1099,28 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
         __syncthreads();   // the buffers are free
+        if constexpr (kBlocked) {
+            // each sampled tile lies in one scale block (blocks hold whole tiles)
+            for (int e = threadIdx.x; e < kThetaTilesPerPass * kMaxHeadDim; e += kSelThreads) {
+                const int tsub = e / kMaxHeadDim, j = e - tsub * kMaxHeadDim;
+                const int tile = t0 + tsub;
+                const int wcol = tile * S.sample_stride * kTileCols;
+                if (j < n_own && tile < S.m_tiles && wcol < S.n_cols) {
+                    const int blk = wcol / S.block_words;
+                    tile_w[tsub][j] = __fmul_rn(
+                        own_w[j], S.scale[((size_t)h * S.nb + blk) * d + own_c[j]]);
+                }
+            }
+            if (threadIdx.x < kThetaTilesPerPass) {
+                const int tile = t0 + threadIdx.x;
+                const int wcol = tile * S.sample_stride * kTileCols;
+                tile_bias[threadIdx.x] =
+                    (tile < S.m_tiles && wcol < S.n_cols)
+                        ? S.bias_blk[((size_t)h * S.nb + wcol / S.block_words) * G + (qq - h * G)]
+                        : 0.0f;
+            }
+            __syncthreads();
+        }
         for (int s2 = 0; s2 < kThetaBufs - 1 && s2 < n_stages; ++s2) load(t0, s2, s2);
         for (int s2 = 0; s2 < n_stages; ++s2) {
             // stage s2 has landed once at most (stages issued after it) groups are pending
@@ -1009,7 +1141,8 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
                                                sub * kTileCols + col, sh);
                 float2 v[4];
                 nibbles_to_floats(nib, neg, v);   // rows past the depth are zero
-                const float2 w2 = make_float2(own_w[j], own_w[j]);
+                const float wj = kBlocked ? tile_w[kBlocked ? sub : 0][kBlocked ? j : 0] : own_w[j];
+                const float2 w2 = make_float2(wj, wj);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = __ffma2_rn(v[i], w2, acc[i]);
             }
@@ -1018,11 +1151,12 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
         const int tile = t0 + sub;
         if (tile < S.m_tiles) {
             const int wcol = tile * S.sample_stride * kTileCols + col;
+            const float tb = kBlocked ? tile_bias[sub] : bias;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int j = wcol * 32 + r + 4 * m;
                 vals[tile * kTileKeys + col * 32 + r + 4 * m] =
-                    (wcol < S.n_cols && j < S.n) ? order_key(score_of(acc, m, bias)) : 0u;
+                    (wcol < S.n_cols && j < S.n) ? order_key(score_of(acc, m, tb)) : 0u;
             }
         }
     }
@@ -1116,11 +1250,12 @@ __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constan
 // One CTA per flagged query: exact top-k by radix select over the composite
 // (order key, ~index), recomputing the query's scores from its own plan on
 // every pass.  Slow, rare, and independent of the sample.
-template <int NS>
+template <int NS, bool kBlocked>
 __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_constant__ Batch<NS> b)
 {
     __shared__ ScanMeta<1> sm;
     __shared__ SelectState ss;
+    __shared__ float q_raw[kBlocked ? kMaxHeadDim : 1];   // unscaled weights (grouped scales)
     extern __shared__ __align__(16) uint32_t fb_dyn[];
     StageBuf stage = reinterpret_cast<StageBuf>(fb_dyn);
     unsigned long long *sel =
@@ -1133,10 +1268,36 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
     const int d = b.d, k = b.k;
     const int h = qq / b.G;
     const uint8_t *trow = S.t + (size_t)qq * d;
-    setup_head<1>(sm, h, 1, d, trow, trow, S.q + (size_t)qq * d, S.mn + h * d, S.scale + h * d);
+    setup_head<1>(sm, h, 1, d, trow, trow, S.q + (size_t)qq * d, kBlocked ? nullptr : S.mn + h * d,
+                  kBlocked ? nullptr : S.scale + h * d);
     select_reset(ss, (unsigned)k);
     const int col = threadIdx.x >> 2, r = threadIdx.x & 3;
-    const float bias = sm.bias[0];
+    float bias = sm.bias[0];
+    int cur_blk = -1;
+    if constexpr (kBlocked) {
+        for (int u = threadIdx.x; u < sm.U; u += blockDim.x) q_raw[u] = sm.Wp[u][0];
+        __syncthreads();
+    }
+    // grouped scales: before scanning tile c0, the weights and bias of its
+    // block (the query reads every union channel at full depth here)
+    auto use_block = [&](int c0) {
+        if constexpr (kBlocked) {
+            const int blk = c0 / S.block_words;
+            if (blk != cur_blk) {
+                __syncthreads();   // the previous tile's compute is done with sm
+                const float *sc_row = S.scale + ((size_t)h * S.nb + blk) * d;
+                for (int u = threadIdx.x; u < sm.U; u += blockDim.x) {
+                    const int c = (int)(sm.row_g[u * kBits] / kBits) - h * d;
+                    const float w = __fmul_rn(q_raw[u], sc_row[c]);
+                    sm.W2[u][0] = make_float2(w, w);
+                    sm.Wp[u][0] = w;
+                }
+                bias = S.bias_blk[((size_t)h * S.nb + blk) * b.G + (qq - h * b.G)];
+                cur_blk = blk;
+                __syncthreads();
+            }
+        }
+    };
     float2 acc[1][4];
     for (int digit = 7; digit >= 0; --digit) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) ss.hist[i] = 0;
@@ -1144,6 +1305,7 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
         const unsigned long long pm = ss.pmask, pf = ss.prefix;
         for (int c0 = 0; c0 < S.n_cols; c0 += kTileCols) {
             const int c1 = min(S.n_cols, c0 + kTileCols);
+            use_block(c0);
             scan_chunk<1, kMainStages>(sm, stage, S.planes, S.n_words, c0, c1, acc);
             const int key0 = (c0 + col) * 32 + r;
 #pragma unroll
@@ -1164,6 +1326,7 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
     const unsigned long long lim = ss.prefix >> shift;
     for (int c0 = 0; c0 < S.n_cols; c0 += kTileCols) {
         const int c1 = min(S.n_cols, c0 + kTileCols);
+        use_block(c0);
         scan_chunk<1, kMainStages>(sm, stage, S.planes, S.n_words, c0, c1, acc);
         const int key0 = (c0 + col) * 32 + r;
 #pragma unroll
@@ -1211,7 +1374,7 @@ struct Sizing {
 // m ~ 128*n/(2k) clamped to [4096, 32768] and to a quarter of the tiles;
 // theta is the r-th largest sampled key, r = ceil(f*k*m/n) with f = 2 (or 3
 // when f = 2 would give r < 128), so about f*k keys pass the filter.
-Sizing size_session(int n, int n_words, int k)
+Sizing size_session(int n, int n_words, int k, int block_keys)
 {
     Sizing z{};
     z.n_cols = std::min(n_words, ceil_div(ceil_div(n, 32), 4) * 4);
@@ -1222,6 +1385,11 @@ Sizing size_session(int n, int n_words, int k)
     const double target = (double)kSampleTargetRank * (double)n / (2.0 * (double)k);
     int m = (int)std::min<double>(std::max<double>(target, kSampleMinKeys), kSampleMaxKeys);
     int mt = ceil_div(m, kTileKeys);
+    // Grouped scales shift every block's scores by its own unread-channel
+    // constant, so a sample of few blocks misplaces theta and sends queries
+    // to the exact fallback; at least kBlockedSampleTiles tiles (from as many
+    // blocks) keep it on the fast path.
+    if (block_keys) mt = std::max(mt, kBlockedSampleTiles);
     mt = std::min(mt, std::max(1, z.n_tiles / 4));
     z.m_tiles = mt;
     z.stride = z.n_tiles / mt;
@@ -1234,7 +1402,7 @@ Sizing size_session(int n, int n_words, int k)
 }
 
 struct WsLayout {
-    size_t qstate, cand, tables, mirror, total;
+    size_t qstate, cand, tables, bias_blk, mirror, total;
 };
 
 // Query heads per KV head rounded up to the kernels' template width.
@@ -1268,6 +1436,9 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     at += align256((size_t)Q * cap * sizeof(unsigned long long));
     L.tables = at;
     at += align256((size_t)ix.n_kv_heads * head_table_bytes(ix.group));
+    L.bias_blk = at;   // grouped scales: a bias per (KV head, block, query head)
+    if (ix.block_keys)
+        at += align256((size_t)ix.n_kv_heads * index_blocks(ix) * ix.group * sizeof(float));
     L.mirror = at;
     if (host_resident(ix)) at += align256(plane_bytes(ix));
     L.total = at;
@@ -1310,10 +1481,9 @@ cudaError_t ensure_smem(int (&done)[64], Kernel kernel, size_t max_bytes)
 // One set of "limit raised" flags per kernel instantiation.
 template <int NS>
 struct SmemFlags {
-    static int final_[64], fallback[64];
+    static int final_[64];
 };
 template <int NS> int SmemFlags<NS>::final_[64];
-template <int NS> int SmemFlags<NS>::fallback[64];
 
 constexpr size_t kStageBytes = (size_t)kStageRows * kTileCols * sizeof(uint32_t);
 
@@ -1344,9 +1514,9 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
     return m;
 }
 
-template <int NS, int GP>
+template <int NS, int GP, bool kBlocked>
 cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, int total_heads,
-                      int max_m_keys,
+                      int total_blocks, int max_m_keys,
                       const FetchJob *fetch, int n_fetch, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
 {
@@ -1362,11 +1532,17 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
             hook->recorded = true;
         }
     }
+    if (kBlocked) {
+        // grouped scales: the bias of every (KV head, block, query head)
+        block_bias_kernel<NS><<<total_blocks, kScanThreads, 0, stream>>>(bt);
+        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "block bias launch");
+        ++launches;
+    }
     {
         // per-head tables, sampled scores and theta per query (or the
         // exact-path flags)
         static int threshold_smem_set[64];
-        auto kern = threshold_kernel<NS, GP>;
+        auto kern = threshold_kernel<NS, GP, kBlocked>;
         const size_t dyn = kThetaBufs * kThetaStageBytes + (size_t)max_m_keys * sizeof(uint32_t);
         if ((e = ensure_smem(threshold_smem_set, kern,
                              kThetaBufs * kThetaStageBytes +
@@ -1383,7 +1559,7 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
     if (!force && total_chunks > 0) {
         const bool timed = hook && hook->enabled && n_fetch == 0;
         static int main_smem_set[64];
-        auto kern = scan_kernel<NS, GP, kMainStages>;
+        auto kern = scan_kernel<NS, GP, kMainStages, kBlocked>;
         const size_t dyn = kMainStages * kStageBytes;
         if ((e = ensure_smem(main_smem_set, kern, dyn)) != cudaSuccess) return note_error(e, "scan set-up");
         if (timed) record_timing_event(hook->begin, stream);
@@ -1406,11 +1582,12 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
     final_kernel<NS><<<total_queries, kSelThreads, final_smem, stream>>>(bt);
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "final launch");
     const size_t fb_smem = kMainStages * kStageBytes + (size_t)bt.kpad * sizeof(unsigned long long);
-    if ((e = ensure_smem(SmemFlags<NS>::fallback, fallback_kernel<NS>,
+    static int fallback_smem_set[64];
+    if ((e = ensure_smem(fallback_smem_set, fallback_kernel<NS, kBlocked>,
                          kMainStages * kStageBytes + (size_t)kMaxK * sizeof(unsigned long long))) !=
         cudaSuccess)
         return note_error(e, "fallback set-up");
-    fallback_kernel<NS><<<total_queries, kScanThreads, fb_smem, stream>>>(bt);
+    fallback_kernel<NS, kBlocked><<<total_queries, kScanThreads, fb_smem, stream>>>(bt);
     launches += 2;
     note_launch(launches);
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "fallback launch");
@@ -1430,13 +1607,13 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, queries = 0, heads = 0, max_m = 0, n_fetch = 0;
+    int groups = 0, queries = 0, heads = 0, blocks = 0, max_m = 0, n_fetch = 0;
     FetchJob fetch[NS];
     size_t at = 0;
     char *base = static_cast<char *>(ws);
     for (int s = 0; s < n_sessions; ++s) {
         const fathom_index &ix = *ss[s].ix;
-        const Sizing z = size_session(ix.n_keys, ix.n_words, k);
+        const Sizing z = size_session(ix.n_keys, ix.n_words, k, ix.block_keys);
         const WsLayout L = layout_session(ix, k, at);
         at = L.total;
         SessionDesc &D = bt.s[s];
@@ -1457,6 +1634,12 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.qstate = reinterpret_cast<uint32_t *>(base + L.qstate);
         D.cand = reinterpret_cast<unsigned long long *>(base + L.cand);
         D.tables = reinterpret_cast<unsigned char *>(base + L.tables);
+        D.bias_blk = reinterpret_cast<float *>(base + L.bias_blk);
+        D.block_words = ix.block_keys / 32;
+        D.nb = index_blocks(ix);
+        D.n_filled = ix.block_keys ? ceil_div(ix.n_keys, ix.block_keys) : 1;
+        D.blk_begin = blocks;
+        if (ix.block_keys) blocks += ix.n_kv_heads * D.n_filled;
         D.H = ix.n_kv_heads;
         D.n = ix.n_keys;
         D.n_words = ix.n_words;
@@ -1468,6 +1651,8 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
         D.chunks = (D.col_groups + kTileGroups - 1) / kTileGroups;   // chunks of <= 64 words
+        if (ix.block_keys)   // the same number of chunks in every scale block
+            D.chunks = D.n_filled * ceil_div(D.block_words / 4, kTileGroups);
         D.q_begin = queries;
         D.head_begin = heads;
         heads += ix.n_kv_heads;
@@ -1484,8 +1669,14 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         groups = 0;
         for (int s = 0; s < n_sessions; ++s) {
             SessionDesc &D = bt.s[s];
-            const int most = std::max(1, D.col_groups / kMinChunkGroups);
-            D.chunks = std::max(D.chunks, std::min(most, (int)(D.chunks * grow)));
+            if (D.block_words) {
+                const int per = D.chunks / D.n_filled;
+                const int most = std::max(1, (D.block_words / 4) / kMinChunkGroups);
+                D.chunks = D.n_filled * std::max(per, std::min(most, (int)(per * grow)));
+            } else {
+                const int most = std::max(1, D.col_groups / kMinChunkGroups);
+                D.chunks = std::max(D.chunks, std::min(most, (int)(D.chunks * grow)));
+            }
             groups += D.H * D.chunks;
         }
     }
@@ -1495,14 +1686,24 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         groups += bt.s[s].H * bt.s[s].chunks;
     }
     const int G = bt.G;
-    if (G <= 1) return run_batch<NS, 1>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
-                                           stream, hook);
-    if (G <= 2) return run_batch<NS, 2>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
-                                           stream, hook);
-    if (G <= 4) return run_batch<NS, 4>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
-                                           stream, hook);
-    return run_batch<NS, 8>(bt, groups, queries, heads, max_m, fetch, n_fetch, flags,
-                                           stream, hook);
+    if (blocks > 0) {   // every session has grouped scales (the C ABI checks)
+        if (G <= 1) return run_batch<NS, 1, true>(bt, groups, queries, heads, blocks, max_m, fetch,
+                                                  n_fetch, flags, stream, hook);
+        if (G <= 2) return run_batch<NS, 2, true>(bt, groups, queries, heads, blocks, max_m, fetch,
+                                                  n_fetch, flags, stream, hook);
+        if (G <= 4) return run_batch<NS, 4, true>(bt, groups, queries, heads, blocks, max_m, fetch,
+                                                  n_fetch, flags, stream, hook);
+        return run_batch<NS, 8, true>(bt, groups, queries, heads, blocks, max_m, fetch, n_fetch,
+                                      flags, stream, hook);
+    }
+    if (G <= 1) return run_batch<NS, 1, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
+                                               flags, stream, hook);
+    if (G <= 2) return run_batch<NS, 2, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
+                                               flags, stream, hook);
+    if (G <= 4) return run_batch<NS, 4, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
+                                               flags, stream, hook);
+    return run_batch<NS, 8, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch, flags,
+                                   stream, hook);
 }
 
 }  // namespace

@@ -33,6 +33,10 @@
  *                 the b-bit code (slot 0 = most significant); bit i of word
  *                 w belongs to key 32*w+i; words past the last key are zero
  *       mn, scale, sigma2  float32 [H][d]; sum_code, sum_code2 int64 [H][d]
+ *                 -- with grouped per-token-block scales (block_keys > 0)
+ *                 mn, scale, sum_code and sum_code2 are [H][n_blocks][d],
+ *                 n_blocks = ceil(32*n_words / block_keys), key j belonging
+ *                 to block j / block_keys; sigma2 stays [H][d]
  *       q         bfloat16 bits (uint16) [Q][d], query q served by KV head
  *                 q / G
  *       budget    int32 [Q] bits per key, 0 <= B <= b*d
@@ -51,6 +55,11 @@
  *     deployment notes (部署前必读, item 3) call for when the upstream K
  *     cache is 8-bit: the same quantiser with 255 levels, plans capped at 8
  *     bits per channel, the same coarse-bin rebuild.
+ *   - Grouped per-token-block scales (block_keys > 0, a multiple of 2048):
+ *     the index is the grouped quantised K of a serving stack (the
+ *     explainer, 亮点 / 适用边界: Fathom reads the 4-bit K the stack already
+ *     holds); every block of block_keys tokens of a channel is quantised on
+ *     its own, and a key is rebuilt with its block's mn and scale.
  */
 #ifndef FATHOM_H
 #define FATHOM_H
@@ -104,6 +113,7 @@ typedef struct {
     int64_t *sum_code;        /* [H][d] sum of codes */
     int64_t *sum_code2;       /* [H][d] sum of squared codes */
     int32_t bits;             /* b: 4 or 8 (0 means 4) */
+    int32_t block_keys;       /* 0, or tokens per scale block (a multiple of 2048) */
 } fathom_index;
 
 /* Scan flags. */
@@ -139,6 +149,12 @@ size_t fathom_pack_workspace_bytes(const fathom_index *index);
  * importance weight the read side uses).
  * keys: device float32 [H][n][d].  Every output array of `index` is
  * written; planes may be a mapped host pointer (written zero-copy).
+ * With grouped scales the min, scale and sums are per (h, block, c), each
+ * block over its own keys (the last one may be short), and sigma2 is the
+ * variance of all n dequantised keys: each block's mean and squared
+ * deviations from its exact sums, combined block by block in fp64 with
+ * the pairwise update of Chan, Golub and LeVeque; the workspace is then
+ * unused (the accumulators live in mn and scale).
  * A non-finite key sets FATHOM_ERR_NONFINITE in the device status. */
 fathom_status fathom_pack_keys(const float *keys, const fathom_index *index,
                                void *workspace, size_t workspace_bytes,
@@ -162,7 +178,11 @@ fathom_status fathom_pack_keys(const float *keys, const fathom_index *index,
  * past key n zero (as fathom_pack_keys and earlier appends leave them);
  * planes may be a mapped host pointer.  On success index->n_keys grows by
  * m (host field).  A non-finite key stores code 0 and sets
- * FATHOM_ERR_NONFINITE in the device status. */
+ * FATHOM_ERR_NONFINITE in the device status.
+ * Grouped scales: n must be a whole number of blocks (the serving stack
+ * hands over a block once it is full); the m keys open new blocks, each
+ * quantised on its own exactly as fathom_pack_keys would, sigma2 is
+ * recombined, and `clamped` is not touched (nothing is clamped). */
 fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t m,
                                  uint32_t *clamped, cudaStream_t stream);
 
@@ -228,6 +248,10 @@ size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k);
  * (9*H + 3*Q)*2d bytes of workspace (each array rounded up to 16 bytes) for
  * the nibble-channel arguments.
  * All sessions of a batched call have the same b.
+ * Grouped scales: key j is scored with mn and scale of its block; one more
+ * small launch computes each (KV head, block, query head) bias, and the
+ * workspace holds those H*n_blocks*G floats.  All sessions of a batched
+ * call have grouped scales or none have.
  * q_bf16, t, t_union, out_idx, out_score, workspace: device pointers.
  * flags: FATHOM_SCAN_* bits. */
 fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16,

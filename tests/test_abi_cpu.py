@@ -76,7 +76,8 @@ def test_host_resident_workspace_holds_a_plane_mirror(lib):
 @pytest.mark.parametrize("field,value", [("head_dim", 48), ("head_dim", 512), ("group", 9),
                                          ("group", 0), ("n_words", 6), ("n_keys", 0),
                                          ("residency", 7), ("bits", 5), ("bits", 2),
-                                         ("n_words", (1 << 22) + 4)])
+                                         ("n_words", (1 << 22) + 4), ("block_keys", 1000),
+                                         ("block_keys", -2048)])
 def test_bad_index_shapes_are_rejected(lib, field, value):
     ix = _desc()
     setattr(ix, field, value)
@@ -188,3 +189,21 @@ def test_eight_plane_index_sizes_and_limits(lib):
     a.bits = 8
     assert fp.fathom_scan_batched_workspace_bytes([a, b], 64) == \
         2 * fp.fathom_scan_workspace_bytes(b, 64)
+
+
+def test_grouped_scale_workspace_holds_the_block_biases(lib):
+    """Grouped per-token-block scales add one float per (KV head, block,
+    query head) to the scan workspace; a batch mixes no scale modes."""
+    for H, G, n, block in ((2, 4, 4096, 2048), (8, 4, 1 << 20, 2048), (1, 8, 5000, 4096)):
+        plain = _desc(H=H, G=G, n=n)
+        grouped = _desc(H=H, G=G, n=n)
+        grouped.block_keys = block
+        nb = -(-32 * fp.fathom_n_words(n) // block)
+        extra = (H * nb * G * 4 + 255) // 256 * 256
+        assert fp.fathom_scan_workspace_bytes(grouped, 64) == \
+            fp.fathom_scan_workspace_bytes(plain, 64) + extra
+    a, b = _desc(), _desc()
+    b.block_keys = 2048
+    assert fp.fathom_scan_batched_workspace_bytes([a, b], 64) == 0
+    a.block_keys = 4096
+    assert fp.fathom_scan_batched_workspace_bytes([a, b], 64) > 0
