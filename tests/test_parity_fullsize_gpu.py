@@ -3,6 +3,9 @@ benchmark times, on sampled queries the oracle scores one by one.
 
 * Qwen3-8B-shaped layer, HBM-resident: 8 KV heads x 4 query heads,
   head_dim 128, 131072 keys, B in {68, 92, 136}, k = 2048.
+* The same layer as an 8-plane index (8-bit K cache) and with grouped
+  per-token-block scales (2048-token blocks), as the benchmark's
+  qwen3_8b_layer_128k_8plane and qwen3_8b_layer_128k_blocked workloads.
 * Million-token host-resident scan, 2 of the 8 KV heads (the oracle's cost
   grows with the heads checked; the kernel's per-head work is the same),
   1,048,576 keys, B in {18, 92}, k = 2048."""
@@ -51,6 +54,43 @@ def test_layer_scan_sampled_queries(layer, B):
     for qq in (0, 13, 31):
         _, _, s, a = oracle_query(ref, ses.q_bf16[qq], t[qq], qq // 4, 2048)
         check_topk(oi[qq], os_[qq], s, a, 2048)
+
+
+def _variant_index(ses, **kw):
+    ix = fp.KeyIndex(ses.n_kv_heads, ses.group, ses.n_keys, ses.head_dim, **kw)
+    ix.pack(torch.from_numpy(ses.keys).cuda())
+    torch.cuda.synchronize()
+    assert fp.fathom_last_device_status() == fp.FATHOM_OK
+    return ix
+
+
+@pytest.mark.parametrize("variant", ["8plane", "blocked"])
+def test_layer_variants_pack_plans_and_sampled_queries(layer, variant):
+    ses, _, _ = layer
+    kw = dict(bits=8) if variant == "8plane" else dict(block_keys=2048)
+    ix = _variant_index(ses, **kw)
+    ref = oracle.build_index(ses.keys, **kw)
+    nbf = oracle.n_blocks_for(131072, 2048) if variant == "blocked" else None
+    planes = ix.planes.cpu().numpy().view(np.uint32)
+    assert np.array_equal(planes, ref["planes"])
+    for name, got in (("mn", ix.mn), ("scale", ix.scale), ("s1", ix.sum_code),
+                      ("s2", ix.sum_code2)):
+        g = got.cpu().numpy()
+        r = ref[name]
+        if nbf:
+            g, r = g[:, :nbf], r[:, :nbf]
+        assert np.array_equal(np.ascontiguousarray(g).view(np.uint8),
+                              np.ascontiguousarray(r).view(np.uint8)), name
+    assert np.array_equal(ix.sigma2.cpu().numpy().view(np.uint32), ref["sigma2"].view(np.uint32))
+    for B in (68, 136):
+        budgets = np.full(32, B, np.int32)
+        t, nb, oi, os_ = _scan(ix, ses, budgets, 2048)
+        rt, rT, rnb = oracle.plan_session(ref, ses.q_bf16, budgets, 4)
+        assert np.array_equal(t, rt)
+        assert np.array_equal(nb.astype(np.uint64), rnb)
+        for qq in (0, 31):
+            _, _, s, a = oracle_query(ref, ses.q_bf16[qq], t[qq], qq // 4, 2048)
+            check_topk(oi[qq], os_[qq], s, a, 2048)
 
 
 @pytest.mark.slow
