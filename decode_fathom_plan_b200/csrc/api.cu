@@ -300,6 +300,7 @@ size_t fathom_pack_workspace_bytes(const fathom_index *index)
 fathom_status fathom_pack_keys(const float *keys, const fathom_index *index, void *workspace,
                                size_t workspace_bytes, cudaStream_t stream)
 {
+    NvtxRange range("fathom_pack_keys");
     if (!keys || !index_shape_ok(index) || !stats_ok(index)) return FATHOM_ERR_INVALID_ARG;
     if (!workspace || !aligned16(workspace) || workspace_bytes < fathom_pack_workspace_bytes(index))
         return FATHOM_ERR_WORKSPACE;
@@ -312,6 +313,7 @@ fathom_status fathom_pack_keys(const float *keys, const fathom_index *index, voi
 fathom_status fathom_append_keys(fathom_index *index, const float *keys, int32_t m,
                                  uint32_t *clamped, cudaStream_t stream)
 {
+    NvtxRange range("fathom_append_keys");
     if (!keys || !index_shape_ok(index) || !stats_ok(index) || m < 1) return FATHOM_ERR_INVALID_ARG;
     if ((long long)index->n_keys + m > (long long)index->n_words * 32) return FATHOM_ERR_INVALID_ARG;
     fathom_index ix = *index;
@@ -332,6 +334,7 @@ fathom_status fathom_plan(const fathom_index *index, const uint16_t *q_bf16,
                           const int32_t *budget, uint8_t *t, uint8_t *t_union, uint64_t *bytes,
                           cudaStream_t stream)
 {
+    NvtxRange range("fathom_plan");
     if (!index_shape_ok(index) || !index->sigma2) return FATHOM_ERR_INVALID_ARG;
     if (!q_bf16 || !budget || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
     return cuda_status(launch_plan(*index, q_bf16, budget, 0, false, t, t_union, bytes, stream));
@@ -341,6 +344,7 @@ fathom_status fathom_plan_marginal(const fathom_index *index, const uint16_t *q_
                                    const int32_t *budget, uint8_t *t, uint8_t *t_union,
                                    uint64_t *bytes, cudaStream_t stream)
 {
+    NvtxRange range("fathom_plan_marginal");
     if (!index_shape_ok(index) || !index->sigma2) return FATHOM_ERR_INVALID_ARG;
     if (!q_bf16 || !budget || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
     return cuda_status(launch_plan_marginal(*index, q_bf16, budget, t, t_union, bytes, stream));
@@ -350,6 +354,7 @@ fathom_status fathom_fixed_plan(const fathom_index *index, const uint16_t *q_bf1
                                 uint8_t *t, uint8_t *t_union, uint64_t *bytes,
                                 cudaStream_t stream)
 {
+    NvtxRange range("fathom_fixed_plan");
     if (!index_shape_ok(index)) return FATHOM_ERR_INVALID_ARG;
     if (!q_bf16 || !t || !t_union || !bytes) return FATHOM_ERR_INVALID_ARG;
     if (r < 0 || r > index->head_dim) return FATHOM_ERR_INVALID_ARG;
@@ -367,6 +372,7 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
                                int32_t *out_idx, float *out_score, void *workspace,
                                size_t workspace_bytes, uint32_t flags, cudaStream_t stream)
 {
+    NvtxRange range("fathom_scan_topk");
     return scan_common(index, 1, &q_bf16, &t, &t_union, k, &out_idx, &out_score, workspace,
                        workspace_bytes, flags, stream);
 }
@@ -389,6 +395,7 @@ fathom_status fathom_scan_topk_batched(const fathom_index *sessions, int32_t n_s
                                        void *workspace, size_t workspace_bytes, uint32_t flags,
                                        cudaStream_t stream)
 {
+    NvtxRange range("fathom_scan_topk_batched");
     return scan_common(sessions, n_sessions, q_bf16, t, t_union, k, out_idx, out_score,
                        workspace, workspace_bytes, flags, stream);
 }
@@ -443,6 +450,7 @@ fathom_status fathom_merge_topk(const int32_t *shard_idx, const float *shard_sco
                                 int32_t k_shard, int32_t k, int32_t *out_idx, float *out_score,
                                 cudaStream_t stream)
 {
+    NvtxRange range("fathom_merge_topk");
     if (!shard_idx || !shard_score || !shard_offset || !out_idx || !out_score)
         return FATHOM_ERR_INVALID_ARG;
     if (n_shards < 1 || n_shards > kMaxMergeShards || n_queries < 1 || k_shard < 1)
@@ -473,6 +481,7 @@ fathom_status fathom_sparse_attention(const float *keys, const float *values, in
                                       float softmax_scale, float *out, void *workspace,
                                       size_t workspace_bytes, cudaStream_t stream)
 {
+    NvtxRange range("fathom_sparse_attention");
     if (n_kv_heads < 1 || group < 1 || group > kMaxGroup || n_keys < 1) return FATHOM_ERR_INVALID_ARG;
     if (head_dim < 32 || head_dim > kMaxHeadDim || head_dim % 32) return FATHOM_ERR_INVALID_ARG;
     if (k < 1 || k > n_keys || !q_bf16 || !idx || !out || !isfinite(softmax_scale))

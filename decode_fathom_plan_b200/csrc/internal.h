@@ -4,10 +4,21 @@
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "fathom.h"
 
 namespace fathom {
+
+// Named NVTX range for the lifetime of a scope: marks each C-ABI call and
+// each scan phase on a profiler's timeline (Nsight Systems); without a
+// profiler attached the calls return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Address of this device's status word (a __device__ int).
 int *device_status_ptr();

@@ -58,6 +58,7 @@ extern "C" fathom_status fathom_scan_topk_static(const fathom_index *index,
                                                  int32_t *out_idx, float *out_score,
                                                  uint32_t flags, cudaStream_t stream)
 {
+    fathom::NvtxRange range("fathom_scan_topk_static");
     const size_t need = fathom_scan_workspace_bytes(index, k);
     if (need == 0) return FATHOM_ERR_INVALID_ARG;
     if (need > kStaticScratchBytes) return FATHOM_ERR_WORKSPACE;   // beyond the fixed maximum
