@@ -376,7 +376,8 @@ def _head_blocks(index, h: int):
     out = []
     for b in range(n_blocks_for(n, block)):
         j0, j1 = b * block, min(n, (b + 1) * block)
-        out.append(((j0, j1), np.ascontiguousarray(index["planes"][h][..., j0 // 32:]),
+        w0, w1 = j0 // 32, (j1 + 31) // 32           # the block's own plane words
+        out.append(((j0, j1), np.ascontiguousarray(index["planes"][h][..., w0:w1]),
                     index["mn"][h, b], index["scale"][h, b]))
     return out
 
