@@ -79,7 +79,7 @@ typedef enum {
     FATHOM_ERR_NONFINITE = 3,     /* non-finite key, query or importance    */
     FATHOM_ERR_TIMEOUT = 4,       /* a bounded device wait ran out          */
     FATHOM_ERR_WORKSPACE = 5,     /* workspace missing or too small         */
-    FATHOM_ERR_UNIMPLEMENTED = 6  /* a mode this build does not provide     */
+    FATHOM_ERR_UNIMPLEMENTED = 6  /* a mode the library does not provide    */
 } fathom_status;
 
 /* Where the planes live.  DEVICE: HBM.  HOST_MAPPED: pinned, device-mapped
