@@ -667,11 +667,13 @@ def run_append(args, wl_name, wl):
     H, G, n, d = wl["H"], wl["G"], wl["n"], wl["d"]
     W, K = max(3, args.warmup), args.steps
     results = []
+    e2e = None
     for m in wl["append"]:
         total = n + (W + K) * m
         sigma, _ = synth.channel_sigma(rank, H, d)
         keys = synth.device_keys(torch, sigma, total, rank)
-        index = fp.KeyIndex(H, G, n, d, wl["residency"], capacity=total)
+        # room for K more appends of the end-to-end leg below
+        index = fp.KeyIndex(H, G, n, d, wl["residency"], capacity=total + K * m)
         index.pack(keys[:, :n].contiguous())
         chunks = [keys[:, n + i * m:n + (i + 1) * m].contiguous() for i in range(W + K)]
         clamped = torch.zeros((H, d), dtype=torch.int32, device="cuda")
@@ -708,6 +710,25 @@ def run_append(args, wl_name, wl):
                         "bytes_per_append": nbytes,
                         "achieved_gbs": nbytes / (med / 1e3) / 1e9,
                         "clamped_keys_total": int(clamped.sum().item())})
+        # end to end through the public call: each step copies its m keys per
+        # KV head in from pinned host memory, appends, and reads the clamp
+        # counters back (host clock)
+        host_chunk = chunks[-1].cpu().pin_memory()
+        stage = torch.empty_like(chunks[-1])
+        cl_host = torch.empty((H, d), dtype=torch.int32).pin_memory()
+        e2e_s = []
+        for i in range(K):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            stage.copy_(host_chunk, non_blocking=True)
+            index.append(stage, clamped)
+            cl_host.copy_(clamped, non_blocking=True)
+            torch.cuda.synchronize()
+            e2e_s.append(time.perf_counter() - t0)
+        assert fp.fathom_last_device_status() == fp.FATHOM_OK
+        e2e = {"value": H * m * K / sum(e2e_s) / 1e9, "unit": "Gkeys/s",
+               "h2d_bytes_per_step": H * m * d * 4, "d2h_bytes_per_step": H * d * 4,
+               "launch_mode": "eager", "m": m}
         del keys, index, chunks
     peak, peak_src = load_peaks()
     bulk = results[-1]
@@ -721,7 +742,7 @@ def run_append(args, wl_name, wl):
                          "unit": "GB/s", "frac": bulk["achieved_gbs"] / peak, "traffic": None,
                          "kernel": f"append_kernel (m = {bulk['m']})",
                          "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},
-            "per_m": results, "launch_mode": "cuda_graph"}
+            "e2e": e2e, "per_m": results, "launch_mode": "cuda_graph"}
     print(json.dumps(line), flush=True)
 
 
@@ -801,6 +822,24 @@ def run_attention_bench(args, wl_name, wl):
                              len(np.intersect1d(buf.idx[i].cpu().numpy(),
                                                 exact_idx[i].cpu().numpy())) / k
                              for i in range(Q)]))})
+    # end to end through the public call: each step copies the queries and the
+    # selected indices in from pinned host memory, attends, and copies the
+    # outputs back (host clock)
+    q_host = q.cpu().pin_memory()
+    idx_host = buf.idx.cpu().pin_memory()
+    idx_stage = torch.empty_like(buf.idx)
+    out_host = torch.empty((Q, d), dtype=torch.float32).pin_memory()
+    e2e_s = []
+    for i in range(K):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        q.copy_(q_host, non_blocking=True)
+        idx_stage.copy_(idx_host, non_blocking=True)
+        attend(idx_stage)
+        out_host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        e2e_s.append(time.perf_counter() - t0)
+    assert fp.fathom_last_device_status() == fp.FATHOM_OK
     nbytes = Q * k * 2 * d * 4
     ms = statistics.median(times)
     peak, peak_src = load_peaks()
@@ -817,6 +856,9 @@ def run_attention_bench(args, wl_name, wl):
                          "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)",
                          "algorithmic_bytes_per_launch": nbytes},
             "attention_error_exact_topk_vs_dense": rel_err(o_exactk),
+            "e2e": {"value": Q * k * K / sum(e2e_s) / 1e9, "unit": "Gkeys/s",
+                    "h2d_bytes_per_step": Q * d * 2 + Q * k * 4,
+                    "d2h_bytes_per_step": Q * d * 4, "launch_mode": "eager"},
             "per_plan": per_plan, "launch_mode": "cuda_graph"}
     print(json.dumps(line), flush=True)
 
