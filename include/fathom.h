@@ -14,6 +14,15 @@
  * and section 解决什么真问题: every decode step ranks n keys and keeps the
  * top-k.
  *
+ * A decode step of one layer, all calls on one stream with no host sync
+ * between them (the sequence may be captured in a CUDA graph):
+ *   fathom_pack_keys once per index, fathom_append_keys as keys arrive;
+ *   fathom_plan (or fathom_plan_marginal / fathom_fixed_plan) per step;
+ *   fathom_scan_topk (workspace sized by fathom_scan_workspace_bytes);
+ *   optionally fathom_sparse_attention over the returned key indices;
+ * then, after a synchronisation, fathom_last_device_status() reports any
+ * error only the device could see.
+ *
  * Conventions for every call:
  *   - All buffers are owned by the caller.  The library allocates no device
  *     or host memory; scratch space is a caller-supplied workspace sized by
