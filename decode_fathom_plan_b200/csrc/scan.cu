@@ -917,6 +917,23 @@ __device__ void bitonic_sort_desc(unsigned long long *x, int kpad)
 constexpr int kBitmapMaxKeys = 1 << 20;                     // index-order output via a bitmap
 constexpr int kChunkWords = 8;                              // bitmap words per prefix entry
 
+// Writes the k selected composites `sel` (okey << 32 | ~index, kpad slots,
+// kpad a power of two >= k) to the outputs in ascending key index by sorting
+// them on the index (bitonic network); for any number of keys.
+__device__ void emit_sorted_by_index(unsigned long long *sel, int k, int kpad, int32_t *out_idx,
+                                     float *out_score)
+{
+    for (int i = threadIdx.x; i < k; i += blockDim.x) sel[i] = (sel[i] << 32) | (sel[i] >> 32);
+    for (int i = k + threadIdx.x; i < kpad; i += blockDim.x) sel[i] = 0ull;
+    __syncthreads();
+    bitonic_sort_desc(sel, kpad);
+    for (int i = threadIdx.x; i < k; i += blockDim.x) {
+        const unsigned long long v = sel[i];
+        out_idx[i] = (int32_t)(~(uint32_t)(v >> 32));
+        out_score[i] = order_key_to_float((uint32_t)(v & 0xFFFFFFFFull));
+    }
+}
+
 // Writes the k selected composites `sel` (okey << 32 | ~index) to the
 // outputs in ascending key index: a bitmap of the selected indices in
 // shared memory (n_keys <= kBitmapMaxKeys) and one prefix count per
@@ -1242,8 +1259,12 @@ __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constan
         }
     }
     __syncthreads();
-    emit_in_index_order(sel, k, S.n, reinterpret_cast<uint32_t *>(x), ss.wsum,
-                        S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
+    if (S.n <= kBitmapMaxKeys)
+        emit_in_index_order(sel, k, S.n, reinterpret_cast<uint32_t *>(x), ss.wsum,
+                            S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
+    else   // the bitmap of so many keys would not fit in shared memory
+        emit_sorted_by_index(sel, k, b.kpad, S.out_idx + (size_t)qq * k,
+                             S.out_score + (size_t)qq * k);
 }
 
 // ------------------------------------------------------------- fallback
@@ -1341,17 +1362,8 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
             }
         }
     }
-    // ascending key index: sort the k selected by ~index, descending
     __syncthreads();   // every selected composite has been written
-    for (int i = threadIdx.x; i < k; i += blockDim.x) sel[i] = (sel[i] << 32) | (sel[i] >> 32);
-    for (int i = k + threadIdx.x; i < b.kpad; i += blockDim.x) sel[i] = 0ull;
-    __syncthreads();
-    bitonic_sort_desc(sel, b.kpad);
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        const unsigned long long v = sel[i];
-        S.out_idx[(size_t)qq * k + i] = (int32_t)(~(uint32_t)(v >> 32));
-        S.out_score[(size_t)qq * k + i] = order_key_to_float((uint32_t)(v & 0xFFFFFFFFull));
-    }
+    emit_sorted_by_index(sel, k, b.kpad, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
 }
 
 // ------------------------------------------------------------- host side
@@ -1380,7 +1392,7 @@ Sizing size_session(int n, int n_words, int k, int block_keys)
     z.n_cols = std::min(n_words, ceil_div(ceil_div(n, 32), 4) * 4);
     z.n_tiles = ceil_div(z.n_cols, kTileCols);
     const int cap = capacity_for(std::min(k, kMaxFastK));
-    z.exact_only = (k > kMaxFastK || n > kBitmapMaxKeys) ? 1 : 0;
+    z.exact_only = (k > kMaxFastK) ? 1 : 0;
     if (z.exact_only || n <= cap) return z;
     const double target = (double)kSampleTargetRank * (double)n / (2.0 * (double)k);
     int m = (int)std::min<double>(std::max<double>(target, kSampleMinKeys), kSampleMaxKeys);
@@ -1509,8 +1521,11 @@ inline size_t bitmap_bytes_for(int n)
 template <int NS>
 size_t final_bitmap_bytes(const Batch<NS> &bt)
 {
+    // sessions past kBitmapMaxKeys keys, and those on the exact path, need no bitmap
     size_t m = 0;
-    for (int s = 0; s < bt.n_sessions; ++s) m = std::max(m, bitmap_bytes_for(bt.s[s].n));
+    for (int s = 0; s < bt.n_sessions; ++s)
+        if (!bt.s[s].exact_only && bt.s[s].n <= kBitmapMaxKeys)
+            m = std::max(m, bitmap_bytes_for(bt.s[s].n));
     return m;
 }
 

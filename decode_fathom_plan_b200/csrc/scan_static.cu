@@ -12,42 +12,30 @@
 // The array below is that workspace: kStaticScratchBytes per GPU, reserved
 // on every device that loads this library and kept until the process exits.
 // Host code may not pass the array's name to a kernel (on the host it is a
-// stand-in, not a device address), so the first call on each device looks up
-// the device address with cudaGetSymbolAddress while that device is current,
-// and later calls reuse it.
-#include <mutex>
-
+// stand-in, not a device address), so every call looks up the device address
+// with cudaGetSymbolAddress while the call's device is current.  Looking it up
+// each time (instead of caching it) keeps the address right after a
+// cudaDeviceReset or a new context on that device, which reloads the module.
 #include "common.cuh"
 #include "internal.h"
 
-// 8 MiB: one Qwen3-8B-shaped layer (32 query heads) at up to 1,048,576 keys
-// with k <= 2048 needs about 7 MiB of per-query state, sampled keys and
-// candidates.
+// 8 MiB: a device index of 64 query heads at 1,048,576 keys with k <= 2048
+// needs about 6.3 MiB (per-query state, candidate buffers, per-KV-head scan
+// tables).  A host-resident index also needs room for the device mirror of
+// its planes, so only small host-resident indices fit.
 static constexpr size_t kStaticScratchBytes = 8u << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kStaticScratchBytes];
 
 namespace {
-std::mutex g_static_mu;
-void *g_static_ptr[64] = {nullptr};
-
-// Device address of g_scan_scratch on the current device (looked up once).
+// Device address of g_scan_scratch on the current device.
 fathom_status static_scratch(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess || !p) {
         cudaGetLastError();
         return FATHOM_ERR_CUDA;
     }
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return FATHOM_ERR_CUDA;
-        }
-        g_static_ptr[dev] = p;
-    }
-    *out = g_static_ptr[dev];
+    *out = p;
     return FATHOM_OK;
 }
 }  // namespace

@@ -283,9 +283,11 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
  *     for it.  For a device index, a layer of 64 query heads at 1,048,576
  *     keys with k <= 2048 needs 6.3 MiB; a host-resident index also needs
  *     room for its plane mirror, so only small ones fit.
- *   - The first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture.
+ *   - Every call looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) on the current device, so the address stays
+ *     right after a device reset.  The first call on a device may also load
+ *     the library's device code there; make that first call before any
+ *     stream capture.
  *   - All calls on a device share the one array.  Calls whose kernels overlap
  *     on the GPU (e.g. on two streams at once) race on it: order them.
  *   - Calls or frees no device memory. */
