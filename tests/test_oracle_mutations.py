@@ -53,6 +53,25 @@ MUTATIONS = {
                                         "const double mean_b = 0.0 + sc *"),
     "attention_unnormalised": ("for (int64_t c = 0; c < d; ++c) out[c] /= denom;",
                                "for (int64_t c = 0; c < d; ++c) out[c] /= (double)cnt;"),
+    "abs_sum_takes_abs_of_the_sum": (
+        "acc += fabs((double)bf16_value(q_bf16[c]) *\n"
+        "                        fo_coarse_midpoint(mn[c], scale[c], tc, u, (int)bits));\n"
+        "        }\n        a[j] = acc;",
+        "acc += ((double)bf16_value(q_bf16[c]) *\n"
+        "                        fo_coarse_midpoint(mn[c], scale[c], tc, u, (int)bits));\n"
+        "        }\n        a[j] = fabs(acc);"),
+    "abs_sum_reads_every_plane": (
+        "int64_t n, int64_t n_words, double *a)\n{\n    if (!fo_bits_ok(bits)) return FO_ERR_ARG;\n"
+        "    for (int64_t j = 0; j < n; ++j) {\n        double acc = 0.0;\n"
+        "        for (int64_t c = 0; c < d; ++c) {\n            int tc = t[c];\n"
+        "            if (tc < 0 || tc > bits) return FO_ERR_ARG;\n            int u = 0;\n"
+        "            for (int slot = 0; slot < tc; ++slot) {",
+        "int64_t n, int64_t n_words, double *a)\n{\n    if (!fo_bits_ok(bits)) return FO_ERR_ARG;\n"
+        "    for (int64_t j = 0; j < n; ++j) {\n        double acc = 0.0;\n"
+        "        for (int64_t c = 0; c < d; ++c) {\n            int tc = t[c];\n"
+        "            if (tc < 0 || tc > bits) return FO_ERR_ARG;\n            int u = 0;\n"
+        "            for (int slot = 0; slot < bits; ++slot) {"),
+    "exact_scores_transposed_keys": ("(double)keys_h[j * d + c]", "(double)keys_h[c * n + j]"),
 }
 
 PIN_TESTS = [
@@ -85,6 +104,8 @@ PIN_TESTS = [
     pins.test_append_8bit_in_range_equals_repacking_and_clamps,
     pins.test_blocked_sigma2_is_the_variance_of_all_dequantised_keys,
     pins.test_blocks_as_large_as_the_keys_are_the_global_quantiser,
+    lambda: pins.test_score_and_absolute_sum_hand_worked(read_golden),
+    lambda: pins.test_exact_scores_hand_worked(read_golden),
 ]
 
 

@@ -234,6 +234,35 @@ def test_coarse_bin_midpoint_hand_worked(golden):
         assert s[0] == kh
 
 
+def test_score_and_absolute_sum_hand_worked(golden):
+    """The score of a key read at t = (2, 1) bits and A_j, the sum of the
+    absolute terms every score tolerance is scaled by, on a key whose terms
+    have opposite signs (|s_j| < A_j) and whose planes past t are set."""
+    g = golden("abs_score_worked.txt")
+    n = int(g["n"][0])
+    planes = np.stack([np.stack([_ints(g[f"ch{c}_slot{s}"]) for s in range(4)])
+                       for c in range(2)]).astype(np.uint32)          # [d][4][n_words]
+    mn = _floats(g["mn"]).astype(np.float32)
+    sc = _floats(g["scale"]).astype(np.float32)
+    q = synth.f32_to_bf16_bits(_floats(g["q"]).astype(np.float32))
+    t = _ints(g["t"]).astype(np.uint8)
+    keys = _ints(g["keys"])
+    s = oracle.score_planes(planes, mn, sc, q, t, n)
+    a = oracle.score_abs_planes(planes, mn, sc, q, t, n)
+    assert np.array_equal(s[keys], _floats(g["s"]))
+    assert np.array_equal(a[keys], _floats(g["A"]))
+    # every other key has code 0 in both channels: the same terms as key 1
+    rest = np.setdiff1d(np.arange(n), keys)
+    assert np.all(a[rest] == a[1]) and np.all(s[rest] == s[1])
+
+
+def test_exact_scores_hand_worked(golden):
+    g = golden("exact_score_worked.txt")
+    keys = np.stack([_floats(g["key0"]), _floats(g["key1"])]).astype(np.float32)   # [n][d]
+    q = synth.f32_to_bf16_bits(_floats(g["q"]).astype(np.float32))
+    assert np.array_equal(oracle.exact_scores(keys, q), _floats(g["s"]))
+
+
 def test_coarse_bin_is_mean_of_its_fine_levels():
     """Reading t bits rebuilds a key at the mean of the 2^(4-t) fine levels of
     its coarse bin (all bins are equally wide)."""
