@@ -71,8 +71,13 @@ WORKLOADS = {
     "qwen3_8b_layer_128k_blocked": dict(H=8, G=4, n=131072, d=128, k=2048, residency="device",
                                         block_keys=2048,
                                         plans=(("wf", 68), ("wf", 92), ("wf", 136))),
+    # the million-token layer with its planes in pinned host memory (the
+    # offloaded setting), followed by the same keys resident in HBM
     "host_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="host_mapped",
-                    plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
+                    plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True,
+                    resident_twin="hbm_1m"),
+    "hbm_1m": dict(H=8, G=4, n=1 << 20, d=128, k=2048, residency="device",
+                   plans=(("wf", 18), ("wf", 68), ("wf", 92), ("wf", 136)), device_keys=True),
     # the host path at a quarter of the keys: the profiling case of the fetch
     # kernel (its traffic scales with n)
     "host_256k": dict(H=8, G=4, n=1 << 18, d=128, k=2048, residency="host_mapped",
@@ -113,7 +118,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
-    p.add_argument("--workload", choices=tuple(WORKLOADS), default="qwen3_8b_layer_128k")
+    p.add_argument("--workload", choices=tuple(WORKLOADS), default="host_1m")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--graph", type=int, default=1,
                    help="replay the timed steps as one CUDA graph (1) or launch them eagerly (0)")
@@ -234,50 +239,98 @@ def measure_host_link(fp, torch, nbytes=1 << 30, reps=10):
 
 
 # ------------------------------------------------------------- CPU oracle
+def host_cpu():
+    """-> (model name from /proc/cpuinfo or None, usable host cores)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        cores = os.cpu_count() or 1
+    return model, cores
+
+
+def _oracle_query_scan(oracle, ref, hi, qrow, spec, k, bits):
+    """One query's plan + fp64 score of every key + full-sort top-k."""
+    if spec[0] == "wf":
+        tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1], bits)
+    elif spec[0] == "mg":
+        tq = oracle.plan_marginal(oracle.importance(qrow, ref["sigma2"][hi]), spec[1], bits)
+    else:
+        tq = oracle.fixed_plan(qrow, spec[1], bits)
+    s = oracle.score_head(ref, hi, qrow, tq)
+    oracle.topk(s, k)
+
+
 def oracle_sample(keys_heads, q_bf16, G, plans, k, ref=None, min_seconds=0.0, bits=4,
-                  block_keys=0):
+                  block_keys=0, threads=1):
     """Time the oracle (plan + fp64 score + full-sort top-k per query) over
     the given KV heads' keys (float32 [h][n][d]) at every plan spec, cycling
-    over (head, plan) until at least min_seconds have passed (one round at
-    least).  The index build (storage side, off the decode path) is not
-    timed.  Returns (seconds, head-scans, keys)."""
+    over (head, plan, query head) until at least min_seconds have passed
+    (every (head, plan) once at least).  threads > 1 runs independent queries
+    on that many host threads at once (the C oracle runs without the GIL).
+    The index build (storage side, off the decode path) is not timed.
+    Returns (seconds, query scans, KV-head keys = query scans * n / G)."""
     import oracle
     if ref is None:
         ref = oracle.build_index(keys_heads, bits=bits, block_keys=block_keys)
+    oracle._load()
     n = keys_heads.shape[1]
-    pairs = [(hi, spec) for hi in range(keys_heads.shape[0]) for spec in plans]
+    items = [(hi, spec, g) for hi in range(keys_heads.shape[0]) for spec in plans
+             for g in range(G)]
+
+    def one(i):
+        hi, spec, g = items[i % len(items)]
+        _oracle_query_scan(oracle, ref, hi, q_bf16[hi * G + g], spec, k, bits)
+
+    done = 0
     t0 = time.perf_counter()
-    scans = 0
-    while scans < len(pairs) or time.perf_counter() - t0 < min_seconds:
-        hi, spec = pairs[scans % len(pairs)]
-        for g in range(G):
-            qrow = q_bf16[hi * G + g]
-            if spec[0] == "wf":
-                tq = oracle.plan_greedy(oracle.importance(qrow, ref["sigma2"][hi]), spec[1],
-                                        bits)
-            elif spec[0] == "mg":
-                tq = oracle.plan_marginal(oracle.importance(qrow, ref["sigma2"][hi]), spec[1],
-                                          bits)
-            else:
-                tq = oracle.fixed_plan(qrow, spec[1], bits)
-            s = oracle.score_head(ref, hi, qrow, tq)
-            oracle.topk(s, k)
-        scans += 1
-    return time.perf_counter() - t0, scans, scans * n
+    if threads <= 1:
+        while done < len(items) or time.perf_counter() - t0 < min_seconds:
+            one(done)
+            done += 1
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        wave = len(items) if min_seconds <= 0 else max(len(items), 2 * threads)
+        with ThreadPoolExecutor(max_workers=threads) as pool:
+            while done < len(items) or time.perf_counter() - t0 < min_seconds:
+                list(pool.map(one, range(done, done + wave)))
+                done += wave
+    secs = time.perf_counter() - t0
+    return secs, done, done * n / G
 
 
 CPU_BASELINE_SECONDS = 12.0
 
 
 def cpu_baseline(keys_heads, q_bf16, G, plans, k, bits=4, block_keys=0):
-    """About 12 s of single-thread oracle work on a few KV heads."""
-    secs, scans, keys = oracle_sample(keys_heads, q_bf16, G, plans, k,
-                                      min_seconds=CPU_BASELINE_SECONDS, bits=bits,
-                                      block_keys=block_keys)
-    return {"value": keys / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{scans} scans of one KV head ({G} query heads, {keys_heads.shape[1]} "
-                      f"keys) cycling over {keys_heads.shape[0]} KV head(s) x plans "
-                      f"{[plan_name(p) for p in plans]}, single thread, {secs:.1f} s"}
+    """The oracle on the host cores, on a sample of the workload: about 12 s
+    on one thread, then about 12 s with one query scan per host core at a
+    time.  value / cores: the all-core run."""
+    import oracle
+    ref = oracle.build_index(keys_heads, bits=bits, block_keys=block_keys)
+    model, cores = host_cpu()
+    plan_names = [plan_name(p) for p in plans]
+    n = keys_heads.shape[1]
+    s1, q1, keys1 = oracle_sample(keys_heads, q_bf16, G, plans, k, ref,
+                                  min_seconds=CPU_BASELINE_SECONDS, bits=bits)
+    sa, qa, keysa = oracle_sample(keys_heads, q_bf16, G, plans, k, ref,
+                                  min_seconds=CPU_BASELINE_SECONDS, bits=bits, threads=cores)
+    what = (f"query scans (plan + fp64 score of all {n} keys + full-sort top-k) cycling over "
+            f"{keys_heads.shape[0]} KV head(s) x {G} query heads x plans {plan_names}")
+    return {"value": keysa / sa / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{qa} {what}, {cores} threads, {sa:.1f} s; KV-head keys = query scans "
+                      f"x n / {G}",
+            "single_thread": {"value": keys1 / s1 / 1e9, "unit": UNIT, "cores": 1,
+                              "sample": f"{q1} {what}, one thread, {s1:.1f} s"},
+            "host_cpu": model, "nproc": cores}
 
 
 def reference_plans(wl):
@@ -287,34 +340,40 @@ def reference_plans(wl):
 
 
 def run_reference(args, wl_name, wl):
+    """The oracle as the reference arm: every step scans one KV head of the
+    workload at its full key count once per plan (each of its G query heads),
+    the query scans spread over the host cores."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    n = wl["n"] if (wl["n"] and wl["residency"] == "device") else min(wl["n"] or (1 << 18), 1 << 18)
+    n = wl["n"] or (1 << 18)
     plans = reference_plans(wl)
     bits = wl.get("bits", 4)
     ses = synth.make_session(0, 1, wl["G"], n, plan_bits(plans[0], bits), head_dim=wl["d"])
     import oracle
     ref = oracle.build_index(ses.keys[:1], bits=bits, block_keys=wl.get("block_keys", 0))
-    times = []
+    model, cores = host_cpu()
+    threads = min(cores, len(plans) * wl["G"])
+    times, keys = [], 0.0
     for i in range(args.warmup + args.steps):
-        secs, _, _ = oracle_sample(ses.keys[:1], ses.q_bf16, wl["G"], (plans[i % len(plans)],),
-                                   wl["k"], ref, bits=bits)
+        secs, _, kk = oracle_sample(ses.keys[:1], ses.q_bf16, wl["G"], plans, wl["k"], ref,
+                                    bits=bits, threads=threads)
         if i >= args.warmup:
             times.append(secs)
-    keys_per_step = n                      # one KV head, one plan, per step
+            keys += kk
     total = sum(times)
-    value = keys_per_step * len(times) / total / 1e9
-    sample = (f"each step: 1 of {wl['H']} KV heads ({wl['G']} query heads), one plan "
-              f"(cycling {[plan_name(p) for p in plans]}), {n} keys, single thread")
+    value = keys / total / 1e9
+    sample = (f"each step: 1 of {wl['H']} KV heads ({wl['G']} query heads) once per plan "
+              f"{[plan_name(p) for p in plans]}, {n} keys, query scans on {threads} threads "
+              f"of {cores} cores ({model})")
     cfg = config_of(wl_name, dict(wl, n=n, plans=plans), "n/a (CPU)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": cfg,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample, "host_cpu": model, "nproc": cores},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -415,13 +474,58 @@ def run_fathom(args, wl_name, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     fp.load_library()
+    sessions = build_sessions(wl, rank, torch, fp)
+    assert fp.fathom_last_device_status() == fp.FATHOM_OK
+    link = measure_host_link(fp, torch) if wl["residency"] != "device" else None
+    line = measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp)
+
+    twin_name = wl.get("resident_twin")
+    if twin_name:
+        # the same keys and queries with the index resident in HBM: the
+        # resident mode of the same configuration, as a sub-record
+        twin = WORKLOADS[twin_name]
+        for S in sessions:
+            S["index"] = None
+        torch.cuda.empty_cache()
+        for S in sessions:
+            ix = fp.KeyIndex(twin["H"], twin["G"], S["n"], twin["d"], twin["residency"])
+            ix.pack(S["keys"])
+            S["index"] = ix
+        torch.cuda.synchronize()
+        assert fp.fathom_last_device_status() == fp.FATHOM_OK
+        sub = measure_workload(args, twin_name, twin, sessions, None, dist, torch, fp)
+        line["hbm_resident"] = {key: sub[key] for key in (
+            "value", "unit", "ms_per_step", "config", "e2e", "gpu_launches", "roofline",
+            "clocks", "per_plan", "step_ms_median")}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        S0 = sessions[0]
+        H, G, k = wl["H"], wl["G"], wl["k"]
+        nh = max(1, min(H, (8 * 131072) // S0["n"]))
+        line["cpu_baseline"] = cpu_baseline(S0["keys"][:nh].cpu().numpy(),
+                                            S0["q"][0].cpu().numpy().view(np.uint16), G,
+                                            S0["plans"], k, wl.get("bits", 4),
+                                            wl.get("block_keys", 0))
+        if "hbm_resident" in line:
+            line["hbm_resident"]["cpu_baseline"] = dict(
+                line["cpu_baseline"], note="the oracle reads host memory either way: "
+                                           "the same measurement as the host-resident line")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp):
+    """Time K steps of one workload over its packed sessions (device-timed
+    value, roofline of the dominant kernel, end to end through the public
+    API) and return its JSON line (without the CPU baseline).  Every rank
+    calls it in the same order (one all-reduce)."""
+    rank, world, local = dist_env()
     H, G, d, k = wl["H"], wl["G"], wl["d"], wl["k"]
     Q = H * G
     batched = bool(wl.get("batched"))
-    sessions = build_sessions(wl, rank, torch, fp)
-    assert fp.fathom_last_device_status() == fp.FATHOM_OK
-
-    link = measure_host_link(fp, torch) if wl["residency"] != "device" else None
     W, K = max(3, args.warmup), args.steps
     # scans of one step: (session, plan spec, buffers, budget vector)
     jobs = []
@@ -639,18 +743,7 @@ def run_fathom(args, wl_name, wl):
             "step_ms_median": statistics.median(step_ms)}
     if link is not None:
         line["host_link"] = link
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        S0 = sessions[0]
-        nh = max(1, min(H, (8 * 131072) // S0["n"]))
-        line["cpu_baseline"] = cpu_baseline(S0["keys"][:nh].cpu().numpy(),
-                                            S0["q"][0].cpu().numpy().view(np.uint16), G,
-                                            S0["plans"], k, wl.get("bits", 4),
-                                            wl.get("block_keys", 0))
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+    return line
 
 
 def run_append(args, wl_name, wl):
