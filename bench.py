@@ -120,6 +120,9 @@ def parse_args():
     p.add_argument("--impl", choices=("fathom", "reference"), default="fathom")
     p.add_argument("--workload", choices=tuple(WORKLOADS), default="host_1m")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-recall", action="store_true",
+                   help="free the float32 keys once packed and skip the recall check (keeps "
+                        "profiler runs small on the device)")
     p.add_argument("--graph", type=int, default=1,
                    help="replay the timed steps as one CUDA graph (1) or launch them eagerly (0)")
     p.add_argument("--heat-seconds", type=float, default=1.0,
@@ -476,11 +479,15 @@ def run_fathom(args, wl_name, wl):
     fp.load_library()
     sessions = build_sessions(wl, rank, torch, fp)
     assert fp.fathom_last_device_status() == fp.FATHOM_OK
+    if args.no_recall:
+        for S in sessions:
+            S["keys"] = None
+        torch.cuda.empty_cache()
     link = measure_host_link(fp, torch) if wl["residency"] != "device" else None
     line = measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp)
 
     twin_name = wl.get("resident_twin")
-    if twin_name:
+    if twin_name and not args.no_recall:   # the twin is packed from the same keys
         # the same keys and queries with the index resident in HBM: the
         # resident mode of the same configuration, as a sub-record
         twin = WORKLOADS[twin_name]
@@ -498,7 +505,7 @@ def run_fathom(args, wl_name, wl):
             "value", "unit", "ms_per_step", "config", "e2e", "gpu_launches", "roofline",
             "clocks", "per_plan", "step_ms_median")}
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_recall:
         S0 = sessions[0]
         H, G, k = wl["H"], wl["G"], wl["k"]
         nh = max(1, min(H, (8 * 131072) // S0["n"]))
@@ -642,7 +649,7 @@ def measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp):
             qf = S["q"][W + K - 1].view(torch.bfloat16).float().reshape(H, G, d)
             got = j["buf"].idx.reshape(H, G, k).long()
             rec = []
-            for h in range(H):
+            for h in range(H if S["keys"] is not None else 0):
                 exact = (S["keys"][h] @ qf[h].T).topk(k, dim=0).indices.T     # [G][k]
                 for g in range(G):
                     inter = np.intersect1d(exact[g].cpu().numpy(), got[h, g].cpu().numpy())
@@ -652,7 +659,7 @@ def measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp):
                              "bytes_per_query": float(qb.mean()),
                              "union_bytes_per_kv_head": float(ub.mean()),
                              "union_factor": float(ub.sum() / (qb.sum() / G)),
-                             "recall_vs_exact_fp32": float(np.mean(rec))})
+                             "recall_vs_exact_fp32": float(np.mean(rec)) if rec else None})
 
     # end to end through the public API with host buffers
     q_host = [torch.from_numpy(S["q"][W:W + K].cpu().numpy()).pin_memory() for S in sessions]

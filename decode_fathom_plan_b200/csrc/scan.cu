@@ -93,6 +93,7 @@ struct SessionDesc {
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
     int chunks, chunk_begin;   // main-scan chunks per KV head, first chunk's CTA
+    int chunk_q, chunk_rem;    // col_groups = chunks * chunk_q + chunk_rem (one scale per channel)
     int q_begin, head_begin;
 };
 
@@ -706,8 +707,6 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
 {
     __shared__ ScanMeta<GP> sm;
     __shared__ uint32_t s_theta[GP];
-    __shared__ unsigned s_wtot[kScanThreads / 32][GP];   // candidates per (warp, query)
-    __shared__ unsigned s_woff[kScanThreads / 32][GP];   // their first slot
     extern __shared__ __align__(16) uint32_t scan_dyn[];
     StageBuf stage = reinterpret_cast<StageBuf>(scan_dyn);
     const int G = b.G;
@@ -733,8 +732,9 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
             g0 = gb0 + (int)((long long)sub * gbn / cpb);
             g1 = gb0 + (int)((long long)(sub + 1) * gbn / cpb);
         } else {
-            g0 = (int)((long long)c * S.col_groups / S.chunks);
-            g1 = (int)((long long)(c + 1) * S.col_groups / S.chunks);
+            // the first chunk_rem chunks take one column group more
+            g0 = c * S.chunk_q + min(c, S.chunk_rem);
+            g1 = g0 + S.chunk_q + (c < S.chunk_rem ? 1 : 0);
         }
         const int col_lo = g0 * 4;
         const int width = (g1 - g0) * 4;               // plane words owned by this chunk
@@ -749,68 +749,49 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
 
-        // keys scoring >= theta: counts per warp and query, one reservation
-        // per (CTA, query) in the query's candidate buffer, then the writes
+        // keys scoring >= theta: each warp reserves room for its own keys in
+        // each query's candidate buffer (one atomic per query with any such
+        // key; no CTA-wide step), then writes them
         const bool mine = col < width && col_lo + col < col_hi;
         const int key0 = (col_lo + col) * 32 + r;
         // keys key0 + 4m for m < live are real keys (the rest pad the last word)
         const int live = mine ? max(0, min(8, (S.n - key0 + 3) >> 2)) : 0;
         const unsigned live_mask = (1u << live) - 1u;
-        unsigned pass[GP];
-        int before[GP];
+        if (col_lo + (warp << 3) >= col_hi) return;   // no keys in this warp
 #pragma unroll
         for (int gg = 0; gg < GP; ++gg) {
-            pass[gg] = 0u;
-            before[gg] = 0;
-            if (gg < G) {
-                const float bias = sm.bias[gg];
-                // order_key(s) >= theta  <=>  s >= theta's float (up to the sign
-                // of zero, which can only add a candidate); theta 0 passes all
-                const uint32_t theta = s_theta[gg];
-                const float theta_f = theta == 0u ? -INFINITY : order_key_to_float(theta);
+            if (gg >= G) break;
+            const float bias = sm.bias[gg];
+            // order_key(s) >= theta  <=>  s >= theta's float (up to the sign
+            // of zero, which can only add a candidate); theta 0 passes all
+            const uint32_t theta = s_theta[gg];
+            const float theta_f = theta == 0u ? -INFINITY : order_key_to_float(theta);
+            unsigned pass = 0u;
 #pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    pass[gg] |= (score_of(acc[gg], m, bias) >= theta_f) ? (1u << m) : 0u;
-                pass[gg] &= live_mask;
-                const int cnt = __popc(pass[gg]);
-                int inc = cnt;
+            for (int m = 0; m < 8; ++m)
+                pass |= (score_of(acc[gg], m, bias) >= theta_f) ? (1u << m) : 0u;
+            pass &= live_mask;
+            if (!__any_sync(0xFFFFFFFFu, pass != 0u)) continue;
+            const int cnt = __popc(pass);
+            int inc = cnt;
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
-                    if (lane >= off) inc += y;
-                }
-                before[gg] = inc - cnt;
-                if (lane == 31) s_wtot[warp][gg] = (unsigned)inc;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+                if (lane >= off) inc += y;
             }
-        }
-        __syncthreads();
-        if (threadIdx.x < G) {
-            const int gg = threadIdx.x;
-            unsigned tot = 0;
+            unsigned at = 0;
+            if (lane == 31) at = atomicAdd(&S.qstate[(q0 + gg) * kQueryStateWords + 1], (unsigned)inc);
+            at = __shfl_sync(0xFFFFFFFFu, at, 31);
+            if (!pass) continue;
+            unsigned pos = at + (unsigned)(inc - cnt);
+            unsigned long long *cq = S.cand + (size_t)(q0 + gg) * b.cap;
 #pragma unroll
-            for (int w = 0; w < kScanThreads / 32; ++w) tot += s_wtot[w][gg];
-            unsigned at = tot ? atomicAdd(&S.qstate[(q0 + gg) * kQueryStateWords + 1], tot) : 0u;
-#pragma unroll
-            for (int w = 0; w < kScanThreads / 32; ++w) {
-                s_woff[w][gg] = at;
-                at += s_wtot[w][gg];
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int gg = 0; gg < GP; ++gg) {
-            if (gg < G && pass[gg]) {
-                const float bias = sm.bias[gg];
-                unsigned pos = s_woff[warp][gg] + (unsigned)before[gg];
-                unsigned long long *cq = S.cand + (size_t)(q0 + gg) * b.cap;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    if (pass[gg] & (1u << m)) {
-                        if (pos < (unsigned)b.cap)
-                            cq[pos] = composite(order_key(score_of(acc[gg], m, bias)),
-                                                (uint32_t)(key0 + 4 * m));
-                        ++pos;
-                    }
+            for (int m = 0; m < 8; ++m) {
+                if (pass & (1u << m)) {
+                    if (pos < (unsigned)b.cap)
+                        cq[pos] = composite(order_key(score_of(acc[gg], m, bias)),
+                                            (uint32_t)(key0 + 4 * m));
+                    ++pos;
                 }
             }
         }
@@ -1697,8 +1678,11 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     }
     groups = 0;
     for (int s = 0; s < n_sessions; ++s) {
-        bt.s[s].chunk_begin = groups;
-        groups += bt.s[s].H * bt.s[s].chunks;
+        SessionDesc &D = bt.s[s];
+        D.chunk_begin = groups;
+        D.chunk_q = D.col_groups / D.chunks;
+        D.chunk_rem = D.col_groups - D.chunk_q * D.chunks;
+        groups += D.H * D.chunks;
     }
     const int G = bt.G;
     if (blocks > 0) {   // every session has grouped scales (the C ABI checks)
