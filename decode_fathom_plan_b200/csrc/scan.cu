@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(kScanThreads, (GP >= 8) ? 2 : 4)
 scan_kernel(const __grid_constant__ Batch<NS> b)
 {
     __shared__ ScanMeta<GP> sm;
-    __shared__ uint32_t s_theta[GP];
+    __shared__ float s_theta_f[GP];
     extern __shared__ __align__(16) uint32_t scan_dyn[];
     StageBuf stage = reinterpret_cast<StageBuf>(scan_dyn);
     const int G = b.G;
@@ -740,11 +740,15 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
         const int width = (g1 - g0) * 4;               // plane words owned by this chunk
         const int col_hi = min(S.n_cols, col_lo + width);
         const int q0 = h * G;
-        if (threadIdx.x < GP)
-            s_theta[threadIdx.x] = (threadIdx.x < G)
+        if (threadIdx.x < GP) {
+            // order_key(s) >= theta  <=>  s >= theta's float (up to the sign of
+            // zero, which can only add a candidate); theta 0 passes every key
+            const uint32_t theta = (threadIdx.x < G)
                                        ? S.qstate[(q0 + threadIdx.x) * kQueryStateWords + 0]
                                        : 0xFFFFFFFFu;
-        load_head<GP>(sm, S.tables, h);
+            s_theta_f[threadIdx.x] = theta == 0u ? -INFINITY : order_key_to_float(theta);
+        }
+        load_head<GP>(sm, S.tables, h);   // ends with a barrier
         if constexpr (kBlocked) apply_block<GP>(sm, S, h, blk, G, b.d);
         float2 acc[GP][4];
         scan_chunk<GP, STAGES>(sm, stage, S.planes, S.n_words, col_lo, col_hi, acc);
@@ -752,26 +756,26 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
         // keys scoring >= theta: each warp reserves room for its own keys in
         // each query's candidate buffer (one atomic per query with any such
         // key; no CTA-wide step), then writes them
+        if (col_lo + (warp << 3) >= col_hi) return;   // no keys in this warp
         const bool mine = col < width && col_lo + col < col_hi;
         const int key0 = (col_lo + col) * 32 + r;
         // keys key0 + 4m for m < live are real keys (the rest pad the last word)
         const int live = mine ? max(0, min(8, (S.n - key0 + 3) >> 2)) : 0;
         const unsigned live_mask = (1u << live) - 1u;
-        if (col_lo + (warp << 3) >= col_hi) return;   // no keys in this warp
 #pragma unroll
         for (int gg = 0; gg < GP; ++gg) {
             if (gg >= G) break;
             const float bias = sm.bias[gg];
-            // order_key(s) >= theta  <=>  s >= theta's float (up to the sign
-            // of zero, which can only add a candidate); theta 0 passes all
-            const uint32_t theta = s_theta[gg];
-            const float theta_f = theta == 0u ? -INFINITY : order_key_to_float(theta);
+            const float th = s_theta_f[gg];
+            // first the thread's best key: most warps hold no key >= theta
+            float mx = fmaxf(fmaxf(acc[gg][0].x, acc[gg][0].y), fmaxf(acc[gg][1].x, acc[gg][1].y));
+            mx = fmaxf(mx, fmaxf(fmaxf(acc[gg][2].x, acc[gg][2].y), fmaxf(acc[gg][3].x, acc[gg][3].y)));
+            if (!__any_sync(0xFFFFFFFFu, live > 0 && bias + mx >= th)) continue;
             unsigned pass = 0u;
 #pragma unroll
             for (int m = 0; m < 8; ++m)
-                pass |= (score_of(acc[gg], m, bias) >= theta_f) ? (1u << m) : 0u;
+                pass |= (score_of(acc[gg], m, bias) >= th) ? (1u << m) : 0u;
             pass &= live_mask;
-            if (!__any_sync(0xFFFFFFFFu, pass != 0u)) continue;
             const int cnt = __popc(pass);
             int inc = cnt;
 #pragma unroll
@@ -780,19 +784,20 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
                 if (lane >= off) inc += y;
             }
             unsigned at = 0;
-            if (lane == 31) at = atomicAdd(&S.qstate[(q0 + gg) * kQueryStateWords + 1], (unsigned)inc);
+            if (lane == 31 && inc) at = atomicAdd(&S.qstate[(q0 + gg) * kQueryStateWords + 1], (unsigned)inc);
             at = __shfl_sync(0xFFFFFFFFu, at, 31);
-            if (!pass) continue;
             unsigned pos = at + (unsigned)(inc - cnt);
             unsigned long long *cq = S.cand + (size_t)(q0 + gg) * b.cap;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                if (pass & (1u << m)) {
-                    if (pos < (unsigned)b.cap)
-                        cq[pos] = composite(order_key(score_of(acc[gg], m, bias)),
-                                            (uint32_t)(key0 + 4 * m));
-                    ++pos;
-                }
+            while (pass) {   // the set bits only
+                const int m = __ffs(pass) - 1;
+                pass &= pass - 1u;
+                const float2 p01 = (m & 1) ? acc[gg][1] : acc[gg][0];
+                const float2 p23 = (m & 1) ? acc[gg][3] : acc[gg][2];
+                const float2 p = (m & 2) ? p23 : p01;
+                const float sc = bias + ((m & 4) ? p.y : p.x);
+                if (pos < (unsigned)b.cap)
+                    cq[pos] = composite(order_key(sc), (uint32_t)(key0 + 4 * m));
+                ++pos;
             }
         }
     }
