@@ -727,12 +727,16 @@ def measure_workload(args, wl_name, wl, sessions, link, dist, torch, fp):
     else:
         peak = max(link["h2d_memcpy_gbs"], link["zero_copy_read_gbs"])
         bound, peak_note = "host_link", "measured in this run: max(pinned copy, zero-copy read)"
-        kernel = "fetch_kernel (union planes, host -> device mirror)"
+        kernel = ("fetch_kernel, one launch per unit of KV heads (union planes, host -> "
+                  "device ring), timed from the first unit's fetch to the last one's end")
     traffic, traffic_note = recorded_traffic(wl_name, wl, "fetch_kernel" if link else "scan_kernel")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_note,
                 "kernel": kernel,
                 "peak_source": peak_note, "avg_launch_us": avg_launch_ms * 1e3,
+                # the whole step against the same peak: every plan's union bytes
+                # over the device-timed step (fetch, scoring, selection, plans)
+                "step_level_frac": union_bytes_total / (total_ms / K / 1e3) / 1e9 / peak,
                 "algorithmic_bytes_per_launch": bytes_per_launch}
 
     cfg = config_of(wl_name, wl, "flushed between steps (256 MiB write)",

@@ -7,8 +7,9 @@
 // union plan's planes once: for channel c the first T_c = t_union[h][c]
 // slots, which are adjacent in the channel-major layout [H][d][4][n_words],
 // so every (head, channel) pair is one contiguous span of
-// T_c * n_words * 4 bytes.  They land at the same offsets of a device mirror
-// of the index; slots past T_c are neither copied nor read afterwards.
+// T_c * n_words * 4 bytes.  They land at the same offsets of a device ring
+// slot laid out like the fetched heads of the index; slots past T_c are
+// neither copied nor read afterwards.
 //
 // The copy streams at the link's rate only while every SM keeps loads in
 // flight without pause, so the work is split into 16 KB items (one per CTA
@@ -94,7 +95,7 @@ fetch_kernel(const __grid_constant__ FetchBatch b)
 
 }  // namespace
 
-cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream)
+cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream, int ctas_per_sm)
 {
     if (n_jobs <= 0) return cudaSuccess;
     if (n_jobs > kMaxSessions) return cudaErrorInvalidValue;
@@ -114,7 +115,8 @@ cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    const long long ctas = std::min<long long>(items, (long long)std::max(1, n_sm) * kFetchCtasPerSm);
+    const int per_sm = std::max(1, std::min(ctas_per_sm, kFetchCtasPerSm));
+    const long long ctas = std::min<long long>(items, (long long)std::max(1, n_sm) * per_sm);
     fetch_kernel<<<(int)ctas, kFetchThreads, 0, stream>>>(b);
     note_launch(1);
     return cudaGetLastError();

@@ -89,12 +89,15 @@ cudaError_t launch_lift(const LiftArgs &a, cudaStream_t stream);
 // (head, channel) pairs, the first t_union[hc] slots of n_words words.
 struct FetchJob {
     const uint32_t *src;       // device-mapped host planes [H][d][4][n_words]
-    uint32_t *dst;             // device mirror, same layout
+    uint32_t *dst;             // device ring slot, same layout
     const uint8_t *t_union;    // [H][d]
     int n_channels;
     int n_words;
 };
-cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream);
+// CTAs per multiprocessor of a fetch that shares the GPU with the scoring
+// kernels of the previous unit (the link needs few SMs to stay busy).
+constexpr int kFetchCtasPerSmShared = 2;
+cudaError_t launch_fetch(const FetchJob *jobs, int n_jobs, cudaStream_t stream, int ctas_per_sm);
 
 // ---- attention.cu
 // Split-K runs per query for k selected keys.

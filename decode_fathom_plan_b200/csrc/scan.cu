@@ -31,8 +31,8 @@
 // float by OR-ing it under the mantissa of a power of two and subtracting
 // that power (exact), two at a time with __fadd2_rn; each reading query head
 // adds W*v with __ffma2_rn (two keys per instruction).  One CTA per 64-word
-// chunk of a KV head; host-resident planes are first fetched into a device
-// mirror (fetch.cu) and read from there.
+// chunk of a KV head; host-resident planes are fetched a unit of KV heads at
+// a time into a two-slot device ring (fetch.cu) and read from there.
 //
 // No tensor cores: this is a sparse binary-weighted reduction.
 //
@@ -56,6 +56,10 @@
 
 #include <algorithm>
 #include <cmath>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -1400,7 +1404,7 @@ Sizing size_session(int n, int n_words, int k, int block_keys)
 }
 
 struct WsLayout {
-    size_t qstate, cand, tables, bias_blk, mirror, total;
+    size_t qstate, cand, tables, bias_blk, total;
 };
 
 // Query heads per KV head rounded up to the kernels' template width.
@@ -1415,13 +1419,7 @@ inline size_t head_table_bytes(int G)
     }
 }
 
-// A host-resident index is fetched into a device mirror of its planes
-// before the scoring passes (fetch.cu); the mirror is part of the workspace.
 inline bool host_resident(const fathom_index &ix) { return ix.residency == FATHOM_RES_HOST_MAPPED; }
-inline size_t plane_bytes(const fathom_index &ix)
-{
-    return (size_t)ix.n_kv_heads * (size_t)ix.head_dim * kBits * (size_t)ix.n_words * sizeof(uint32_t);
-}
 
 WsLayout layout_session(const fathom_index &ix, int k, size_t at)
 {
@@ -1437,8 +1435,6 @@ WsLayout layout_session(const fathom_index &ix, int k, size_t at)
     L.bias_blk = at;   // grouped scales: a bias per (KV head, block, query head)
     if (ix.block_keys)
         at += align256((size_t)ix.n_kv_heads * index_blocks(ix) * ix.group * sizeof(float));
-    L.mirror = at;
-    if (host_resident(ix)) at += align256(plane_bytes(ix));
     L.total = at;
     return L;
 }
@@ -1517,22 +1513,12 @@ size_t final_bitmap_bytes(const Batch<NS> &bt)
 
 template <int NS, int GP, bool kBlocked>
 cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, int total_heads,
-                      int total_blocks, int max_m_keys,
-                      const FetchJob *fetch, int n_fetch, uint32_t flags, cudaStream_t stream,
+                      int total_blocks, int max_m_keys, uint32_t flags, cudaStream_t stream,
                       ScanProfileHook *hook)
 {
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
     int launches = 0;
-    if (n_fetch > 0) {
-        // host-resident planes: bring the union plan's planes into the mirror
-        if (hook && hook->enabled) record_timing_event(hook->begin, stream);
-        if ((e = launch_fetch(fetch, n_fetch, stream)) != cudaSuccess) return note_error(e, "fetch launch");
-        if (hook && hook->enabled) {
-            record_timing_event(hook->end, stream);
-            hook->recorded = true;
-        }
-    }
     if (kBlocked) {
         // grouped scales: the bias of every (KV head, block, query head)
         block_bias_kernel<NS><<<total_blocks, kScanThreads, 0, stream>>>(bt);
@@ -1558,7 +1544,7 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
         ++launches;
     }
     if (!force && total_chunks > 0) {
-        const bool timed = hook && hook->enabled && n_fetch == 0;
+        const bool timed = hook && hook->enabled;
         static int main_smem_set[64];
         auto kern = scan_kernel<NS, GP, kMainStages, kBlocked>;
         const size_t dyn = kMainStages * kStageBytes;
@@ -1608,8 +1594,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    int groups = 0, queries = 0, heads = 0, blocks = 0, max_m = 0, n_fetch = 0;
-    FetchJob fetch[NS];
+    int groups = 0, queries = 0, heads = 0, blocks = 0, max_m = 0;
     size_t at = 0;
     char *base = static_cast<char *>(ws);
     for (int s = 0; s < n_sessions; ++s) {
@@ -1618,13 +1603,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         const WsLayout L = layout_session(ix, k, at);
         at = L.total;
         SessionDesc &D = bt.s[s];
-        D.planes = ix.planes;
-        if (host_resident(ix)) {
-            uint32_t *mirror = reinterpret_cast<uint32_t *>(base + L.mirror);
-            fetch[n_fetch++] = FetchJob{ix.planes, mirror, ss[s].t_union,
-                                        ix.n_kv_heads * ix.head_dim, ix.n_words};
-            D.planes = mirror;
-        }
+        D.planes = ix.planes;   // device rows (a host-resident index arrives as ring-slot views)
         D.mn = ix.mn;
         D.scale = ix.scale;
         D.q = ss[s].q;
@@ -1691,29 +1670,180 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     }
     const int G = bt.G;
     if (blocks > 0) {   // every session has grouped scales (the C ABI checks)
-        if (G <= 1) return run_batch<NS, 1, true>(bt, groups, queries, heads, blocks, max_m, fetch,
-                                                  n_fetch, flags, stream, hook);
-        if (G <= 2) return run_batch<NS, 2, true>(bt, groups, queries, heads, blocks, max_m, fetch,
-                                                  n_fetch, flags, stream, hook);
-        if (G <= 4) return run_batch<NS, 4, true>(bt, groups, queries, heads, blocks, max_m, fetch,
-                                                  n_fetch, flags, stream, hook);
-        return run_batch<NS, 8, true>(bt, groups, queries, heads, blocks, max_m, fetch, n_fetch,
-                                      flags, stream, hook);
+        if (G <= 1) return run_batch<NS, 1, true>(bt, groups, queries, heads, blocks, max_m, flags, stream, hook);
+        if (G <= 2) return run_batch<NS, 2, true>(bt, groups, queries, heads, blocks, max_m, flags, stream, hook);
+        if (G <= 4) return run_batch<NS, 4, true>(bt, groups, queries, heads, blocks, max_m, flags, stream, hook);
+        return run_batch<NS, 8, true>(bt, groups, queries, heads, blocks, max_m, flags, stream, hook);
     }
-    if (G <= 1) return run_batch<NS, 1, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
-                                               flags, stream, hook);
-    if (G <= 2) return run_batch<NS, 2, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
-                                               flags, stream, hook);
-    if (G <= 4) return run_batch<NS, 4, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch,
-                                               flags, stream, hook);
-    return run_batch<NS, 8, false>(bt, groups, queries, heads, 0, max_m, fetch, n_fetch, flags,
+    if (G <= 1) return run_batch<NS, 1, false>(bt, groups, queries, heads, 0, max_m, flags, stream, hook);
+    if (G <= 2) return run_batch<NS, 2, false>(bt, groups, queries, heads, 0, max_m, flags, stream, hook);
+    if (G <= 4) return run_batch<NS, 4, false>(bt, groups, queries, heads, 0, max_m, flags, stream, hook);
+    return run_batch<NS, 8, false>(bt, groups, queries, heads, 0, max_m, flags,
                                    stream, hook);
+}
+
+
+// ------------------------------------------------- host-resident indices
+// A scan over host-resident planes is pipelined over units of KV heads (one
+// head per unit for a single session, one session per unit for a batch): the
+// union planes of unit u + 1 cross the host link into one slot of a two-slot
+// device ring while unit u is scored from the other slot, so only the last
+// unit's scoring adds to the link time, and the device holds two units'
+// planes instead of the whole index.  The fetches run on a side stream that
+// forks from the caller's stream and joins it again before the call returns
+// (event waits only, so the sequence can be captured in a CUDA graph).
+struct HostUnit {
+    int s, h0, nh;   // session, first KV head, KV heads
+};
+
+inline bool any_host(const fathom_index *sessions, int n)
+{
+    for (int s = 0; s < n; ++s)
+        if (host_resident(sessions[s])) return true;
+    return false;
+}
+
+std::vector<HostUnit> host_units(const fathom_index *sessions, int n)
+{
+    std::vector<HostUnit> u;
+    for (int s = 0; s < n; ++s) {
+        if (n == 1)
+            for (int h = 0; h < sessions[s].n_kv_heads; ++h) u.push_back(HostUnit{s, h, 1});
+        else
+            u.push_back(HostUnit{s, 0, sessions[s].n_kv_heads});
+    }
+    return u;
+}
+
+// Heads h0 .. h0+nh-1 of an index as a device-resident index of nh heads
+// whose planes start at `planes` (a ring slot, or the index's own rows).
+fathom_index unit_view(const fathom_index &ix, int h0, int nh, uint32_t *planes)
+{
+    fathom_index v = ix;
+    const size_t stat = (size_t)h0 * index_blocks(ix) * ix.head_dim;
+    v.n_kv_heads = nh;
+    v.residency = FATHOM_RES_DEVICE;
+    v.planes = planes;
+    v.mn = ix.mn + stat;
+    v.scale = ix.scale + stat;
+    v.sigma2 = ix.sigma2 ? ix.sigma2 + (size_t)h0 * ix.head_dim : nullptr;
+    v.sum_code = ix.sum_code ? ix.sum_code + stat : nullptr;
+    v.sum_code2 = ix.sum_code2 ? ix.sum_code2 + stat : nullptr;
+    return v;
+}
+
+inline size_t head_plane_bytes(const fathom_index &ix)
+{
+    return (size_t)ix.head_dim * kBits * (size_t)ix.n_words * sizeof(uint32_t);
+}
+
+struct HostLayout {
+    size_t unit_ws;      // scratch of one unit's scan (reused by every unit)
+    size_t slot_bytes;   // one ring slot
+    size_t total;
+};
+
+HostLayout host_layout(const fathom_index *sessions, int n, int k)
+{
+    HostLayout L{};
+    for (const HostUnit &u : host_units(sessions, n)) {
+        const fathom_index &ix = sessions[u.s];
+        const fathom_index v = unit_view(ix, u.h0, u.nh, nullptr);
+        L.unit_ws = std::max(L.unit_ws, layout_session(v, k, 0).total);
+        if (host_resident(ix)) L.slot_bytes = std::max(L.slot_bytes, u.nh * head_plane_bytes(ix));
+    }
+    L.unit_ws = align256(L.unit_ws);
+    L.slot_bytes = align256(L.slot_bytes);
+    L.total = L.unit_ws + 2 * L.slot_bytes;
+    return L;
+}
+
+// The side stream and events of the pipelined path, one set per (device,
+// caller stream), created on first use and kept for the process.
+struct SideContext {
+    cudaStream_t side;
+    cudaEvent_t fork, join, fetched[2], done[2];
+};
+
+cudaError_t side_context(cudaStream_t stream, SideContext **out)
+{
+    static std::mutex mu;
+    static std::map<std::pair<int, cudaStream_t>, SideContext> contexts;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = contexts.find({dev, stream});
+    if (it == contexts.end()) {
+        SideContext c{};
+        if ((e = cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        cudaEvent_t *evs[] = {&c.fork, &c.join, &c.fetched[0], &c.fetched[1], &c.done[0], &c.done[1]};
+        for (cudaEvent_t *ev : evs)
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        it = contexts.emplace(std::make_pair(dev, stream), c).first;
+    }
+    *out = &it->second;
+    return cudaSuccess;
+}
+
+cudaError_t run_host_pipelined(const ScanSessionArgs *ss, int n_sessions, int k, void *ws,
+                               uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
+{
+    std::vector<fathom_index> ix(n_sessions);
+    for (int s = 0; s < n_sessions; ++s) ix[s] = *ss[s].ix;
+    const HostLayout L = host_layout(ix.data(), n_sessions, k);
+    const std::vector<HostUnit> units = host_units(ix.data(), n_sessions);
+    char *base = static_cast<char *>(ws);
+    SideContext *c = nullptr;
+    cudaError_t e = side_context(stream, &c);
+    if (e != cudaSuccess) return note_error(e, "side stream set-up");
+    if ((e = cudaEventRecord(c->fork, stream)) != cudaSuccess) return note_error(e, "fork");
+    if ((e = cudaStreamWaitEvent(c->side, c->fork, 0)) != cudaSuccess) return note_error(e, "fork");
+    const bool timed = hook && hook->enabled;
+    if (timed) record_timing_event(hook->begin, c->side);
+    for (size_t u = 0; u < units.size(); ++u) {
+        const HostUnit &U = units[u];
+        const ScanSessionArgs &a = ss[U.s];
+        const fathom_index &x = ix[U.s];
+        const int d = x.head_dim, G = x.group;
+        const size_t row0 = (size_t)U.h0 * d * kBits * (size_t)x.n_words;
+        uint32_t *planes = x.planes + row0;
+        if (host_resident(x)) {
+            uint32_t *slot = reinterpret_cast<uint32_t *>(base + L.unit_ws + (u % 2) * L.slot_bytes);
+            if (u >= 2 && (e = cudaStreamWaitEvent(c->side, c->done[u % 2], 0)) != cudaSuccess)
+                return note_error(e, "ring wait");
+            const FetchJob job{planes, slot, a.t_union + (size_t)U.h0 * d, U.nh * d, x.n_words};
+            if ((e = launch_fetch(&job, 1, c->side, kFetchCtasPerSmShared)) != cudaSuccess)
+                return note_error(e, "fetch launch");
+            if ((e = cudaEventRecord(c->fetched[u % 2], c->side)) != cudaSuccess)
+                return note_error(e, "fetch event");
+            if ((e = cudaStreamWaitEvent(stream, c->fetched[u % 2], 0)) != cudaSuccess)
+                return note_error(e, "fetch wait");
+            planes = slot;
+        }
+        const fathom_index v = unit_view(x, U.h0, U.nh, planes);
+        const size_t qo = (size_t)U.h0 * G;
+        const ScanSessionArgs ua{&v, a.q + qo * d, a.t + qo * d, a.t_union + (size_t)U.h0 * d,
+                                 a.out_idx + qo * k, a.out_score + qo * k};
+        if ((e = build_and_run<1>(&ua, 1, k, ws, flags & ~FATHOM_SCAN_PROFILE, stream, nullptr)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaEventRecord(c->done[u % 2], stream)) != cudaSuccess) return note_error(e, "done event");
+    }
+    if (timed) {
+        record_timing_event(hook->end, c->side);
+        hook->recorded = true;
+    }
+    if ((e = cudaEventRecord(c->join, c->side)) != cudaSuccess) return note_error(e, "join");
+    if ((e = cudaStreamWaitEvent(stream, c->join, 0)) != cudaSuccess) return note_error(e, "join");
+    return cudaSuccess;
 }
 
 }  // namespace
 
 size_t scan_workspace_bytes(const fathom_index *sessions, int n_sessions, int k)
 {
+    if (any_host(sessions, n_sessions)) return host_layout(sessions, n_sessions, k).total;
     size_t at = 0;
     for (int s = 0; s < n_sessions; ++s) at = layout_session(sessions[s], k, at).total;
     return at;
@@ -1724,6 +1854,10 @@ cudaError_t launch_scan(const ScanSessionArgs *sessions, int n_sessions, int k, 
                         ScanProfileHook *hook)
 {
     (void)ws_bytes;
+    std::vector<fathom_index> ix(n_sessions);
+    for (int s = 0; s < n_sessions; ++s) ix[s] = *sessions[s].ix;
+    if (any_host(ix.data(), n_sessions))
+        return run_host_pipelined(sessions, n_sessions, k, ws, flags, stream, hook);
     if (n_sessions == 1) return build_and_run<1>(sessions, 1, k, ws, flags, stream, hook);
     return build_and_run<kMaxSessions>(sessions, n_sessions, k, ws, flags, stream, hook);
 }

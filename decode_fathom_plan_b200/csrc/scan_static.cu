@@ -21,8 +21,8 @@
 
 // 8 MiB: a device index of 64 query heads at 1,048,576 keys with k <= 2048
 // needs about 6.3 MiB (per-query state, candidate buffers, per-KV-head scan
-// tables).  A host-resident index also needs room for the device mirror of
-// its planes, so only small host-resident indices fit.
+// tables).  A host-resident index also needs room for the two-slot ring its
+// planes are fetched into, so only small host-resident indices fit.
 static constexpr size_t kStaticScratchBytes = 8u << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kStaticScratchBytes];
 

@@ -93,10 +93,16 @@ typedef enum {
 
 /* Where the planes live.  DEVICE: HBM.  HOST_MAPPED: pinned, device-mapped
  * host memory (the explainer's setting: the 4-bit K index is offloaded to
- * host memory).  A scan of a HOST_MAPPED index first fetches the planes its
- * union plan selects over the host link into a device mirror held in the
- * workspace (so its workspace includes H*d*4*n_words*4 bytes), then scores
- * from the mirror. */
+ * host memory).  A scan of a HOST_MAPPED index moves only the planes its
+ * union plan selects over the host link, one unit of KV heads at a time (one
+ * head for a single index, one index for a batched call), into a two-slot
+ * device ring held in the workspace: unit u + 1 is fetched on a side stream
+ * while unit u is scored from the other slot.  The workspace therefore holds
+ * two units' planes (2 * heads_per_unit * d*4*n_words*4 bytes) plus one
+ * unit's scan scratch, not the whole index.  The side stream and its events
+ * are created on the first such call for a (device, stream) pair and kept;
+ * they fork from and join the caller's stream within the call (event waits
+ * only), so a captured call stays a CUDA graph on the caller's stream. */
 typedef enum {
     FATHOM_RES_DEVICE = 0,
     FATHOM_RES_HOST_MAPPED = 1
@@ -282,7 +288,7 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
  *     FATHOM_ERR_WORKSPACE before anything is enqueued; use fathom_scan_topk
  *     for it.  For a device index, a layer of 64 query heads at 1,048,576
  *     keys with k <= 2048 needs 6.3 MiB; a host-resident index also needs
- *     room for its plane mirror, so only small ones fit.
+ *     room for its two-slot plane ring, so only small ones fit.
  *   - Every call looks up the scratch array's device address
  *     (cudaGetSymbolAddress) on the current device, so the address stays
  *     right after a device reset.  The first call on a device may also load

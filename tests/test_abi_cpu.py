@@ -63,14 +63,19 @@ def test_workspace_sizes_are_host_computable(lib):
         fp.fathom_scan_workspace_bytes(ix, 64) + fp.fathom_scan_workspace_bytes(big, 64)
 
 
-def test_host_resident_workspace_holds_a_plane_mirror(lib):
-    # a HOST_MAPPED index is fetched into a device mirror of its planes
-    # [H][d][4][n_words] uint32 held in the workspace
+def test_host_resident_workspace_holds_a_two_head_ring(lib):
+    # a HOST_MAPPED index is scanned one KV head at a time: the workspace holds
+    # the scratch of a one-head scan and a ring of two one-head plane slots
+    # [d][4][n_words] uint32, so it does not grow with the number of heads
     for H, d, n in ((2, 128, 4096), (8, 128, 1 << 20), (1, 64, 1000)):
-        dev = fp.fathom_scan_workspace_bytes(_desc(H=H, d=d, n=n, residency=0), 64)
+        one_head = fp.fathom_scan_workspace_bytes(_desc(H=1, d=d, n=n, residency=0), 64)
         host = fp.fathom_scan_workspace_bytes(_desc(H=H, d=d, n=n, residency=1), 64)
-        mirror = H * d * 4 * fp.fathom_n_words(n) * 4
-        assert host - dev == (mirror + 255) // 256 * 256
+        slot = d * 4 * fp.fathom_n_words(n) * 4
+        assert host == (one_head + 255) // 256 * 256 + 2 * ((slot + 255) // 256 * 256)
+    # the million-key layer: well under the size of the index it scans
+    index = 8 * 128 * 4 * fp.fathom_n_words(1 << 20) * 4
+    assert fp.fathom_scan_workspace_bytes(_desc(H=8, d=128, n=1 << 20, residency=1), 2048) \
+        < 0.3 * index
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 48), ("head_dim", 512), ("group", 9),
