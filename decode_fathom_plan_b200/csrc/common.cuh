@@ -27,7 +27,7 @@ constexpr int kStages = 3;
 
 // Sample-threshold sizing (see the scan launcher).
 constexpr int kSampleMinKeys = 4096;
-constexpr int kSampleMaxKeys = 32768;
+constexpr int kSampleMaxKeys = 8192;   // past this the rank is 3k*m/n (see the scan launcher)
 constexpr int kSampleTargetRank = 128;
 
 // Per-query state kept in the workspace: threshold, candidate count,

@@ -1,5 +1,8 @@
 """Shared helpers of the GPU parity tests: run the oracle on the same seeded
 inputs and compare with the CUDA path under the stated tolerances."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 import oracle
@@ -50,3 +53,16 @@ def check_topk(gpu_idx, gpu_score, s, a, k, rtol=SCORE_RTOL):
                                          f"oracle top-{k} outside the tie band (k-th {kth})")
     assert np.all(np.diff(gpu_idx) > 0), "indices not in ascending order"
     return len(diff) // 2
+
+
+def check_queries(ix, q_bf16, t, group, k, gpu_idx, gpu_score, queries, heads=None):
+    """check_topk for each query row in `queries` against oracle index `ix`,
+    the oracle runs on all host cores at once (its C calls release the GIL).
+    heads: KV head of each query in `ix` (default qq // group)."""
+    def one(i):
+        qq = queries[i]
+        h = qq // group if heads is None else heads[i]
+        _, _, s, a = oracle_query(ix, q_bf16[qq], t[qq], h, k)
+        return check_topk(gpu_idx[qq], gpu_score[qq], s, a, k)
+    with ThreadPoolExecutor(max_workers=min(len(queries), os.cpu_count() or 1)) as ex:
+        return list(ex.map(one, range(len(queries))))
