@@ -904,9 +904,6 @@ __device__ void bitonic_sort_desc(unsigned long long *x, int kpad)
     }
 }
 
-constexpr int kBitmapMaxKeys = 1 << 20;                     // index-order output via a bitmap
-constexpr int kChunkWords = 8;                              // bitmap words per prefix entry
-
 // Writes the k selected composites `sel` (okey << 32 | ~index, kpad slots,
 // kpad a power of two >= k) to the outputs in ascending key index by sorting
 // them on the index (bitonic network); for any number of keys.
@@ -924,52 +921,73 @@ __device__ void emit_sorted_by_index(unsigned long long *sel, int k, int kpad, i
     }
 }
 
-// Writes the k selected composites `sel` (okey << 32 | ~index) to the
-// outputs in ascending key index: a bitmap of the selected indices in
-// shared memory (n_keys <= kBitmapMaxKeys) and one prefix count per
-// kChunkWords bitmap words give each key its output position.  `bm` holds
-// ceil(n/32) words followed by the prefixes.
-__device__ void emit_in_index_order(const unsigned long long *sel, int k, int n, uint32_t *bm,
-                                    unsigned *wsum, int32_t *out_idx, float *out_score)
+// Writes the k <= kMaxFastK selected composites `sel` (okey << 32 | ~index)
+// to the outputs in ascending key index, for any number of keys n: the keys
+// are counted into at most kSelBins buckets of consecutive indices, the
+// buckets' exclusive prefix gives each bucket its output range, every key is
+// scattered into its bucket's range (`tmp`, k slots), and each key's place
+// inside its bucket is the number of keys there with a smaller index (the
+// buckets hold about one key each).  The cost follows k, not n.
+// Called by all kSelThreads threads; uses ss.hist and ss.wsum.
+constexpr int kEmitPerThread = kMaxFastK / kSelThreads;   // 4
+__device__ void emit_by_buckets(const unsigned long long *sel, int k, int n,
+                                unsigned long long *tmp, SelShared &ss, int32_t *out_idx,
+                                float *out_score)
 {
-    const int words = (n + 31) >> 5;
-    const int chunks = (words + kChunkWords - 1) / kChunkWords;
-    uint32_t *pre = bm + chunks * kChunkWords;
-    for (int w = threadIdx.x; w < chunks * kChunkWords; w += kSelThreads) bm[w] = 0u;
+    const int shift = max(0, bit_length((uint32_t)max(n - 1, 1)) - kSelBits);
+    unsigned *cnt = ss.hist;
+#pragma unroll
+    for (int i = 0; i < kSelBinsPerThread; ++i) cnt[threadIdx.x + i * kSelThreads] = 0u;
     __syncthreads();
-    for (int i = threadIdx.x; i < k; i += kSelThreads) {
-        const uint32_t j = ~(uint32_t)(sel[i] & 0xFFFFFFFFull);
-        atomicOr(&bm[j >> 5], 1u << (j & 31));
+    unsigned slot[kEmitPerThread];
+#pragma unroll
+    for (int e = 0; e < kEmitPerThread; ++e) {
+        const int i = threadIdx.x + e * kSelThreads;
+        if (i < k) {
+            const uint32_t j = ~(uint32_t)(sel[i] & 0xFFFFFFFFull);
+            slot[e] = atomicAdd(&cnt[j >> shift], 1u);
+        }
     }
     __syncthreads();
-    // prefix over chunks: each thread sums a contiguous run of chunks
-    const int per = (chunks + kSelThreads - 1) / kSelThreads;
-    const int c0 = threadIdx.x * per, c1 = min(chunks, c0 + per);
-    unsigned mine = 0;
-    for (int c = c0; c < c1; ++c) {
-        unsigned cc = 0;
+    // thread t owns bins 4t .. 4t+3: their exclusive prefix, in place
+    unsigned c4[kSelBinsPerThread], mine = 0;
 #pragma unroll
-        for (int w = 0; w < kChunkWords; ++w) cc += __popc(bm[c * kChunkWords + w]);
-        pre[c] = cc;
-        mine += cc;
+    for (int i = 0; i < kSelBinsPerThread; ++i) {
+        c4[i] = cnt[kSelBinsPerThread * threadIdx.x + i];
+        mine += c4[i];
     }
     unsigned total;
-    unsigned run = block_exclusive_scan(mine, wsum, &total);
-    for (int c = c0; c < c1; ++c) {
-        const unsigned cc = pre[c];
-        pre[c] = run;
-        run += cc;
+    unsigned run = block_exclusive_scan(mine, ss.wsum, &total);
+#pragma unroll
+    for (int i = 0; i < kSelBinsPerThread; ++i) {
+        cnt[kSelBinsPerThread * threadIdx.x + i] = run;
+        run += c4[i];
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < k; i += kSelThreads) {
-        const unsigned long long v = sel[i];
-        const uint32_t j = ~(uint32_t)(v & 0xFFFFFFFFull);
-        const int wj = (int)(j >> 5), c = wj / kChunkWords;
-        unsigned pos = pre[c];
-        for (int w = c * kChunkWords; w < wj; ++w) pos += __popc(bm[w]);
-        pos += __popc(bm[wj] & ((1u << (j & 31)) - 1u));
-        out_idx[pos] = (int32_t)j;
-        out_score[pos] = order_key_to_float((uint32_t)(v >> 32));
+#pragma unroll
+    for (int e = 0; e < kEmitPerThread; ++e) {
+        const int i = threadIdx.x + e * kSelThreads;
+        if (i < k) {
+            const uint32_t j = ~(uint32_t)(sel[i] & 0xFFFFFFFFull);
+            tmp[cnt[j >> shift] + slot[e]] = sel[i];
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kEmitPerThread; ++e) {
+        const int i = threadIdx.x + e * kSelThreads;
+        if (i < k) {
+            const unsigned long long v = sel[i];
+            const uint32_t j = ~(uint32_t)(v & 0xFFFFFFFFull);
+            const unsigned bk = j >> shift;
+            const unsigned lo = cnt[bk];
+            const unsigned hi = (bk + 1 < (unsigned)kSelBins) ? cnt[bk + 1] : (unsigned)k;
+            unsigned pos = lo;
+            for (unsigned x = lo; x < hi; ++x)
+                pos += (~(uint32_t)(tmp[x] & 0xFFFFFFFFull) < j) ? 1u : 0u;
+            out_idx[pos] = (int32_t)j;
+            out_score[pos] = order_key_to_float((uint32_t)(v >> 32));
+        }
     }
 }
 
@@ -1189,7 +1207,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
 // ---------------------------------------------------------------- final
 // One CTA per query: exact top-k of the candidates when k <= count <= cap,
 // written in ascending key index.  Shared memory: the selected k (kMaxFastK
-// composites), then the candidates, later reused for the index bitmap.
+// composites), then the candidates, later reused to put the k in index order.
 template <int NS>
 __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constant__ Batch<NS> b)
 {
@@ -1209,7 +1227,7 @@ __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constan
         return;
     }
     unsigned long long *sel = dyn;                  // [kMaxFastK]
-    unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the bitmap
+    unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the emit scratch
     const unsigned long long *cq = S.cand + (size_t)qq * b.cap;
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
     for (unsigned i = 2 * threadIdx.x; i < cnt; i += 2 * kSelThreads) {
@@ -1249,12 +1267,7 @@ __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constan
         }
     }
     __syncthreads();
-    if (S.n <= kBitmapMaxKeys)
-        emit_in_index_order(sel, k, S.n, reinterpret_cast<uint32_t *>(x), ss.wsum,
-                            S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
-    else   // the bitmap of so many keys would not fit in shared memory
-        emit_sorted_by_index(sel, k, b.kpad, S.out_idx + (size_t)qq * k,
-                             S.out_score + (size_t)qq * k);
+    emit_by_buckets(sel, k, S.n, x, ss, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
 }
 
 // ------------------------------------------------------------- fallback
@@ -1497,25 +1510,6 @@ inline void record_timing_event(cudaEvent_t ev, cudaStream_t stream)
         cudaEventRecord(ev, stream);
 }
 
-// Shared-memory bytes of the index-order bitmap and its chunk prefixes.
-inline size_t bitmap_bytes_for(int n)
-{
-    const size_t words = ((size_t)n + 31) / 32;
-    const size_t chunks = (words + kChunkWords - 1) / kChunkWords;
-    return (chunks * kChunkWords + chunks) * sizeof(uint32_t);
-}
-
-template <int NS>
-size_t final_bitmap_bytes(const Batch<NS> &bt)
-{
-    // sessions past kBitmapMaxKeys keys, and those on the exact path, need no bitmap
-    size_t m = 0;
-    for (int s = 0; s < bt.n_sessions; ++s)
-        if (!bt.s[s].exact_only && bt.s[s].n <= kBitmapMaxKeys)
-            m = std::max(m, bitmap_bytes_for(bt.s[s].n));
-    return m;
-}
-
 template <int NS, int GP, bool kBlocked>
 cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, int total_heads,
                       int total_blocks, int max_m_keys, uint32_t flags, cudaStream_t stream,
@@ -1563,13 +1557,10 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
         }
         ++launches;
     }
-    const size_t bitmap_bytes = final_bitmap_bytes(bt);
-    const size_t final_smem = kMaxFastK * sizeof(unsigned long long) +
-                              std::max((size_t)bt.cap * sizeof(unsigned long long), bitmap_bytes);
+    const size_t final_smem = (kMaxFastK + (size_t)bt.cap) * sizeof(unsigned long long);
     if ((e = ensure_smem(SmemFlags<NS>::final_, final_kernel<NS>,
-                         kMaxFastK * sizeof(unsigned long long) +
-                             std::max((size_t)capacity_for(kMaxFastK) * sizeof(unsigned long long),
-                                      bitmap_bytes_for(kBitmapMaxKeys)))) != cudaSuccess)
+                         (kMaxFastK + (size_t)capacity_for(kMaxFastK)) *
+                             sizeof(unsigned long long))) != cudaSuccess)
         return note_error(e, "final set-up");
     final_kernel<NS><<<total_queries, kSelThreads, final_smem, stream>>>(bt);
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "final launch");
