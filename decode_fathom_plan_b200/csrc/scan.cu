@@ -37,19 +37,18 @@
 // No tensor cores: this is a sparse binary-weighted reduction.
 //
 // Selection without materialising n scores per query:
-//   1. threshold: per query, score evenly strided whole tiles (about 3% of
-//                 the keys) from the query's own plan, and take theta = the
-//                 r-th largest sampled key, r about 2*k*m/n, so ~2k keys are
-//                 expected to pass;
+//   1. threshold: per query, score evenly strided whole tiles (4096 to 8192
+//                 keys) from the query's own plan, and take theta = the r-th
+//                 largest sampled key, r about 2*k*m/n (3*k*m/n for large n),
+//                 so ~2k (3k) keys are expected to pass;
 //   2. filter:    the full scan appends (key, index) of every key scoring
 //                 >= theta to a per-query candidate buffer;
 //   3. final:     if k <= candidates <= capacity, an exact radix select over
 //                 the unique composite (order key, ~index) gives the top-k,
-//                 listed in ascending key index; otherwise the query is
-//                 flagged;
-//   4. fallback:  a flagged query is redone exactly by one CTA that
-//                 recomputes its scores once per radix digit (no score
-//                 buffer), so results never depend on the sample.
+//                 listed in ascending key index; otherwise the same CTA
+//                 redoes the query exactly, recomputing its scores once per
+//                 radix digit (no score buffer), so results never depend on
+//                 the sample.
 // Correctness needs only that every key scoring at least the k-th largest
 // score is a candidate, which "count >= k" guarantees for any theta.
 #include <math.h>
@@ -74,8 +73,8 @@ constexpr int kMaskOrderValues = 16;   // reader sets of up to 4 query heads
 constexpr int kMinChunkGroups = 8;     // smallest chunk of the main scan: 32 words
 // Sampled tiles of a session with grouped per-token-block scales (Qwen3-8B
 // layer, 128K keys in 2048-key blocks: 2 tiles sent some queries to the
-// exact fallback, 4 kept all on the fast path, 8 and 16 cost more threshold
-// passes than the fallbacks they saved).
+// exact path, 4 kept all on the fast path, 8 and 16 cost more threshold
+// passes than the exact paths they saved).
 constexpr int kBlockedSampleTiles = 4;
 
 struct SessionDesc {
@@ -87,7 +86,7 @@ struct SessionDesc {
     const uint8_t *tu;           // [H][d]
     int32_t *out_idx;            // [Q][k]
     float *out_score;            // [Q][k]
-    uint32_t *qstate;            // [Q][4]: theta, count, fallback flag, spare
+    uint32_t *qstate;            // [Q][4]: theta, count, exact-path flag, spare
     unsigned long long *cand;    // [Q][cap]
     unsigned char *tables;       // [H] per-head scan tables (ScanMeta of the batch's GP)
     float *bias_blk;             // grouped scales: [H][nb][G] bias per (head, block, query)
@@ -381,6 +380,7 @@ __device__ __forceinline__ void load_stage(const ScanMeta<GP> &sm, StageBuf stag
                                            int buf, const uint32_t *planes, int n_words,
                                            int col_lo, int col_hi)
 {
+    if (threadIdx.x >= kScanThreads) return;   // a larger CTA's extra threads copy nothing
     const int chunk = threadIdx.x & 15;
     const int col = col_lo + chunk * 4;
     const bool ok = col < col_hi;
@@ -1204,78 +1204,16 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     }
 }
 
-// ---------------------------------------------------------------- final
-// One CTA per query: exact top-k of the candidates when k <= count <= cap,
-// written in ascending key index.  Shared memory: the selected k (kMaxFastK
-// composites), then the candidates, later reused to put the k in index order.
-template <int NS>
-__global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constant__ Batch<NS> b)
-{
-    extern __shared__ unsigned long long dyn[];
-    __shared__ SelShared ss;
-    const int gq = blockIdx.x;
-    const int si = find_session_by_query(b, gq);
-    const SessionDesc &S = b.s[si];
-    const int qq = gq - S.q_begin;
-    uint32_t *st = S.qstate + qq * kQueryStateWords;
-    if (st[2]) return;
-    const unsigned cnt = st[1];
-    const int k = b.k;
-    if (cnt < (unsigned)k || cnt > (unsigned)b.cap) {
-        __syncthreads();
-        if (threadIdx.x == 0) st[2] = 1;
-        return;
-    }
-    unsigned long long *sel = dyn;                  // [kMaxFastK]
-    unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the emit scratch
-    const unsigned long long *cq = S.cand + (size_t)qq * b.cap;
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (unsigned i = 2 * threadIdx.x; i < cnt; i += 2 * kSelThreads) {
-        unsigned long long v0, v1 = 0ull;
-        if (i + 1 < cnt) {
-            const ulonglong2 p = *reinterpret_cast<const ulonglong2 *>(cq + i);
-            v0 = p.x;
-            v1 = p.y;
-            x[i + 1] = v1;
-            lo = min(lo, (uint32_t)(v1 >> 32));
-            hi = max(hi, (uint32_t)(v1 >> 32));
-        } else {
-            v0 = cq[i];
-        }
-        x[i] = v0;
-        lo = min(lo, (uint32_t)(v0 >> 32));
-        hi = max(hi, (uint32_t)(v0 >> 32));
-    }
-    sel_range(ss, lo, hi);
-    const unsigned long long base = (unsigned long long)ss.lo << 32;
-    const int top = 32 + bit_length(ss.hi - ss.lo);
-    sel_run(ss, cnt, (unsigned)k, top, 0, [&](unsigned i) { return x[i] - base; });
-    // compact exactly the k selected, in candidate order (block scan)
-    const int cut = ss.cut;
-    const unsigned long long lim = ss.prefix >> cut;
-    const unsigned per = (cnt + kSelThreads - 1) / kSelThreads;
-    const unsigned i0 = threadIdx.x * per, i1 = min(cnt, i0 + per);
-    unsigned mine = 0;
-    for (unsigned i = i0; i < i1; ++i) mine += ((x[i] - base) >> cut) >= lim;
-    unsigned total;
-    unsigned pos = block_exclusive_scan(mine, ss.wsum, &total);
-    for (unsigned i = i0; i < i1; ++i) {
-        const unsigned long long v = x[i];
-        if (((v - base) >> cut) >= lim) {
-            if (pos < (unsigned)k) sel[pos] = v;
-            ++pos;
-        }
-    }
-    __syncthreads();
-    emit_by_buckets(sel, k, S.n, x, ss, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
-}
-
-// ------------------------------------------------------------- fallback
-// One CTA per flagged query: exact top-k by radix select over the composite
-// (order key, ~index), recomputing the query's scores from its own plan on
-// every pass.  Slow, rare, and independent of the sample.
+// ------------------------------------------------------------- exact path
+// The exact top-k of query qq of session S by radix select over the
+// composite (order key, ~index), recomputing the query's scores from its own
+// plan on every pass: slow, rare (a query the sampled threshold did not suit,
+// or a forced or k > kMaxFastK scan), and independent of the sample.  Run by
+// the query's final CTA; threads past kScanThreads only take part in the
+// barriers (the scan stages cover kScanThreads threads).  Uses the dynamic
+// shared memory for its stages and the k selected.
 template <int NS, bool kBlocked>
-__global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_constant__ Batch<NS> b)
+__device__ void exact_query(const Batch<NS> &b, const SessionDesc &S, int qq)
 {
     __shared__ ScanMeta<1> sm;
     __shared__ SelectState ss;
@@ -1284,11 +1222,6 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
     StageBuf stage = reinterpret_cast<StageBuf>(fb_dyn);
     unsigned long long *sel =
         reinterpret_cast<unsigned long long *>(fb_dyn + kMainStages * kStageRows * kTileCols);
-    const int gq = blockIdx.x;
-    const int si = find_session_by_query(b, gq);
-    const SessionDesc &S = b.s[si];
-    const int qq = gq - S.q_begin;
-    if (!S.qstate[qq * kQueryStateWords + 2]) return;
     const int d = b.d, k = b.k;
     const int h = qq / b.G;
     const uint8_t *trow = S.t + (size_t)qq * d;
@@ -1369,6 +1302,70 @@ __global__ void __launch_bounds__(kScanThreads) fallback_kernel(const __grid_con
     emit_sorted_by_index(sel, k, b.kpad, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
 }
 
+// ---------------------------------------------------------------- final
+// One CTA per query: exact top-k of the candidates when k <= count <= cap,
+// written in ascending key index.  Shared memory: the selected k (kMaxFastK
+// composites), then the candidates, later reused to put the k in index order.
+template <int NS, bool kBlocked>
+__global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constant__ Batch<NS> b)
+{
+    extern __shared__ unsigned long long dyn[];
+    __shared__ SelShared ss;
+    const int gq = blockIdx.x;
+    const int si = find_session_by_query(b, gq);
+    const SessionDesc &S = b.s[si];
+    const int qq = gq - S.q_begin;
+    const uint32_t *st = S.qstate + qq * kQueryStateWords;
+    const unsigned cnt = st[1];
+    const int k = b.k;
+    if (st[2] || cnt < (unsigned)k || cnt > (unsigned)b.cap) {
+        exact_query<NS, kBlocked>(b, S, qq);   // the exact path, in this CTA
+        return;
+    }
+    unsigned long long *sel = dyn;                  // [kMaxFastK]
+    unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the emit scratch
+    const unsigned long long *cq = S.cand + (size_t)qq * b.cap;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (unsigned i = 2 * threadIdx.x; i < cnt; i += 2 * kSelThreads) {
+        unsigned long long v0, v1 = 0ull;
+        if (i + 1 < cnt) {
+            const ulonglong2 p = *reinterpret_cast<const ulonglong2 *>(cq + i);
+            v0 = p.x;
+            v1 = p.y;
+            x[i + 1] = v1;
+            lo = min(lo, (uint32_t)(v1 >> 32));
+            hi = max(hi, (uint32_t)(v1 >> 32));
+        } else {
+            v0 = cq[i];
+        }
+        x[i] = v0;
+        lo = min(lo, (uint32_t)(v0 >> 32));
+        hi = max(hi, (uint32_t)(v0 >> 32));
+    }
+    sel_range(ss, lo, hi);
+    const unsigned long long base = (unsigned long long)ss.lo << 32;
+    const int top = 32 + bit_length(ss.hi - ss.lo);
+    sel_run(ss, cnt, (unsigned)k, top, 0, [&](unsigned i) { return x[i] - base; });
+    // compact exactly the k selected, in candidate order (block scan)
+    const int cut = ss.cut;
+    const unsigned long long lim = ss.prefix >> cut;
+    const unsigned per = (cnt + kSelThreads - 1) / kSelThreads;
+    const unsigned i0 = threadIdx.x * per, i1 = min(cnt, i0 + per);
+    unsigned mine = 0;
+    for (unsigned i = i0; i < i1; ++i) mine += ((x[i] - base) >> cut) >= lim;
+    unsigned total;
+    unsigned pos = block_exclusive_scan(mine, ss.wsum, &total);
+    for (unsigned i = i0; i < i1; ++i) {
+        const unsigned long long v = x[i];
+        if (((v - base) >> cut) >= lim) {
+            if (pos < (unsigned)k) sel[pos] = v;
+            ++pos;
+        }
+    }
+    __syncthreads();
+    emit_by_buckets(sel, k, S.n, x, ss, S.out_idx + (size_t)qq * k, S.out_score + (size_t)qq * k);
+}
+
 // ------------------------------------------------------------- host side
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1391,7 +1388,7 @@ struct Sizing {
 // when f = 2 would give r < 128), so about f*k keys pass the filter.  The
 // count of passing keys has a relative spread of about 1/sqrt(r): at one
 // million keys and k = 2048, m = 8192 gives r = 48 at f = 3, so falling
-// below k (the exact fallback) is a 4.6-sigma event and passing the
+// below k (the exact path) is a 4.6-sigma event and passing the
 // capacity of 6k a 7-sigma one, while the sampled pass reads a quarter of
 // what 32768 keys cost (B200: 50 -> 17 us per plan on that layer).
 Sizing size_session(int n, int n_words, int k, int block_keys)
@@ -1407,7 +1404,7 @@ Sizing size_session(int n, int n_words, int k, int block_keys)
     int mt = ceil_div(m, kTileKeys);
     // Grouped scales shift every block's scores by its own unread-channel
     // constant, so a sample of few blocks misplaces theta and sends queries
-    // to the exact fallback; at least kBlockedSampleTiles tiles (from as many
+    // to the exact path; at least kBlockedSampleTiles tiles (from as many
     // blocks) keep it on the fast path.
     if (block_keys) mt = std::max(mt, kBlockedSampleTiles);
     mt = std::min(mt, std::max(1, z.n_tiles / 4));
@@ -1557,23 +1554,22 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
         }
         ++launches;
     }
-    const size_t final_smem = (kMaxFastK + (size_t)bt.cap) * sizeof(unsigned long long);
-    if ((e = ensure_smem(SmemFlags<NS>::final_, final_kernel<NS>,
-                         (kMaxFastK + (size_t)capacity_for(kMaxFastK)) *
-                             sizeof(unsigned long long))) != cudaSuccess)
+    // the fast path's selected k and candidates, or the exact path's stages
+    // and its k selected, whichever is larger
+    const size_t exact_smem = kMainStages * kStageBytes + (size_t)bt.kpad * sizeof(unsigned long long);
+    const size_t final_smem =
+        std::max((kMaxFastK + (size_t)bt.cap) * sizeof(unsigned long long), exact_smem);
+    static int final_smem_set[64];
+    if ((e = ensure_smem(final_smem_set, final_kernel<NS, kBlocked>,
+                         std::max((kMaxFastK + (size_t)capacity_for(kMaxFastK)) *
+                                      sizeof(unsigned long long),
+                                  kMainStages * kStageBytes +
+                                      (size_t)kMaxK * sizeof(unsigned long long)))) != cudaSuccess)
         return note_error(e, "final set-up");
-    final_kernel<NS><<<total_queries, kSelThreads, final_smem, stream>>>(bt);
-    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "final launch");
-    const size_t fb_smem = kMainStages * kStageBytes + (size_t)bt.kpad * sizeof(unsigned long long);
-    static int fallback_smem_set[64];
-    if ((e = ensure_smem(fallback_smem_set, fallback_kernel<NS, kBlocked>,
-                         kMainStages * kStageBytes + (size_t)kMaxK * sizeof(unsigned long long))) !=
-        cudaSuccess)
-        return note_error(e, "fallback set-up");
-    fallback_kernel<NS, kBlocked><<<total_queries, kScanThreads, fb_smem, stream>>>(bt);
-    launches += 2;
+    final_kernel<NS, kBlocked><<<total_queries, kSelThreads, final_smem, stream>>>(bt);
+    launches += 1;
     note_launch(launches);
-    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "fallback launch");
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "final launch");
     return cudaSuccess;
 }
 
