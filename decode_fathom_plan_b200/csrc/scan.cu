@@ -1778,19 +1778,15 @@ cudaError_t side_context(cudaStream_t stream, SideContext **out)
     return cudaSuccess;
 }
 
-cudaError_t run_host_pipelined(const ScanSessionArgs *ss, int n_sessions, int k, void *ws,
-                               uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
+// The units of a pipelined scan, enqueued after the fork; the first error
+// stops the enqueueing (the caller joins the side stream either way).
+cudaError_t enqueue_units(const ScanSessionArgs *ss, const std::vector<fathom_index> &ix,
+                          const std::vector<HostUnit> &units, const HostLayout &L, int k,
+                          void *ws, uint32_t flags, cudaStream_t stream, SideContext *c,
+                          ScanProfileHook *hook)
 {
-    std::vector<fathom_index> ix(n_sessions);
-    for (int s = 0; s < n_sessions; ++s) ix[s] = *ss[s].ix;
-    const HostLayout L = host_layout(ix.data(), n_sessions, k);
-    const std::vector<HostUnit> units = host_units(ix.data(), n_sessions);
     char *base = static_cast<char *>(ws);
-    SideContext *c = nullptr;
-    cudaError_t e = side_context(stream, &c);
-    if (e != cudaSuccess) return note_error(e, "side stream set-up");
-    if ((e = cudaEventRecord(c->fork, stream)) != cudaSuccess) return note_error(e, "fork");
-    if ((e = cudaStreamWaitEvent(c->side, c->fork, 0)) != cudaSuccess) return note_error(e, "fork");
+    cudaError_t e;
     const bool timed = hook && hook->enabled;
     if (timed) record_timing_event(hook->begin, c->side);
     for (size_t u = 0; u < units.size(); ++u) {
@@ -1820,15 +1816,35 @@ cudaError_t run_host_pipelined(const ScanSessionArgs *ss, int n_sessions, int k,
         if ((e = build_and_run<1>(&ua, 1, k, ws, flags & ~FATHOM_SCAN_PROFILE, stream, nullptr)) !=
             cudaSuccess)
             return e;
-        if ((e = cudaEventRecord(c->done[u % 2], stream)) != cudaSuccess) return note_error(e, "done event");
+        if ((e = cudaEventRecord(c->done[u % 2], stream)) != cudaSuccess)
+            return note_error(e, "done event");
     }
     if (timed) {
         record_timing_event(hook->end, c->side);
         hook->recorded = true;
     }
-    if ((e = cudaEventRecord(c->join, c->side)) != cudaSuccess) return note_error(e, "join");
-    if ((e = cudaStreamWaitEvent(stream, c->join, 0)) != cudaSuccess) return note_error(e, "join");
     return cudaSuccess;
+}
+
+cudaError_t run_host_pipelined(const ScanSessionArgs *ss, int n_sessions, int k, void *ws,
+                               uint32_t flags, cudaStream_t stream, ScanProfileHook *hook)
+{
+    std::vector<fathom_index> ix(n_sessions);
+    for (int s = 0; s < n_sessions; ++s) ix[s] = *ss[s].ix;
+    const HostLayout L = host_layout(ix.data(), n_sessions, k);
+    const std::vector<HostUnit> units = host_units(ix.data(), n_sessions);
+    SideContext *c = nullptr;
+    cudaError_t e = side_context(stream, &c);
+    if (e != cudaSuccess) return note_error(e, "side stream set-up");
+    if ((e = cudaEventRecord(c->fork, stream)) != cudaSuccess) return note_error(e, "fork");
+    if ((e = cudaStreamWaitEvent(c->side, c->fork, 0)) != cudaSuccess) return note_error(e, "fork");
+    e = enqueue_units(ss, ix, units, L, k, ws, flags, stream, c, hook);
+    // join whatever was enqueued on the side stream, also after an error, so
+    // the caller's stream (and a capture in progress) waits for all of it
+    cudaError_t j = cudaEventRecord(c->join, c->side);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(stream, c->join, 0);
+    if (j != cudaSuccess) note_error(j, "join");
+    return e != cudaSuccess ? e : j;
 }
 
 }  // namespace

@@ -251,6 +251,43 @@ def test_scan_batched_sessions():
         check_scan(ses, ref, t, oi.cpu().numpy(), os_.cpu().numpy(), k)
 
 
+def test_host_mapped_scan_replays_as_a_cuda_graph():
+    """A host-resident scan fetches its heads on a side stream forked from the
+    caller's stream and joined back: captured (global capture mode, on a
+    stream of its own) as one CUDA graph and replayed twice, it gives the
+    eager call's result bit for bit, and the oracle's."""
+    ses = synth.make_session(61, 3, 4, 40000, [18, 68, 92, 136] * 3)
+    ix = gpu_index(ses, "host_mapped")
+    q, t, tu, _ = run_plan(ix, ses, ses.budgets)
+    k = 512
+    eager_i, eager_s = run_scan(ix, ses, q, t, tu, k)
+    check_scan(ses, oracle.build_index(ses.keys), t, eager_i, eager_s, k)
+    Q = 12
+    out_i = torch.full((Q, k), -1, dtype=torch.int32, device="cuda")
+    out_s = torch.zeros((Q, k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(fp.fathom_scan_workspace_bytes(ix.desc, k), dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    # first call on this stream outside the capture (creates its side stream)
+    with torch.cuda.stream(side):
+        fp.fathom_scan_topk(ix.desc, q, t, tu, k, out_i, out_s, ws)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fp.fathom_scan_topk(ix.desc, q, t, tu, k, out_i, out_s, ws)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        out_i.fill_(-1)
+        out_s.fill_(0.0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert fp.fathom_last_device_status() == fp.FATHOM_OK
+        assert np.array_equal(out_i.cpu().numpy(), eager_i)
+        assert np.array_equal(out_s.cpu().numpy().view(np.uint32), eager_s.view(np.uint32))
+    del g
+
+
 def test_scan_rejects_small_workspace():
     ses = synth.make_session(5, 1, 1, 1000, 16)
     ix = gpu_index(ses)
