@@ -133,7 +133,7 @@ struct ScanSessionArgs {
 size_t scan_workspace_bytes(const fathom_index *sessions, int n_sessions, int k);
 
 // Profiling events around the dominant kernel of a scan call
-// (FATHOM_SCAN_PROFILE): the fetch when any index is host-resident, else
+// (FATHOM_SCAN_PROFILE): the fetch sequence when any index is host-resident, else
 // the main scan.
 struct ScanProfileHook {
     bool enabled;

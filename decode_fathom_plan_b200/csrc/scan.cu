@@ -1001,8 +1001,11 @@ __device__ void emit_by_buckets(const unsigned long long *sel, int k, int n,
 // head's scan tables for the filtering pass.  Stages of 8 own
 // channels x 2 tiles are copied with cp.async, three in flight; every query of
 // a KV head reads its sampled rows itself (a few tens of KB, mostly L2 hits).
-constexpr int kThetaTilesPerPass = kSelThreads / kScanThreads;            // 2
-constexpr int kThetaCols = kThetaTilesPerPass * kTileCols;                // 128 words
+// A pass scores 2 tiles (one per thread) or, with more than 2 sampled tiles,
+// 4 (two per thread), so a sample of up to 4 tiles takes one pass.
+constexpr int kThetaThreadTiles = kSelThreads / kScanThreads;             // 2
+constexpr int kThetaTilesPerPass = 2 * kThetaThreadTiles;                 // 4
+constexpr int kThetaCols = kThetaTilesPerPass * kTileCols;                // 256 words
 typedef uint32_t (*ThetaBuf)[kStageRows][kThetaCols];
 constexpr size_t kThetaStageBytes = (size_t)kStageRows * kThetaCols * sizeof(uint32_t);
 constexpr int kThetaResolutionBits = 2 * kSelBits;
@@ -1021,7 +1024,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     __shared__ float own_w[kMaxHeadDim];      // ... and weights q*scale (q with grouped scales)
     __shared__ double bias_part[kSelThreads / 32];
     __shared__ float bias_s;
-    // grouped scales: the weights and bias of the pass's two tiles' blocks
+    // grouped scales: the weights and bias of the pass's tiles' blocks
     __shared__ float tile_w[kBlocked ? kThetaTilesPerPass : 1][kBlocked ? kMaxHeadDim : 1];
     __shared__ float tile_bias[kThetaTilesPerPass];
     ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
@@ -1091,7 +1094,10 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     }
     const int n_own = (int)ss.krem;
     const int n_stages = (n_own + kStageChannels - 1) / kStageChannels;
-    const int sub = threadIdx.x / kScanThreads;             // tile of the pass
+    // tiles per pass, and per thread (tiles sub and sub + kThetaThreadTiles)
+    const int pass_tiles = S.m_tiles > kThetaThreadTiles ? kThetaTilesPerPass : kThetaThreadTiles;
+    const int thread_tiles = pass_tiles / kThetaThreadTiles;
+    const int sub = threadIdx.x / kScanThreads;             // first tile of the pass
     const int lt = threadIdx.x - sub * kScanThreads;
     const int col = lt >> 2, r = lt & 3;
     uint32_t sh[4];
@@ -1103,10 +1109,11 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     const size_t head_row0 = (size_t)h * d * kBits;
     // copy stage s of tile pass t0 into buffer bufi: plane rows of own
     // channels 8s..8s+7 (4 slots each, zeros past the channel's depth),
-    // 2 tiles x 16 column groups per row
+    // pass_tiles tiles x 16 column groups per row
     auto load = [&](int t0, int s, int bufi) {
-        for (int e = threadIdx.x; e < kStageRows * (kThetaCols / 4); e += kSelThreads) {
-            const int row = e / (kThetaCols / 4), part = e - row * (kThetaCols / 4);
+        const int groups = pass_tiles * (kTileCols / 4);
+        for (int e = threadIdx.x; e < kStageRows * groups; e += kSelThreads) {
+            const int row = e / groups, part = e - row * groups;
             const int tsub = part / (kTileCols / 4), c16 = part - tsub * (kTileCols / 4);
             const int tile = t0 + tsub;
             const int j = s * kStageChannels + row / kBits, slot = row % kBits;
@@ -1119,14 +1126,16 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
         }
         cp_async_commit();
     };
-    for (int t0 = 0; t0 < S.m_tiles; t0 += kThetaTilesPerPass) {
-        float2 acc[4];
+    for (int t0 = 0; t0 < S.m_tiles; t0 += pass_tiles) {
+        float2 acc[2][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[k2][i] = make_float2(0.0f, 0.0f);
         __syncthreads();   // the buffers are free
         if constexpr (kBlocked) {
             // each sampled tile lies in one scale block (blocks hold whole tiles)
-            for (int e = threadIdx.x; e < kThetaTilesPerPass * kMaxHeadDim; e += kSelThreads) {
+            for (int e = threadIdx.x; e < pass_tiles * kMaxHeadDim; e += kSelThreads) {
                 const int tsub = e / kMaxHeadDim, j = e - tsub * kMaxHeadDim;
                 const int tile = t0 + tsub;
                 const int wcol = tile * S.sample_stride * kTileCols;
@@ -1136,7 +1145,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
                         own_w[j], S.scale[((size_t)h * S.nb + blk) * d + own_c[j]]);
                 }
             }
-            if (threadIdx.x < kThetaTilesPerPass) {
+            if (threadIdx.x < pass_tiles) {
                 const int tile = t0 + threadIdx.x;
                 const int wcol = tile * S.sample_stride * kTileCols;
                 tile_bias[threadIdx.x] =
@@ -1161,27 +1170,38 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
             const uint32_t(*rows)[kThetaCols] = stage[s2 % kThetaBufs];
             const int j1 = min(n_own, (s2 + 1) * kStageChannels);
             for (int j = s2 * kStageChannels; j < j1; ++j) {
-                const uint32_t nib =
-                    gather_nibbles<kThetaCols>(rows + kBits * (j - s2 * kStageChannels),
-                                               sub * kTileCols + col, sh);
-                float2 v[4];
-                nibbles_to_floats(nib, neg, v);   // rows past the depth are zero
-                const float wj = kBlocked ? tile_w[kBlocked ? sub : 0][kBlocked ? j : 0] : own_w[j];
-                const float2 w2 = make_float2(wj, wj);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[i] = __ffma2_rn(v[i], w2, acc[i]);
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    if (k2 < thread_tiles) {
+                        const int tsub = sub + k2 * kThetaThreadTiles;
+                        const uint32_t nib =
+                            gather_nibbles<kThetaCols>(rows + kBits * (j - s2 * kStageChannels),
+                                                       tsub * kTileCols + col, sh);
+                        float2 v[4];
+                        nibbles_to_floats(nib, neg, v);   // rows past the depth are zero
+                        const float wj =
+                            kBlocked ? tile_w[kBlocked ? tsub : 0][kBlocked ? j : 0] : own_w[j];
+                        const float2 w2 = make_float2(wj, wj);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[k2][i] = __ffma2_rn(v[i], w2, acc[k2][i]);
+                    }
+                }
             }
             __syncthreads();   // buffer s2 % kThetaBufs is reloaded kThetaBufs stages on
         }
-        const int tile = t0 + sub;
-        if (tile < S.m_tiles) {
-            const int wcol = tile * S.sample_stride * kTileCols + col;
-            const float tb = kBlocked ? tile_bias[sub] : bias;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int j = wcol * 32 + r + 4 * m;
-                vals[tile * kTileKeys + col * 32 + r + 4 * m] =
-                    (wcol < S.n_cols && j < S.n) ? order_key(score_of(acc, m, tb)) : 0u;
+        for (int k2 = 0; k2 < 2; ++k2) {
+            const int tsub = sub + k2 * kThetaThreadTiles;
+            const int tile = t0 + tsub;
+            if (k2 < thread_tiles && tile < S.m_tiles) {
+                const int wcol = tile * S.sample_stride * kTileCols + col;
+                const float tb = kBlocked ? tile_bias[tsub] : bias;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int j = wcol * 32 + r + 4 * m;
+                    vals[tile * kTileKeys + col * 32 + r + 4 * m] =
+                        (wcol < S.n_cols && j < S.n) ? order_key(score_of(acc[k2], m, tb)) : 0u;
+                }
             }
         }
     }

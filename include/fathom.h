@@ -136,9 +136,10 @@ typedef struct {
 /* Skip the sampled candidate threshold and select every query's top-k with
  * the exact multi-pass radix select (the path the fast path falls back to). */
 #define FATHOM_SCAN_FORCE_EXACT 1u
-/* Record CUDA events around the dominant kernel of the call (benchmarking
- * only): the fetch of host-resident planes when the index is HOST_MAPPED,
- * else the main scan kernel. */
+/* Record CUDA events around the dominant work of the call (benchmarking
+ * only): for a HOST_MAPPED index the fetch sequence (from the first KV head's
+ * fetch to the end of the last one's, on the side stream), else the main
+ * scan kernel. */
 #define FATHOM_SCAN_PROFILE 2u
 
 /* Words per plane for n keys: n rounded up to 128 keys, i.e. 16-byte rows. */
@@ -381,8 +382,8 @@ fathom_status fathom_last_device_status(cudaStream_t stream);
 /* Kernels this library has launched in this process. */
 uint64_t fathom_launch_count(void);
 
-/* Time of the kernel FATHOM_SCAN_PROFILE times (the fetch for a
- * host-resident index, else the main scan), recorded with CUDA events:
+/* Time of what FATHOM_SCAN_PROFILE times (the fetch sequence for a
+ * host-resident index, else the main scan kernel), recorded with CUDA events:
  * synchronises on the recorded events and returns the summed milliseconds
  * and the number of launches timed, then forgets them.  Not thread-safe;
  * benchmarking only. */
