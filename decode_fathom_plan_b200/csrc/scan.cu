@@ -1790,8 +1790,13 @@ cudaError_t side_context(cudaStream_t stream, SideContext **out)
         SideContext c{};
         if ((e = cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking)) != cudaSuccess) return e;
         cudaEvent_t *evs[] = {&c.fork, &c.join, &c.fetched[0], &c.fetched[1], &c.done[0], &c.done[1]};
-        for (cudaEvent_t *ev : evs)
-            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        for (int i = 0; i < 6; ++i) {
+            if ((e = cudaEventCreateWithFlags(evs[i], cudaEventDisableTiming)) != cudaSuccess) {
+                for (int j = 0; j < i; ++j) cudaEventDestroy(*evs[j]);   // nothing half-made stays
+                cudaStreamDestroy(c.side);
+                return e;
+            }
+        }
         it = contexts.emplace(std::make_pair(dev, stream), c).first;
     }
     *out = &it->second;

@@ -100,9 +100,11 @@ typedef enum {
  * while unit u is scored from the other slot.  The workspace therefore holds
  * two units' planes (2 * heads_per_unit * d*4*n_words*4 bytes) plus one
  * unit's scan scratch, not the whole index.  The side stream and its events
- * are created on the first such call for a (device, stream) pair and kept;
- * they fork from and join the caller's stream within the call (event waits
- * only), so a captured call stays a CUDA graph on the caller's stream. */
+ * are created on the first such call for a (device, stream) pair and kept
+ * until the process exits (make that first call before a stream capture,
+ * and make no such call across a cudaDeviceReset); they fork from and join
+ * the caller's stream within the call (event waits only), so a captured
+ * call stays a CUDA graph on the caller's stream. */
 typedef enum {
     FATHOM_RES_DEVICE = 0,
     FATHOM_RES_HOST_MAPPED = 1
