@@ -21,9 +21,9 @@ pytestmark = pytest.mark.gpu
 SCORE_RTOL = 1e-4   # the tolerance of the parity tests
 
 
-def _prepare(seed, budgets, n=20000, H=8, G=4):
+def _prepare(seed, budgets, n=20000, H=8, G=4, residency="device"):
     ses = synth.make_session(seed, H, G, n, budgets)
-    ix = fp.KeyIndex(H, G, n, 128, "device")
+    ix = fp.KeyIndex(H, G, n, 128, residency)
     ix.pack(torch.from_numpy(ses.keys).cuda())
     q = torch.from_numpy(ses.q_bf16.view(np.int16)).cuda()
     b = torch.from_numpy(ses.budgets).cuda()
@@ -54,7 +54,9 @@ def test_static_scratch_matches_workspace_call_twice_in_a_row():
     fp.load_library()
     k = 256
     calls = [(_prepare(301, np.tile([68, 92, 136, 18], 8)), 0),
-             (_prepare(302, np.tile([136, 18, 92, 68], 8)), fp.FATHOM_SCAN_FORCE_EXACT)]
+             (_prepare(302, np.tile([136, 18, 92, 68], 8)), fp.FATHOM_SCAN_FORCE_EXACT),
+             # a small host-resident index: its two-head plane ring fits the scratch too
+             (_prepare(303, np.tile([18, 136, 68, 92], 8), residency="host_mapped"), 0)]
     for (ix, q, t, tu), flags in calls:
         Q = ix.n_kv_heads * ix.group
         ref_i, ref_s = _outputs(Q, k)
