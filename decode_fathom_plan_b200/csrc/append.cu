@@ -66,14 +66,14 @@ append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_
     };
     const float *kc = keys + (size_t)h * m * d + c;   // key j at kc[(j - n) * d]
     if (j_hi - j_lo == 32) {
-        // a whole word: 8 independent loads in flight per round
+        // a whole word: 16 independent loads in flight per round
 #pragma unroll
-        for (int j0 = 0; j0 < 32; j0 += 8) {
-            float x[8];
+        for (int j0 = 0; j0 < 32; j0 += 16) {
+            float x[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = kc[(size_t)(j_lo + j0 + i - n) * d];
+            for (int i = 0; i < 16; ++i) x[i] = kc[(size_t)(j_lo + j0 + i - n) * d];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) take(j_lo + j0 + i, x[i]);
+            for (int i = 0; i < 16; ++i) take(j_lo + j0 + i, x[i]);
         }
     } else {
         for (int j = j_lo; j < j_hi; ++j) take(j, kc[(size_t)(j - n) * d]);
@@ -82,12 +82,19 @@ append_kernel(const float *__restrict__ keys, int H, int n, int m, int d, int n_
 #pragma unroll
     for (int s = 0; s < BITS; ++s)
         if (slot[s]) pw[(size_t)s * n_words] |= slot[s];
-    const unsigned long long o1 = atomicAdd(reinterpret_cast<unsigned long long *>(&s1[hc]), a1);
-    const unsigned long long o2 = atomicAdd(reinterpret_cast<unsigned long long *>(&s2[hc]), a2);
-    // all new keys in one word: this thread is the channel's only writer and
-    // holds its final sums (several words: a second pass recomputes sigma^2)
-    if (words == 1)
+    unsigned long long *p1 = reinterpret_cast<unsigned long long *>(&s1[hc]);
+    unsigned long long *p2 = reinterpret_cast<unsigned long long *>(&s2[hc]);
+    if (words == 1) {
+        // all new keys in one word: this thread is the channel's only writer
+        // and holds its final sums
+        const unsigned long long o1 = atomicAdd(p1, a1), o2 = atomicAdd(p2, a2);
         sigma2[hc] = channel_sigma2((long long)(o1 + a1), (long long)(o2 + a2), sc, n + m);
+    } else {
+        // several words: the sums only accumulate (no value waited for); a
+        // second pass recomputes sigma^2
+        atomicAdd(p1, a1);
+        atomicAdd(p2, a2);
+    }
     if (clamped && n_clamped) atomicAdd(&clamped[hc], n_clamped);
     if (bad) set_status(status, FATHOM_ERR_NONFINITE);
 }
