@@ -92,7 +92,7 @@ struct SessionDesc {
     float *bias_blk;             // grouped scales: [H][nb][G] bias per (head, block, query)
     int block_words;             // grouped scales: plane words per scale block (0: none)
     int nb, n_filled;            // statistics rows per head; blocks holding keys
-    int blk_begin;               // first CTA of this session in block_bias_kernel
+    int blk_begin;               // first of this session's (KV head, block) bias CTAs
     int H, n, n_words, n_cols, col_groups;
     int m_tiles, sample_stride, m_keys, sample_rank, exact_only;
     int chunks, chunk_begin;   // main-scan chunks per KV head, first chunk's CTA
@@ -633,17 +633,18 @@ __device__ __forceinline__ int find_session_by_block(const Batch<NS> &b, int gi)
 }
 
 // ------------------------------------------------ grouped per-block biases
-// One CTA per (session, KV head, scale block holding keys): the bias of
-// each query head of the KV head with that block's scales,
+// The CTA of (session, KV head, scale block holding keys) number gi: the
+// bias of each query head of the KV head with that block's scales,
 //   bias_g = sum_c q_gc * (mn_bc + scale_bc * (2^(4-t)-1)/2),
 // t the query's depth clamped to the union, summed exactly as setup_head
-// sums the bias of a one-block index (fp64 terms, warp shuffles, warps in
-// order).  Thread c handles channel c.
+// sums the bias of a one-block index (fp64 terms, warp shuffles, the first
+// kScanThreads / 32 warps in order).  Thread c handles channel c; a CTA of
+// more threads leaves the rest idle.  Runs as extra CTAs of the threshold
+// launch, for the scan and the exact path.
 template <int NS>
-__global__ void __launch_bounds__(kScanThreads) block_bias_kernel(const __grid_constant__ Batch<NS> b)
+__device__ void block_bias_cta(const Batch<NS> &b, int gi)
 {
     __shared__ double part[kScanThreads / 32][kMaxGroup];
-    const int gi = blockIdx.x;
     const SessionDesc &S = b.s[find_session_by_block(b, gi)];
     const int local = gi - S.blk_begin;
     const int h = local / S.n_filled, blk = local - h * S.n_filled;
@@ -667,7 +668,7 @@ __global__ void __launch_bounds__(kScanThreads) block_bias_kernel(const __grid_c
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
-        if (lane == 0) part[warp][g] = term;
+        if (lane == 0 && warp < kScanThreads / 32) part[warp][g] = term;
     }
     __syncthreads();
     if (c < G) {
@@ -1014,7 +1015,7 @@ constexpr int kThetaBufs = 3;   // stages in flight
 template <int NS, int GP, bool kBlocked>
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_constant__ Batch<NS> b,
                                                                 uint32_t force_exact,
-                                                                int total_queries)
+                                                                int total_queries, int table_ctas)
 {
     extern __shared__ __align__(16) uint32_t th_dyn[];
     __shared__ ScanMeta<GP> sm;
@@ -1027,9 +1028,16 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     // grouped scales: the weights and bias of the pass's tiles' blocks
     __shared__ float tile_w[kBlocked ? kThetaTilesPerPass : 1][kBlocked ? kMaxHeadDim : 1];
     __shared__ float tile_bias[kThetaTilesPerPass];
+    __shared__ float tile_bias_part[kBlocked ? kSelThreads / 32 : 1][kThetaTilesPerPass];
     ThetaBuf stage = reinterpret_cast<ThetaBuf>(th_dyn);
     uint32_t *vals = th_dyn + kThetaBufs * kStageRows * kThetaCols;
     const int G = b.G, d = b.d;
+    if constexpr (kBlocked) {
+        if (blockIdx.x >= total_queries + table_ctas) {   // a (KV head, block)'s biases
+            block_bias_cta(b, blockIdx.x - total_queries - table_ctas);
+            return;
+        }
+    }
     if (blockIdx.x >= total_queries) {   // a KV head's tables for the filtering pass
         const int gh = blockIdx.x - total_queries;
         const SessionDesc &S = b.s[find_session_by_head(b, gh)];
@@ -1145,13 +1153,37 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
                         own_w[j], S.scale[((size_t)h * S.nb + blk) * d + own_c[j]]);
                 }
             }
-            if (threadIdx.x < pass_tiles) {
-                const int tile = t0 + threadIdx.x;
-                const int wcol = tile * S.sample_stride * kTileCols;
-                tile_bias[threadIdx.x] =
-                    (tile < S.m_tiles && wcol < S.n_cols)
-                        ? S.bias_blk[((size_t)h * S.nb + wcol / S.block_words) * G + (qq - h * G)]
-                        : 0.0f;
+            // and the query's bias with each tile's block scales, summed here
+            // in float (the threshold only sizes the candidate set; the scan
+            // uses the biases the bias CTAs of this launch write)
+            {
+                const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+                float qf = 0.0f;
+                int tq = 0;
+                if (c < d) {
+                    qf = bf16_to_float(S.q[(size_t)qq * d + c]);
+                    tq = min((int)S.t[(size_t)qq * d + c], min((int)S.tu[h * d + c], kBits));
+                }
+                for (int tsub = 0; tsub < pass_tiles; ++tsub) {
+                    const int tile = t0 + tsub;
+                    const int wcol = tile * S.sample_stride * kTileCols;
+                    float term = 0.0f;
+                    if (c < d && tile < S.m_tiles && wcol < S.n_cols) {
+                        const size_t e = ((size_t)h * S.nb + wcol / S.block_words) * d + c;
+                        term = qf * (S.mn[e] + S.scale[e] * (float)bin_offset(tq));
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        term += __shfl_xor_sync(0xFFFFFFFFu, term, off);
+                    if (lane == 0) tile_bias_part[warp][tsub] = term;
+                }
+                __syncthreads();
+                if (c < pass_tiles) {
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < kSelThreads / 32; ++w) acc += tile_bias_part[w][c];
+                    tile_bias[c] = acc;
+                }
             }
             __syncthreads();
         }
@@ -1535,12 +1567,6 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
     cudaError_t e;
     const bool force = (flags & FATHOM_SCAN_FORCE_EXACT) != 0;
     int launches = 0;
-    if (kBlocked) {
-        // grouped scales: the bias of every (KV head, block, query head)
-        block_bias_kernel<NS><<<total_blocks, kScanThreads, 0, stream>>>(bt);
-        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "block bias launch");
-        ++launches;
-    }
     {
         // per-head tables, sampled scores and theta per query (or the
         // exact-path flags)
@@ -1553,9 +1579,12 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
             cudaSuccess)
             return note_error(e, "threshold set-up");
         // one CTA per query, then (unless the exact path is forced) one per
-        // KV head building its tables
-        const int ctas = total_queries + (force ? 0 : total_heads);
-        kern<<<ctas, kSelThreads, dyn, stream>>>(bt, force ? 1u : 0u, total_queries);
+        // KV head building its tables, then with grouped scales one per
+        // (KV head, block) writing its biases (the scan and the exact path
+        // read them)
+        const int table_ctas = force ? 0 : total_heads;
+        const int ctas = total_queries + table_ctas + (kBlocked ? total_blocks : 0);
+        kern<<<ctas, kSelThreads, dyn, stream>>>(bt, force ? 1u : 0u, total_queries, table_ctas);
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "threshold launch");
         ++launches;
     }

@@ -266,9 +266,9 @@ size_t fathom_scan_workspace_bytes(const fathom_index *index, int32_t k);
  * (9*H + 3*Q)*2d bytes of workspace (each array rounded up to 16 bytes) for
  * the nibble-channel arguments.
  * All sessions of a batched call have the same b.
- * Grouped scales: key j is scored with mn and scale of its block; one more
- * small launch computes each (KV head, block, query head) bias, and the
- * workspace holds those H*n_blocks*G floats.  All sessions of a batched
+ * Grouped scales: key j is scored with mn and scale of its block; extra
+ * CTAs of the call's threshold launch compute each (KV head, block, query
+ * head) bias, and the workspace holds those H*n_blocks*G floats.  All sessions of a batched
  * call have grouped scales or none have.
  * q_bf16, t, t_union, out_idx, out_score, workspace: device pointers.
  * flags: FATHOM_SCAN_* bits. */
