@@ -31,7 +31,6 @@ FATHOM_RES_HOST_MAPPED = 1
 FATHOM_SCAN_DEFAULT = 0
 FATHOM_SCAN_FORCE_EXACT = 1
 FATHOM_SCAN_PROFILE = 2
-FATHOM_SCAN_TENSOR_CORES = 4
 
 EXPORTED = (
     "fathom_n_words", "fathom_status_str", "fathom_pack_workspace_bytes", "fathom_pack_keys",

@@ -170,8 +170,7 @@ fathom_status scan_common(const fathom_index *sessions, int n_sessions,
 {
     if (!sessions || n_sessions < 1 || n_sessions > kMaxSessions) return FATHOM_ERR_INVALID_ARG;
     if (!q || !t || !tu || !out_idx || !out_score) return FATHOM_ERR_INVALID_ARG;
-    if (flags & ~(FATHOM_SCAN_FORCE_EXACT | FATHOM_SCAN_PROFILE | FATHOM_SCAN_TENSOR_CORES))
-        return FATHOM_ERR_INVALID_ARG;
+    if (flags & ~(FATHOM_SCAN_FORCE_EXACT | FATHOM_SCAN_PROFILE)) return FATHOM_ERR_INVALID_ARG;
     if (k < 1 || k > kMaxK) return FATHOM_ERR_INVALID_ARG;
     std::vector<fathom_index> resolved(n_sessions);
     std::vector<ScanSessionArgs> args(n_sessions);

@@ -34,9 +34,7 @@
 // chunk of a KV head; host-resident planes are fetched a unit of KV heads at
 // a time into a two-slot device ring (fetch.cu) and read from there.
 //
-// The same filtering pass can run on the tensor cores (scan_tc.cuh, flag
-// FATHOM_SCAN_TENSOR_CORES): the union-channel sum as an int8 matrix product
-// of the keys' codes and the weights' base-256 digits.
+// No tensor cores: this is a sparse binary-weighted reduction.
 //
 // Selection without materialising n scores per query:
 //   1. threshold: per query, score evenly strided whole tiles (4096 to 8192
@@ -105,7 +103,6 @@ struct SessionDesc {
 template <int NS>
 struct Batch {
     int n_sessions, G, d, k, cap, kpad;
-    int tc;   // filtering pass on the tensor cores (scan_tc_kernel and its tables)
     SessionDesc s[NS];
 };
 
@@ -811,8 +808,6 @@ scan_kernel(const __grid_constant__ Batch<NS> b)
     }
 }
 
-#include "scan_tc.cuh"
-
 // ------------------------------------------------------- radix selection
 // Warp 0 finds, in a 256-bin histogram, the bin holding the krem-th largest
 // element: above = elements in higher bins < krem <= above + hist[bin].
@@ -1049,12 +1044,6 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
         const int h = gh - S.head_begin;
         setup_head<GP>(sm, h, G, d, S.tu + h * d, S.t + (size_t)h * G * d, S.q + (size_t)h * G * d,
                        kBlocked ? nullptr : S.mn + h * d, kBlocked ? nullptr : S.scale + h * d);
-        if constexpr (!kBlocked && GP <= kTcMaxGroup) {
-            if (b.tc) {
-                build_tc_table<GP>(sm, G, reinterpret_cast<TcMeta *>(S.tables) + h, ss);
-                return;
-            }
-        }
         constexpr int kUnits = (int)(sizeof(ScanMeta<GP>) / 16);
         const uint4 *src = reinterpret_cast<const uint4 *>(&sm);
         uint4 *dst = reinterpret_cast<uint4 *>(S.tables + (size_t)h * sizeof(ScanMeta<GP>));
@@ -1487,14 +1476,12 @@ struct WsLayout {
 
 // Query heads per KV head rounded up to the kernels' template width.
 inline int gp_for(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
-// Bytes of one KV head's scan tables: the CUDA-core scan's, or (up to 4
-// query heads) the tensor-core scan's, whichever is larger.
 inline size_t head_table_bytes(int G)
 {
     switch (gp_for(G)) {
-    case 1: return std::max(sizeof(ScanMeta<1>), sizeof(TcMeta));
-    case 2: return std::max(sizeof(ScanMeta<2>), sizeof(TcMeta));
-    case 4: return std::max(sizeof(ScanMeta<4>), sizeof(TcMeta));
+    case 1: return sizeof(ScanMeta<1>);
+    case 2: return sizeof(ScanMeta<2>);
+    case 4: return sizeof(ScanMeta<4>);
     default: return sizeof(ScanMeta<8>);
     }
 }
@@ -1601,22 +1588,7 @@ cudaError_t run_batch(const Batch<NS> &bt, int total_chunks, int total_queries, 
         if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "threshold launch");
         ++launches;
     }
-    if (!force && total_chunks > 0 && bt.tc) {
-        // filtering pass on the tensor cores
-        const bool timed = hook && hook->enabled;
-        static int tc_smem_set[64];
-        auto kern = scan_tc_kernel<NS>;
-        if ((e = ensure_smem(tc_smem_set, kern, tc_smem_bytes(kMaxHeadDim))) != cudaSuccess)
-            return note_error(e, "scan set-up");
-        if (timed) record_timing_event(hook->begin, stream);
-        kern<<<total_chunks, kScanThreads, tc_smem_bytes(bt.d), stream>>>(bt);
-        if ((e = cudaGetLastError()) != cudaSuccess) return note_error(e, "scan launch");
-        if (timed) {
-            record_timing_event(hook->end, stream);
-            hook->recorded = true;
-        }
-        ++launches;
-    } else if (!force && total_chunks > 0) {
+    if (!force && total_chunks > 0) {
         const bool timed = hook && hook->enabled;
         static int main_smem_set[64];
         auto kern = scan_kernel<NS, GP, kMainStages, kBlocked>;
@@ -1663,12 +1635,6 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     bt.k = k;
     bt.cap = capacity_for(std::min(k, kMaxFastK));
     bt.kpad = next_pow2(k);
-    // the tensor-core filtering pass when asked for: one scale per channel,
-    // up to 4 query heads per KV head
-    bool tc = bt.G <= kTcMaxGroup && (flags & FATHOM_SCAN_TENSOR_CORES);
-    for (int s = 0; s < n_sessions; ++s)
-        if (ss[s].ix->block_keys) tc = false;
-    bt.tc = tc ? 1 : 0;
     int groups = 0, queries = 0, heads = 0, blocks = 0, max_m = 0;
     size_t at = 0;
     char *base = static_cast<char *>(ws);
@@ -1706,7 +1672,6 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
         D.sample_rank = z.rank;
         D.exact_only = z.exact_only;
         D.chunks = (D.col_groups + kTileGroups - 1) / kTileGroups;   // chunks of <= 64 words
-        if (tc) D.chunks = ceil_div(D.col_groups, kTcWords / 4);       // <= 32 words
         if (ix.block_keys)   // the same number of chunks in every scale block
             D.chunks = D.n_filled * ceil_div(D.block_words / 4, kTileGroups);
         D.q_begin = queries;
@@ -1720,22 +1685,7 @@ cudaError_t build_and_run(const ScanSessionArgs *ss, int n_sessions, int k, void
     // least kMinChunkGroups groups each) so the grid fills the slots evenly;
     // a chunk never spans two heads.
     const int slots = sm_count() * ((bt.G > 4) ? 2 : 4);
-    if (tc) {
-        // whole waves of 2 CTAs per SM: more, smaller chunks (at least
-        // kTcMinGroups column groups) up to the next multiple of the slots
-        const int tc_slots = sm_count() * 2;
-        const int target = ceil_div(groups, tc_slots) * tc_slots;
-        if (groups > 0 && groups < target) {
-            const double grow = (double)target / (double)groups;
-            groups = 0;
-            for (int s = 0; s < n_sessions; ++s) {
-                SessionDesc &D = bt.s[s];
-                const int most = std::max(1, D.col_groups / kTcMinGroups);
-                D.chunks = std::max(D.chunks, std::min(most, (int)std::ceil(D.chunks * grow)));
-                groups += D.H * D.chunks;
-            }
-        }
-    } else if (groups < slots) {
+    if (groups < slots) {
         const double grow = (double)slots / (double)groups;
         groups = 0;
         for (int s = 0; s < n_sessions; ++s) {

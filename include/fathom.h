@@ -143,15 +143,6 @@ typedef struct {
  * fetch to the end of the last one's, on the side stream), else the main
  * scan kernel. */
 #define FATHOM_SCAN_PROFILE 2u
-/* Run the filtering pass on the tensor cores (int8 tcgen05 MMAs) instead of
- * the CUDA cores (fp32 fused multiply-adds of the rebuilt codes); honoured
- * for an index with one scale per channel and at most 4 query heads per KV
- * head, ignored otherwise.  Every channel weight W_gc = q_gc*scale_c is
- * scaled by the power of two 2^(29-e_g) (2^e_g > max_c |W_gc|) and rounded
- * to an integer, so a filtering score differs from the fp32 one by at most
- * 15*C*2^(e_g-30) (C <= 4d columns) plus fp32 rounding.  Either way the final
- * top-k is exact over the candidates' scores. */
-#define FATHOM_SCAN_TENSOR_CORES 4u
 
 /* Words per plane for n keys: n rounded up to 128 keys, i.e. 16-byte rows. */
 int32_t fathom_n_words(int32_t n_keys);

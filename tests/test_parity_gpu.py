@@ -164,12 +164,10 @@ def test_scan_tiny_4k(flags):
     assert len(set(ses.planted[0].tolist()) & set(oi[0].tolist())) >= 12
 
 
-@pytest.mark.parametrize("flags", [0, fp.FATHOM_SCAN_FORCE_EXACT, fp.FATHOM_SCAN_TENSOR_CORES])
+@pytest.mark.parametrize("flags", [0, fp.FATHOM_SCAN_FORCE_EXACT])
 def test_scan_layer_ragged_sampled_path(flags):
     """8 KV heads x 4 query heads, 20000 keys (ragged last tile), budgets
-    mixed inside each GQA group, k = 256: the sampled-threshold path with the
-    filtering pass on the CUDA cores (default) and on the tensor cores, and
-    the exact path."""
+    mixed inside each GQA group, k = 256: the sampled-threshold path."""
     budgets = np.tile(np.array([68, 92, 136, 18], np.int32), 8)
     ses = synth.make_session(31, 8, 4, 20000, budgets)
     ix = gpu_index(ses)
@@ -183,18 +181,17 @@ def test_scan_layer_ragged_sampled_path(flags):
                                        (2, 64, 1000, 7, 40), (3, 128, 9000, 100, 92),
                                        (8, 32, 5000, 64, 50), (8, 256, 9001, 512, 300),
                                        (4, 128, 40000, 2048, 136), (2, 128, 6000, 3000, 68)])
-@pytest.mark.parametrize("flags", [0, fp.FATHOM_SCAN_TENSOR_CORES])
-def test_scan_shapes(G, d, n, k, B, flags):
+def test_scan_shapes(G, d, n, k, B):
     H = 2
     ses = synth.make_session(50 + n + G, H, G, n, B, head_dim=d)
     ix = gpu_index(ses)
     ref = oracle.build_index(ses.keys)
     q, t, tu, _ = run_plan(ix, ses, ses.budgets)
-    oi, os_ = run_scan(ix, ses, q, t, tu, k, flags)
+    oi, os_ = run_scan(ix, ses, q, t, tu, k)
     check_scan(ses, ref, t, oi, os_, k)
 
 
-@pytest.mark.parametrize("flags", [0, fp.FATHOM_SCAN_FORCE_EXACT, fp.FATHOM_SCAN_TENSOR_CORES])
+@pytest.mark.parametrize("flags", [0, fp.FATHOM_SCAN_FORCE_EXACT])
 def test_scan_exact_ties_resolve_to_lower_index(flags):
     """B = 4: one channel read at 4 bits -> at most 16 distinct scores, equal
     on both sides bit for bit; the top-k must be the oracle's exactly.
