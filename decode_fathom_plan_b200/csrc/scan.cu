@@ -1378,40 +1378,55 @@ __global__ void __launch_bounds__(kSelThreads) final_kernel(const __grid_constan
     unsigned long long *x = dyn + kMaxFastK;        // [cap] candidates, then the emit scratch
     const unsigned long long *cq = S.cand + (size_t)qq * b.cap;
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (unsigned i = 2 * threadIdx.x; i < cnt; i += 2 * kSelThreads) {
-        unsigned long long v0, v1 = 0ull;
-        if (i + 1 < cnt) {
-            const ulonglong2 p = *reinterpret_cast<const ulonglong2 *>(cq + i);
-            v0 = p.x;
-            v1 = p.y;
-            x[i + 1] = v1;
-            lo = min(lo, (uint32_t)(v1 >> 32));
-            hi = max(hi, (uint32_t)(v1 >> 32));
-        } else {
-            v0 = cq[i];
+    // 16-byte loads, kLoadDepth in flight per thread before any is used
+    constexpr int kLoadDepth = 4;
+    for (unsigned i0 = 2 * threadIdx.x; i0 < cnt; i0 += 2 * kSelThreads * kLoadDepth) {
+        ulonglong2 p[kLoadDepth];
+#pragma unroll
+        for (int u = 0; u < kLoadDepth; ++u) {
+            const unsigned i = i0 + u * 2 * kSelThreads;
+            p[u] = make_ulonglong2(0ull, 0ull);
+            if (i + 1 < cnt) p[u] = *reinterpret_cast<const ulonglong2 *>(cq + i);
+            else if (i < cnt) p[u].x = cq[i];
         }
-        x[i] = v0;
-        lo = min(lo, (uint32_t)(v0 >> 32));
-        hi = max(hi, (uint32_t)(v0 >> 32));
+#pragma unroll
+        for (int u = 0; u < kLoadDepth; ++u) {
+            const unsigned i = i0 + u * 2 * kSelThreads;
+            if (i < cnt) {
+                x[i] = p[u].x;
+                lo = min(lo, (uint32_t)(p[u].x >> 32));
+                hi = max(hi, (uint32_t)(p[u].x >> 32));
+            }
+            if (i + 1 < cnt) {
+                x[i + 1] = p[u].y;
+                lo = min(lo, (uint32_t)(p[u].y >> 32));
+                hi = max(hi, (uint32_t)(p[u].y >> 32));
+            }
+        }
     }
     sel_range(ss, lo, hi);
     const unsigned long long base = (unsigned long long)ss.lo << 32;
     const int top = 32 + bit_length(ss.hi - ss.lo);
     sel_run(ss, cnt, (unsigned)k, top, 0, [&](unsigned i) { return x[i] - base; });
-    // compact exactly the k selected, in candidate order (block scan)
+    // compact exactly the k selected in any order (the emit sorts them by
+    // key index): one shared-memory reservation per warp and round
     const int cut = ss.cut;
     const unsigned long long lim = ss.prefix >> cut;
-    const unsigned per = (cnt + kSelThreads - 1) / kSelThreads;
-    const unsigned i0 = threadIdx.x * per, i1 = min(cnt, i0 + per);
-    unsigned mine = 0;
-    for (unsigned i = i0; i < i1; ++i) mine += ((x[i] - base) >> cut) >= lim;
-    unsigned total;
-    unsigned pos = block_exclusive_scan(mine, ss.wsum, &total);
-    for (unsigned i = i0; i < i1; ++i) {
-        const unsigned long long v = x[i];
-        if (((v - base) >> cut) >= lim) {
-            if (pos < (unsigned)k) sel[pos] = v;
-            ++pos;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) ss.above = 0u;   // the selected count so far
+    __syncthreads();
+    for (unsigned r0 = 0; r0 < cnt; r0 += kSelThreads) {
+        const unsigned i = r0 + threadIdx.x;
+        const unsigned long long v = (i < cnt) ? x[i] : 0ull;
+        const bool take = i < cnt && ((v - base) >> cut) >= lim;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+        if (m) {
+            const int leader = __ffs(m) - 1;
+            unsigned at = 0;
+            if (lane == leader) at = atomicAdd(&ss.above, (unsigned)__popc(m));
+            at = __shfl_sync(0xFFFFFFFFu, at, leader);
+            const unsigned pos = at + (unsigned)__popc(m & ((1u << lane) - 1u));
+            if (take && pos < (unsigned)k) sel[pos] = v;
         }
     }
     __syncthreads();
