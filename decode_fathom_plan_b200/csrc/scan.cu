@@ -1115,26 +1115,38 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
     magic_negatives(neg);
     const float bias = bias_s;
     const size_t head_row0 = (size_t)h * d * kBits;
-    // copy stage s of tile pass t0 into buffer bufi: plane rows of own
-    // channels 8s..8s+7 (4 slots each, zeros past the channel's depth),
-    // pass_tiles tiles x 16 column groups per row
-    auto load = [&](int t0, int s, int bufi) {
-        const int groups = pass_tiles * (kTileCols / 4);
-        for (int e = threadIdx.x; e < kStageRows * groups; e += kSelThreads) {
-            const int row = e / groups, part = e - row * groups;
-            const int tsub = part / (kTileCols / 4), c16 = part - tsub * (kTileCols / 4);
-            const int tile = t0 + tsub;
-            const int j = s * kStageChannels + row / kBits, slot = row % kBits;
-            const int wcol = tile * S.sample_stride * kTileCols + c16 * 4;
-            const bool live = j < n_own && slot < own_t[min(j, kMaxHeadDim - 1)] &&
-                              tile < S.m_tiles && wcol < S.n_cols;
-            const size_t grow = live ? head_row0 + (size_t)own_c[j] * kBits + slot : 0;
-            copy_or_zero16(&stage[bufi][row][part * 4], S.planes + grow * (size_t)S.n_words + wcol,
-                           live);
+    // A stage: plane rows of own channels 8s..8s+7 (4 slots each, zeros past
+    // the channel's depth), pass_tiles tiles x 16 column groups per row.
+    // Thread copies e = tid + i*kSelThreads: row e >> lg_groups, 16-byte
+    // group e & (groups - 1); the part that does not depend on the stage is
+    // worked out once per pass.
+    constexpr int kLoadIters = kStageRows * kThetaCols / 4 / kSelThreads;   // 4
+    const int lg_groups = (pass_tiles == kThetaTilesPerPass) ? 6 : 5;       // 16 * pass_tiles
+    const int n_copies = kStageRows << lg_groups;
+    int l_wcol[kLoadIters];   // source column of copy i; -1: past the sample
+    auto load = [&](int s, int bufi) {
+#pragma unroll
+        for (int i = 0; i < kLoadIters; ++i) {
+            const int e = threadIdx.x + i * kSelThreads;
+            if (e < n_copies) {
+                const int row = e >> lg_groups, part = e & ((1 << lg_groups) - 1);
+                const int j = s * kStageChannels + (row >> 2), slot = row & 3;
+                const bool live = l_wcol[i] >= 0 && j < n_own && slot < own_t[min(j, kMaxHeadDim - 1)];
+                const size_t grow = live ? head_row0 + (size_t)own_c[j] * kBits + slot : 0;
+                copy_or_zero16(&stage[bufi][row][part * 4],
+                               S.planes + grow * (size_t)S.n_words + max(l_wcol[i], 0), live);
+            }
         }
         cp_async_commit();
     };
     for (int t0 = 0; t0 < S.m_tiles; t0 += pass_tiles) {
+#pragma unroll
+        for (int i = 0; i < kLoadIters; ++i) {
+            const int part = (threadIdx.x + i * kSelThreads) & ((1 << lg_groups) - 1);
+            const int tile = t0 + (part >> 4);
+            const int wcol = tile * S.sample_stride * kTileCols + (part & 15) * 4;
+            l_wcol[i] = (tile < S.m_tiles && wcol < S.n_cols) ? wcol : -1;
+        }
         float2 acc[2][4];
 #pragma unroll
         for (int k2 = 0; k2 < 2; ++k2)
@@ -1187,11 +1199,11 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const __grid_con
             }
             __syncthreads();
         }
-        for (int s2 = 0; s2 < kThetaBufs - 1 && s2 < n_stages; ++s2) load(t0, s2, s2);
+        for (int s2 = 0; s2 < kThetaBufs - 1 && s2 < n_stages; ++s2) load(s2, s2);
         for (int s2 = 0; s2 < n_stages; ++s2) {
             // stage s2 has landed once at most (stages issued after it) groups are pending
             if (s2 + kThetaBufs - 1 < n_stages) {
-                load(t0, s2 + kThetaBufs - 1, (s2 + kThetaBufs - 1) % kThetaBufs);
+                load(s2 + kThetaBufs - 1, (s2 + kThetaBufs - 1) % kThetaBufs);
                 cp_async_wait<kThetaBufs - 1>();
             } else if (s2 + 1 < n_stages) {
                 cp_async_wait<1>();
