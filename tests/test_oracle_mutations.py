@@ -72,6 +72,22 @@ MUTATIONS = {
         "            if (tc < 0 || tc > bits) return FO_ERR_ARG;\n            int u = 0;\n"
         "            for (int slot = 0; slot < bits; ++slot) {"),
     "exact_scores_transposed_keys": ("(double)keys_h[j * d + c]", "(double)keys_h[c * n + j]"),
+    "plan_ties_to_higher_channel": ("return (a->c < b->c) ? -1 : (a->c > b->c);",
+                                    "return (a->c > b->c) ? -1 : (a->c < b->c);"),
+    "plan_leftover_skips_zero_importance": ("        if (left > 0) {\n            take = left < bits",
+                                            "        if (left > 0 && order[i].key > 0.0f) {\n"
+                                            "            take = left < bits"),
+    "bytes_per_plane_in_words": ("(uint64_t)t[c] * (uint64_t)n_words * 4u", "(uint64_t)t[c] * (uint64_t)n_words"),
+    "variance_over_n_minus_1": ("double nn = (double)n * (double)n;",
+                                "double nn = (double)n * (double)(n - 1);"),
+    "score_skips_zero_depth_channels": (
+        "            acc += (double)bf16_value(q_bf16[c]) *\n                   fo_coarse_midpoint",
+        "            if (tc > 0) acc += (double)bf16_value(q_bf16[c]) *\n                   fo_coarse_midpoint"),
+    "importance_ignores_variance": ("float wc = qq * sigma2[c];", "float wc = qq;"),
+    "marginal_gain_ties_to_higher_channel": ("if (best < 0 || gain > best_gain) {",
+                                             "if (best < 0 || gain >= best_gain) {"),
+    "topk_keeps_lowest_scores": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
+                                 "if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
 }
 
 PIN_TESTS = [
@@ -81,6 +97,7 @@ PIN_TESTS = [
     lambda: pins.test_plane_layout_hand_worked(read_golden),
     pins.test_importance_values,
     lambda: pins.test_plan_hand_worked(read_golden),
+    lambda: pins.test_plan_is_optimal_by_brute_force_small(3),
     lambda: pins.test_fixed_plan_hand_worked(read_golden),
     pins.test_union_and_bytes,
     lambda: pins.test_coarse_bin_midpoint_hand_worked(read_golden),

@@ -117,7 +117,7 @@ def test_importance_rejects_nonfinite():
 # ---------------------------------------------------------------------- plan
 def test_plan_hand_worked(golden):
     g = golden("plan_worked.txt")
-    for case in ("case1", "case2", "case3", "case4"):
+    for case in ("case1", "case2", "case3", "case4", "case5"):
         w = _floats(g[case + "_w"]).astype(np.float32)
         t = oracle.plan_greedy(w, int(g[case + "_B"][0]))
         assert np.array_equal(t, _ints(g[case + "_t"])), case
