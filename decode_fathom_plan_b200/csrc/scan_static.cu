@@ -13,9 +13,10 @@
 // on every device that loads this library and kept until the process exits.
 // Host code may not pass the array's name to a kernel (on the host it is a
 // stand-in, not a device address), so every call looks up the device address
-// with cudaGetSymbolAddress while the call's device is current.  Looking it up
-// each time (instead of caching it) keeps the address right after a
-// cudaDeviceReset or a new context on that device, which reloads the module.
+// with cudaGetSymbolAddress while the call's device is current (a call costs
+// little next to the scan's launches, and nothing here goes stale).  The rest
+// of the library still keeps per-device state for the life of the process,
+// so no call may follow a cudaDeviceReset of the device.
 #include "common.cuh"
 #include "internal.h"
 

@@ -28,6 +28,11 @@
  *     or host memory; scratch space is a caller-supplied workspace sized by
  *     the matching *_workspace_bytes call (16-byte aligned).  The one
  *     exception is the fixed scratch array behind fathom_scan_topk_static.
+ *   - Per-device state is set up on the first call that needs it and kept
+ *     until the process exits: the status word's address, the raised
+ *     shared-memory limits of the kernels, and the side stream of
+ *     host-resident scans.  A cudaDeviceReset discards what it refers to, so
+ *     make no call on a device after resetting it in the same process.
  *   - Calls are stream-ordered and asynchronous: they validate what the host
  *     can see, enqueue kernels on `stream` and return.  Argument errors are
  *     returned at once and enqueue nothing.  Errors that only the device can
@@ -293,10 +298,11 @@ fathom_status fathom_scan_topk(const fathom_index *index, const uint16_t *q_bf16
  *     keys with k <= 2048 needs 6.3 MiB; a host-resident index also needs
  *     room for its two-slot plane ring, so only small ones fit.
  *   - Every call looks up the scratch array's device address
- *     (cudaGetSymbolAddress) on the current device, so the address stays
- *     right after a device reset.  The first call on a device may also load
- *     the library's device code there; make that first call before any
- *     stream capture.
+ *     (cudaGetSymbolAddress) on the current device instead of caching it.
+ *     The first call on a device may also load the library's device code
+ *     there; make that first call before any stream capture.  Like every
+ *     call of this library it must not follow a cudaDeviceReset of that
+ *     device (see the conventions above).
  *   - All calls on a device share the one array.  Calls whose kernels overlap
  *     on the GPU (e.g. on two streams at once) race on it: order them.
  *   - Calls or frees no device memory. */
