@@ -4,6 +4,7 @@ import os
 import shutil
 import subprocess
 import tempfile
+import types
 
 import pytest
 
@@ -150,3 +151,57 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
         assert caught >= 1, f"no pin caught mutation {name}"
     finally:
         shutil.rmtree(tmp)
+
+
+# Planted mistakes in the Python side of the oracle (the session-level steps
+# around the C routines: per-head plans, the GQA union, bytes, block ranges,
+# appends of whole blocks, the per-head absolute sum, the error metric).
+PY_MUTATIONS = {
+    "session_plan_reads_another_heads_variance": ("        h = q // group\n", "        h = q % group\n"),
+    "session_union_over_the_wrong_queries": ("union(t[h * group:(h + 1) * group])",
+                                             "union(t[h:h + group])"),
+    "session_head_bytes_from_a_query_plan": ('[plan_bytes(T[h], index["n_words"]) for h in range(H)]',
+                                             '[plan_bytes(t[h], index["n_words"]) for h in range(H)]'),
+    "blocked_index_quantises_the_first_keys_for_every_block": (
+        "quantize(keys[:, j0:j1], bits)", "quantize(keys[:, :j1 - j0], bits)"),
+    "append_blocks_overwrites_the_first_blocks": ("b = (n + i0) // block", "b = i0 // block"),
+    "append_blocks_variance_of_the_old_key_count": ('index["s2"][h], n + m, block)',
+                                                    'index["s2"][h], n, block)'),
+    "head_blocks_use_the_first_blocks_scales": ('index["mn"][h, b], index["scale"][h, b]))',
+                                                'index["mn"][h, 0], index["scale"][h, 0]))'),
+    "score_head_ignores_absolute": ("fn = score_abs_planes if absolute else score_planes",
+                                    "fn = score_planes"),
+    "attention_error_not_relative": ("np.linalg.norm(o - o_exact) / np.linalg.norm(o_exact)",
+                                     "np.linalg.norm(o - o_exact)"),
+    "plane_rows_of_32_keys": ("((n + 127) // 128) * 4", "(n + 31) // 32"),
+}
+
+PY_PIN_TESTS = [
+    pins.test_union_and_bytes,
+    pins.test_plans_of_a_blocked_index_use_its_channel_variance,
+    pins.test_blocked_append_of_whole_blocks_equals_packing_everything,
+    pins.test_blocked_scores_full_zero_and_prefix_depths,
+    pins.test_blocked_sigma2_is_the_variance_of_all_dequantised_keys,
+    pins.test_absolute_scores_bound_the_scores_and_equal_them_when_no_term_is_negative,
+    pins.test_attention_error_metric,
+    lambda: pins.test_planes_round_trip_and_padding(1),
+    pins.test_tiny_workload_planted_keys_rank_high,
+]
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_pins_catch_planted_mistake_in_the_python_oracle(name, monkeypatch):
+    old, new = PY_MUTATIONS[name]
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, "mutation anchor not found once"
+    mutant = types.ModuleType("oracle_mutant")
+    mutant.__file__ = oracle.__file__
+    exec(compile(src.replace(old, new), oracle.__file__, "exec"), mutant.__dict__)
+    monkeypatch.setattr(pins, "oracle", mutant)
+    caught = 0
+    for fn in PY_PIN_TESTS:
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught >= 1, f"no pin caught mutation {name}"

@@ -482,6 +482,8 @@ def test_attention_error_metric():
     o = np.array([1.0, 0.0, 0.0])
     assert oracle.attention_error(o, o) == 0.0
     assert abs(oracle.attention_error(np.array([1.0, 0.5, 0.0]), o) - 0.5) < 1e-15
+    # relative to the exact output's norm: |(0, 0, 2.5)| / |(3, 4, 0)| = 2.5 / 5
+    assert abs(oracle.attention_error(np.array([3.0, 4.0, 2.5]), np.array([3.0, 4.0, 0.0])) - 0.5) < 1e-15
     with pytest.raises(ValueError):
         oracle.attention(np.zeros((4, 2), np.float32), np.zeros((4, 2), np.float32),
                          np.zeros(2, np.uint16), np.array([4]))
@@ -822,3 +824,30 @@ def test_plans_of_a_blocked_index_use_its_channel_variance():
         w = oracle.importance(ses.q_bf16[q], ix["sigma2"][q // 2])
         assert np.array_equal(t[q], oracle.plan_greedy(w, 40))
     assert T.shape == (2, 32) and int(nb[0]) == 40 * oracle.n_words_for(5000) * 4
+
+
+def test_absolute_scores_bound_the_scores_and_equal_them_when_no_term_is_negative():
+    """A_j of a whole head (score_head with absolute=True, the scale of every
+    score tolerance of the parity tests) is the sum of the absolute terms:
+    it bounds |s_j| (triangle inequality), is strictly larger for keys whose
+    terms differ in sign, and equals s_j bit for bit when no term is
+    negative (q >= 0 and every rebuilt key >= 0: the same terms, summed in
+    the same order).  Checked on a one-scale and a block-scaled index."""
+    ses, keys = _drifting_keys(38, 1, 5000, 128, 2048, 1.5)
+    rng = np.random.default_rng(38)
+    t = rng.integers(0, 5, size=128).astype(np.uint8)
+    for block in (0, 2048):
+        ix = oracle.build_index(keys, block_keys=block)
+        q = ses.q_bf16[0]
+        s = oracle.score_head(ix, 0, q, t)
+        a = oracle.score_head(ix, 0, q, t, absolute=True)
+        assert a.shape == s.shape == (5000,)
+        assert np.all(a >= np.abs(s))
+        assert np.count_nonzero(a > np.abs(s)) > 4900        # mixed-sign q: almost every key
+        # non-negative terms: |q| and keys shifted so that every channel's minimum is >= 0
+        q_pos = synth.f32_to_bf16_bits(np.abs(synth.bf16_bits_to_f32(q)))
+        pos = keys - keys.min(axis=1, keepdims=True)
+        ixp = oracle.build_index(pos, block_keys=block)
+        assert np.all(ixp["mn"] >= 0)
+        assert np.array_equal(oracle.score_head(ixp, 0, q_pos, t, absolute=True),
+                              oracle.score_head(ixp, 0, q_pos, t))
